@@ -1,0 +1,289 @@
+"""Pins for the fp64 oracle: facts fixed by the pages or by mathematics.
+
+Each ``pin_*`` takes the oracle module and raises AssertionError when the
+oracle disagrees.  None of them re-types the oracle's own formula: they use
+closed forms, invariants, a different formulation (complex multiplication
+for RoPE, torch's scaled-dot-product attention for the whole attention),
+brute force on tiny inputs, or numbers printed on the pages.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import scipy.special
+import torch
+
+from mla_latent_kv_43_b200 import inputs as gen
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _close(a, b, rtol=1e-12, atol=1e-12):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    assert a.shape == b.shape, (a.shape, b.shape)
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    ref = max(np.max(np.abs(b)) if b.size else 0.0, 1e-300)
+    assert err <= atol + rtol * ref, f"max|d|={err:.3e} max|ref|={ref:.3e}"
+
+
+def _np(t):
+    return t.double().numpy()
+
+
+# --------------------------------------------------------------------- RoPE
+def pin_rope_identity_at_zero(O):
+    """Rotation by angle 0 is the identity (position 0)."""
+    x = np.random.default_rng(1).standard_normal((5, 16))
+    _close(O.rope(x, 0), x, rtol=0, atol=0)
+
+
+def pin_rope_preserves_norm(O):
+    """A rotation preserves every pair's length, hence the vector's norm."""
+    x = np.random.default_rng(2).standard_normal((7, 64))
+    y = O.rope(x, np.arange(7) * 1000 + 3)
+    _close(np.hypot(y[:, 0::2], y[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]), rtol=1e-14)
+
+
+def pin_rope_2d_is_plane_rotation(O):
+    """With d_R = 2, theta_0 = 1: the textbook 2-D rotation by pos radians."""
+    x = np.array([0.3, -1.7])
+    for p in (0, 1, 2, 5, 100, 131071):
+        R = np.array([[math.cos(p), -math.sin(p)], [math.sin(p), math.cos(p)]])
+        _close(O.rope(x, p), R @ x, rtol=1e-14, atol=1e-15)
+
+
+def pin_rope_complex_form(O):
+    """Interleaved pair i as the complex number x[2i] + i x[2i+1], multiplied by
+    exp(i * pos * base^(-2i/d)): the same map written another way."""
+    rng = np.random.default_rng(3)
+    for d in (4, 16, 64):
+        x = rng.standard_normal((6, d))
+        pos = np.array([0, 1, 7, 4095, 4096, 131071])
+        z = x[:, 0::2] + 1j * x[:, 1::2]
+        freq = np.power(10000.0, -np.arange(0, d, 2) / d)
+        zr = z * np.exp(1j * pos[:, None] * freq[None, :])
+        ref = np.empty_like(x)
+        ref[:, 0::2], ref[:, 1::2] = zr.real, zr.imag
+        _close(O.rope(x, pos), ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_rope_relative(O):
+    """(R_m q) . (R_n k) = q^T R_(n-m) k: the score sees only the offset
+    ("Understanding MLA", section 4)."""
+    rng = np.random.default_rng(4)
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    for m, n in ((0, 0), (3, 10), (4097, 12), (100000, 99999)):
+        lhs = O.rope(q, m) @ O.rope(k, n)
+        rhs = q @ O.rope(k, n - m)
+        _close(lhs, rhs, rtol=1e-10, atol=1e-10)
+
+
+# ------------------------------------------------------------ decode checks
+def _tiny_inputs(seed=0, n_q=1, lens=(5, 9), qk_nope=6, v_dim=5, heads=3, d_c=8, d_rope=4):
+    w = gen.tiny("fp32", lens=lens, n_q=n_q, seed=seed, qk_nope=qk_nope, v_dim=v_dim,
+                 heads=heads, d_c=d_c, d_rope=d_rope)
+    return w, gen.generate(w)
+
+
+def _rot_cache(O, inp, lens=None):
+    return O.rope_cache(inp["k_rope"], inp["seq_lens"] if lens is None else lens)
+
+
+def pin_absorbed_equals_naive(O):
+    """Moving W_K to the query side is an exact regrouping ("Understanding MLA",
+    section 4): absorbed and materialised decode agree to rounding."""
+    for n_q in (1, 2):
+        w, inp = _tiny_inputs(seed=5, n_q=n_q, lens=(3, 11))
+        k = _rot_cache(O, inp)
+        a = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                           k, inp["seq_lens"], n_q, w.softmax_scale)
+        b = O.decode_absorbed(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"],
+                              inp["c_kv"], k, inp["seq_lens"], n_q, w.softmax_scale)
+        _close(a, b, rtol=1e-12)
+
+
+def pin_length_one_returns_value(O):
+    """One visible key: softmax weight 1, output = c_0 W_V^(h) for any query."""
+    w, inp = _tiny_inputs(seed=6, lens=(1, 1))
+    out = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                         _rot_cache(O, inp), inp["seq_lens"], 1, w.softmax_scale)
+    c, Wv = _np(inp["c_kv"]), _np(inp["W_uv"])
+    for b in range(2):
+        for h in range(w.heads):
+            ref = [sum(c[b, 0, i] * Wv[h, i, v] for i in range(w.d_c)) for v in range(w.v_dim)]
+            _close(out[b, 0, h], ref, rtol=1e-14)
+
+
+def pin_zero_query_is_uniform_mean(O):
+    """q = 0: all scores 0, uniform weights, output = mean(c_0..c_p) W_V^(h)."""
+    w, inp = _tiny_inputs(seed=7, lens=(4, 9), n_q=2)
+    inp["q_nope"].zero_()
+    inp["q_rope"].zero_()
+    out = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                         _rot_cache(O, inp), inp["seq_lens"], 2, w.softmax_scale)
+    c, Wv = _np(inp["c_kv"]), _np(inp["W_uv"])
+    for b, L in enumerate((4, 9)):
+        for j in range(2):
+            p = L - 2 + j
+            for h in range(w.heads):
+                _close(out[b, j, h], c[b, : p + 1].mean(axis=0) @ Wv[h], rtol=1e-13)
+
+
+def pin_weights_sum_to_one(O):
+    w, inp = _tiny_inputs(seed=8, lens=(6, 13), n_q=2)
+    _, ws = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                           _rot_cache(O, inp), inp["seq_lens"], 2, w.softmax_scale,
+                           return_weights=True)
+    for (b, j, h), wt in ws.items():
+        L = (6, 13)[b]
+        assert wt.shape == (L - 2 + j + 1,), (wt.shape, b, j)
+        assert np.all(wt >= 0)
+        assert abs(wt.sum() - 1.0) < 1e-14
+
+
+def pin_global_shift_invariance(O):
+    """Shifting every position by the same amount leaves the output unchanged
+    (RoPE scores depend on n - m only)."""
+    w, inp = _tiny_inputs(seed=9, lens=(7, 12), n_q=2)
+    k = _rot_cache(O, inp)
+    args = (inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"], k,
+            inp["seq_lens"], 2, w.softmax_scale)
+    _close(O.decode_naive(*args), O.decode_naive(*args, pos_offset=777), rtol=1e-10)
+
+
+def pin_causal(O):
+    """Query j sees keys 0..L-n_q+j: changing the last entry changes only the
+    last query's output."""
+    w, inp = _tiny_inputs(seed=10, lens=(6, 9), n_q=2)
+    k = _rot_cache(O, inp)
+    base = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                          k, inp["seq_lens"], 2, w.softmax_scale)
+    c2 = inp["c_kv"].clone()
+    k2 = k.copy()
+    for b, L in enumerate((6, 9)):
+        c2[b, L - 1] += 3.0
+        k2[b, L - 1] += 2.0
+    mod = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], c2, k2,
+                         inp["seq_lens"], 2, w.softmax_scale)
+    _close(mod[:, 0], base[:, 0], rtol=0, atol=0)
+    assert np.max(np.abs(mod[:, 1] - base[:, 1])) > 1e-3
+
+
+def pin_rope_only_scores_match_scipy_softmax(O):
+    """W_K = 0 leaves only the rope dot in the score; the weights are then
+    scipy's softmax of scale * (R_n k_n) . (R_p q_rope).  The rope key is
+    never up-projected ("Understanding MLA", section 7)."""
+    w, inp = _tiny_inputs(seed=11, lens=(8, 3))
+    inp["W_uk"].zero_()
+    k = _rot_cache(O, inp)
+    out = O.decode_naive(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"],
+                         k, inp["seq_lens"], 1, w.softmax_scale)
+    c, Wv, qr, kraw = _np(inp["c_kv"]), _np(inp["W_uv"]), _np(inp["q_rope"]), _np(inp["k_rope"])
+    for b, L in enumerate((8, 3)):
+        p = L - 1
+        kz = kraw[b, :L, 0::2] + 1j * kraw[b, :L, 1::2]
+        freq = np.power(10000.0, -np.arange(0, w.d_rope, 2) / w.d_rope)
+        kz = kz * np.exp(1j * np.arange(L)[:, None] * freq)
+        for h in range(w.heads):
+            qz = (qr[b, 0, h, 0::2] + 1j * qr[b, 0, h, 1::2]) * np.exp(1j * p * freq)
+            s = (kz.real @ qz.real + kz.imag @ qz.imag) * w.softmax_scale
+            ref = scipy.special.softmax(s) @ (c[b, :L] @ Wv[h])
+            _close(out[b, 0, h], ref, rtol=1e-12)
+
+
+def _torch_rope(x, pos, base=10000.0):
+    """RoPE through torch complex arithmetic (independent of the oracle)."""
+    d = x.shape[-1]
+    z = torch.view_as_complex(x.reshape(*x.shape[:-1], d // 2, 2).contiguous())
+    freq = base ** (-torch.arange(0, d, 2, dtype=torch.float64) / d)
+    ang = pos.to(torch.float64)[..., None] * freq
+    return torch.view_as_real(z * torch.polar(torch.ones_like(ang), ang)).reshape(x.shape)
+
+
+def _torch_reference(w, inp):
+    """Whole decode step written with torch float64 ops and SDPA."""
+    f = lambda k: inp[k].to(torch.float64)
+    c, kr = f("c_kv").clone(), f("k_rope").clone()
+    lens = inp["seq_lens"].long()
+    B = w.batch
+    slots = torch.arange(w.capacity)
+    kr = _torch_rope(kr, slots.expand(B, -1))
+    if w.n_new:
+        y = f("x") @ f("W_dkv")
+        pos = inp["positions"].long()
+        y_r = _torch_rope(y[:, w.d_c:], pos)
+        for r in range(B * w.n_new):
+            b = r // w.n_new
+            c[b, pos[r]] = y[r, : w.d_c]
+            kr[b, pos[r]] = y_r[r]
+    out = torch.zeros(B, w.n_q, w.heads, w.v_dim, dtype=torch.float64)
+    for b in range(B):
+        L = int(lens[b])
+        Kn = torch.einsum("ld,hdk->hlk", c[b, :L], f("W_uk"))
+        V = torch.einsum("ld,hdv->hlv", c[b, :L], f("W_uv"))
+        K = torch.cat([Kn, kr[b, :L].expand(w.heads, L, w.d_rope)], dim=-1)
+        qpos = torch.arange(L - w.n_q, L)
+        qr = _torch_rope(f("q_rope")[b].transpose(0, 1), qpos.expand(w.heads, -1))
+        Q = torch.cat([f("q_nope")[b].transpose(0, 1), qr], dim=-1)        # [H][n_q][192]
+        mask = slots[:L][None, :] <= qpos[:, None]                          # [n_q][L]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            Q, K, V, attn_mask=mask, scale=w.softmax_scale)
+        out[b] = o.transpose(0, 1)
+    return out.numpy()
+
+
+def pin_whole_step_matches_torch_sdpa(O):
+    """The whole step from raw stored inputs (rope keys rotated at their slot,
+    queries at L - n_q + j, causal mask) against torch's SDPA in float64."""
+    for n_q, lens in ((1, (5, 9)), (2, (4, 11)), (3, (3, 6))):
+        w, inp = _tiny_inputs(seed=12 + n_q, lens=lens, n_q=n_q)
+        got = O.decode_step(inp, n_q, w.d_c, w.softmax_scale)
+        _close(got, _torch_reference(w, inp), rtol=1e-11)
+
+
+def pin_step_with_append_matches_torch(O):
+    """Append-then-attend: new rows from x W_DKV, split, rope key rotated at the
+    new positions, then two causal queries (the second sees the first)."""
+    w = gen.tiny("fp32", lens=(6, 9), capacity=10, n_q=2, n_new=2, hidden=12, seed=21)
+    inp = gen.generate(w)
+    got = O.decode_step(inp, 2, w.d_c, w.softmax_scale)
+    _close(got, _torch_reference(w, inp), rtol=1e-11)
+
+
+def pin_append_brute_force(O):
+    """Append rows by explicit loops on a tiny input: latent = first d_c
+    outputs of the one projection, rope key = the last d_R, rotated."""
+    rng = np.random.default_rng(13)
+    M, hidden, d_c, d_r = 3, 5, 4, 4
+    x = rng.standard_normal((M, hidden))
+    W = rng.standard_normal((hidden, d_c + d_r))
+    pos = np.array([0, 5, 4097])
+    rows = O.append_rows(x, W, pos, d_c)
+    for m in range(M):
+        y = [sum(x[m, k] * W[k, n] for k in range(hidden)) for n in range(d_c + d_r)]
+        _close(rows[m, :d_c], y[:d_c], rtol=1e-13)
+        for i in range(d_r // 2):
+            ang = pos[m] * 10000.0 ** (-2 * i / d_r)
+            a, b = y[d_c + 2 * i], y[d_c + 2 * i + 1]
+            _close(rows[m, d_c + 2 * i], a * math.cos(ang) - b * math.sin(ang), rtol=1e-12, atol=1e-13)
+            _close(rows[m, d_c + 2 * i + 1], a * math.sin(ang) + b * math.cos(ang), rtol=1e-12, atol=1e-13)
+
+
+def pin_cache_arithmetic(O):
+    """Per-token storage figures printed on the pages."""
+    g = json.load(open(os.path.join(GOLDEN, "cache_arithmetic.json")))
+    v3, v2 = g["v3"], g["v2"]
+    mla = O.cache_values_per_token(v3["d_c"], v3["d_rope"])
+    mha = O.mha_values_per_token(v3["heads"], v3["qk_dim"], v3["v_dim"])
+    assert mla == v3["mla_values_per_token_layer"]
+    assert mha == v3["mha_values_per_token_layer"]
+    assert round(mha / mla) == v3["ratio_approx"]
+    assert round(mla * 2 * v3["layers"] / 1000) == v3["kb_per_token_approx"]
+    assert O.cache_values_per_token(v2["d_c"], v2["d_rope"]) * v2["layers"] == v2["scalars_per_token"]
+    assert v2["scalars_per_token"] * 2 / 1024 == v2["kb_per_token_fp16"]
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
