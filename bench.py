@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""Benchmark of the MLA absorbed-decode step on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole decode path over one batch: absorption with
+query RoPE, attention against the latent cache, split-KV combine, W_UV
+up-projection (and, for the append workload, the cache append first).  The
+default workload is the batched DeepSeek-V3-shaped decode: B=64 sequences,
+128 heads, latent 512 + rope 64, ragged lengths uniform in [1024, 4096], one
+query token each, bf16, seeded synthetic data.
+
+Timing: W untimed warm-up steps (extended to >= 1.5 s so clocks settle), then
+K steps timed with CUDA events on the launching stream, L2 flushed (512 MiB
+write) before every step outside the timed events; barrier + synchronize on
+both sides, max over ranks.  A second K-step pass with per-kernel events gives
+the dominant kernel's roofline; an end-to-end pass times the same call with
+the step's queries copied from pinned host memory and the output read back.
+With N > 1 every rank runs its own shard of B sequences (weak scaling, no
+collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+import torch.distributed as dist
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_latent_kv_43_b200 import binding as B  # noqa: E402
+from mla_latent_kv_43_b200 import inputs as gen  # noqa: E402
+from mla_latent_kv_43_b200 import roofline as RF  # noqa: E402
+
+METRIC = "MLA decode query-tokens/s; cache GB/s and TFLOP/s as % of B200 roofline"
+DEFAULT_WORKLOAD = "v3_b64_ragged"
+FLUSH_BYTES = 512 << 20
+KERNEL_SOURCES = {  # kernel name prefix -> source file whose hash keys committed ncu traffic
+    "sm100_attend": "mla_latent_kv_43_b200/csrc/sm100_attend.cu",
+    "generic_attend": "mla_latent_kv_43_b200/csrc/generic.cu",
+}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(gen.WORKLOADS))
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        win = [p for t, p in self.samples if t0 <= t <= t1]
+        if len(win) < 3:   # short timed region: include the last seconds of warm-up
+            win = [p for t, p in self.samples if t0 - 2.0 <= t <= t1 + 0.2]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(p[1]) for p in win if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in win if p[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in win for n, v in zip(names, p[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+# ----------------------------------------------------------------- helpers
+def barrier(world):
+    if world > 1:
+        t = torch.ones(1, device="cuda")
+        dist.all_reduce(t)
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def source_sha(path: str) -> str:
+    return hashlib.sha256(open(os.path.join(ROOT, path), "rb").read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel's
+    source has not changed since (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    src = next((s for k, s in KERNEL_SOURCES.items() if kernel.startswith(k)), None)
+    if not e or not src or e.get("source_sha") != source_sha(src):
+        return None
+    return e.get("bytes_per_launch")
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_sample(w, host, budget_s: float):
+    """Time the fp64 oracle on whole sequences (all heads) until the budget is
+    spent; returns (query-tokens/s, description, threads)."""
+    from oracle import mla_oracle as O
+    t0 = time.perf_counter()
+    done = 0
+    for b in range(w.batch):
+        O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=[b])
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"fp64 oracle (naive non-absorbed form), {done} of {w.batch} sequences x all {w.heads} heads "
+            f"x {w.n_q} query token(s), {dt:.1f} s")
+    return done * w.n_q / dt, desc, blas_threads()
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(a, rank, world):
+    if rank != 0:
+        return
+    from oracle import mla_oracle as O
+    w = gen.WORKLOADS[a.workload]
+    host = gen.generate(w)
+    heads = list(range(0, w.heads, max(1, w.heads // 16)))[:16]
+    def one(k):
+        O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=[k % w.batch],
+                      heads=heads)
+    for k in range(a.warmup):
+        one(k)
+    t0 = time.perf_counter()
+    for k in range(a.steps):
+        one(k)
+    dt = time.perf_counter() - t0
+    qtok = a.steps * w.n_q * len(heads) / w.heads
+    value = qtok / dt
+    cores = blas_threads()
+    sample = (f"each step: 1 sequence x {len(heads)} of {w.heads} heads x {w.n_q} query token(s) "
+              f"of {w.name}, fp64 oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "query-tokens/s",
+            "n_gpus": world, "steps": a.steps, "warmup": a.warmup, "ms_per_step": dt / a.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": workload_config(w, host, world),
+            "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, host, world):
+    lens = host["seq_lens"].tolist()
+    return {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world,
+            "n_q": w.n_q, "heads": w.heads, "d_c": w.d_c, "d_rope": w.d_rope, "qk_nope": w.qk_nope,
+            "v_dim": w.v_dim, "seq_len_mean": sum(lens) / len(lens), "seq_len_min": min(lens),
+            "seq_len_max": max(lens), "capacity": w.capacity, "n_new": w.n_new, "hidden": w.hidden,
+            "l2": "flushed before every timed step (512 MiB write, outside the timed events)",
+            "parallelism": f"dp{world} (independent sequence shards)"}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(a, rank, world, local):
+    from mla_latent_kv_43_b200.runner import DeviceProblem
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = gen.WORKLOADS[a.workload]
+    w_rank = w.with_(seed=w.seed + 1000 * rank) if rank else w
+    host = gen.generate(w_rank)
+    stream = torch.cuda.current_stream()
+    prob = DeviceProblem(w_rank, host, device=dev, splits=a.splits)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lens = host["seq_lens"].tolist()
+    work = RF.step_work(w_rank, lens)
+    peaks = RF.load_peaks()
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+
+    # warm-up: at least W steps and at least 1.5 s
+    t_w = time.time()
+    k = 0
+    while k < a.warmup or time.time() - t_w < 1.5:
+        flush.zero_()
+        prob.step()
+        k += 1
+        if k % 64 == 0:
+            torch.cuda.synchronize()
+    st = prob.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {B.STATUS.get(st, st)}")
+
+    # pass A: headline timing
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.steps)]
+    barrier(world)
+    t0 = time.time()
+    launches = 0
+    for s, e in ev:
+        flush.zero_()
+        s.record(stream)
+        launches += prob.step()
+        e.record(stream)
+    barrier(world)
+    t1 = time.time()
+    total_ms = sum(s.elapsed_time(e) for s, e in ev)
+    total_ms = max_over_ranks(total_ms, world)
+
+    # pass B: per-kernel events (dominant kernel roofline)
+    B.mla_profile_enable(True)
+    B.mla_profile_read()
+    barrier(world)
+    for _ in range(a.steps):
+        flush.zero_()
+        prob.step()
+    barrier(world)
+    prof = B.mla_profile_read()
+    B.mla_profile_enable(False)
+
+    # pass C: end to end through the public call with host buffers
+    h_qn = host["q_nope"].pin_memory()
+    h_qr = host["q_rope"].pin_memory()
+    h_len = host["seq_lens"].pin_memory()
+    h_out = torch.empty(prob.out.shape, dtype=prob.out.dtype).pin_memory()
+    h2d = h_qn.numel() * h_qn.element_size() + h_qr.numel() * h_qr.element_size() + h_len.numel() * 4
+    if prob.has_append:
+        h_x = host["x"].pin_memory()
+        h2d += h_x.numel() * h_x.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_ms = 0.0
+    barrier(world)
+    for _ in range(a.steps):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        prob.q_nope.copy_(h_qn, non_blocking=True)
+        prob.q_rope.copy_(h_qr, non_blocking=True)
+        prob.seq_lens.copy_(h_len, non_blocking=True)
+        if prob.has_append:
+            prob.x.copy_(h_x, non_blocking=True)
+        prob.step()
+        h_out.copy_(prob.out, non_blocking=True)
+        e.record(stream)
+        e.synchronize()
+        e2e_ms += s.elapsed_time(e)
+    barrier(world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    st = prob.get_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {B.STATUS.get(st, st)}")
+
+    clocks = sampler.summary(t0, t1) if sampler else None
+    if sampler:
+        sampler.stop()
+    if rank != 0:
+        return
+
+    ms_step = total_ms / a.steps
+    qtok = work["query_tokens"] * world
+    value = qtok / (ms_step * 1e-3)
+    step_s = ms_step * 1e-3
+    # dominant kernel
+    kern = max(prof.items(), key=lambda kv: kv[1][1])
+    kname, (kcount, kms) = kern
+    avg_s = kms / kcount * 1e-3
+    L = prob.layout
+    q_el = 2 if L["compute_dtype"] == 0 else 4
+    kbytes = RF.kernel_bytes(kname, w_rank, lens, q_el, q_el)
+    achieved = kbytes / avg_s / 1e9
+    roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(kname),
+            "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": avg_s * 1e6,
+            "peak_source": peaks["source"]}
+    kernels = {n: {"launches": c, "avg_us": t / c * 1e3, "share": t / sum(v[1] for v in prof.values())}
+               for n, (c, t) in sorted(prof.items())}
+    t_hbm = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_tc = work["flops"] / (peaks["bf16_tflops"] * 1e12)
+    line = {
+        "metric": METRIC, "value": value, "unit": "query-tokens/s", "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded normal draws, DeepSeek-V3 shapes, random weights)",
+        "config": workload_config(w_rank, host, world),
+        "cache_gbs": work["cache_bytes"] / step_s / 1e9,
+        "total_gbs": work["bytes"] / step_s / 1e9,
+        "tflops": work["flops"] / step_s / 1e12,
+        "step_roofline": {"bytes": work["bytes"], "flops": work["flops"], "t_hbm_us": t_hbm * 1e6,
+                          "t_tensor_us": t_tc * 1e6, "frac": max(t_hbm, t_tc) / step_s,
+                          "peaks": f"{peaks['source']}: {peaks['hbm_gbs']} GB/s, {peaks['bf16_tflops']} TFLOP/s"},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "e2e": {"value": qtok / (e2e_ms / a.steps * 1e-3), "unit": "query-tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / a.steps},
+        "clocks": clocks,
+    }
+    if world == 1 and a.cpu_seconds > 0:
+        v, desc, cores = cpu_sample(w_rank, host, a.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "query-tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if a.impl == "reference":
+        run_reference(a, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_ours(a, rank, world, local)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+/*
+ * mla.h -- C ABI of the MLA absorbed-decode library (libmla.so).
+ *
+ * Multi-head Latent Attention caches, per token and layer, one 576-wide entry:
+ * a 512-wide latent c_KV followed by a 64-wide rope key that is already
+ * rotated at the token's position ("Understanding MLA (Multi-head Latent
+ * Attention)", section 5 "What gets cached").  Decode scores every head's
+ * query directly against that cache after moving the key up-projection onto
+ * the query side (same page, section 4), and applies the value up-projection
+ * to the softmax-weighted latent (aicassindra "Multi-head latent attention",
+ * "End-to-end flow").
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked (device) are CUDA device pointers; nothing is copied to
+ *    or from the host except where stated.  The caller allocates every buffer
+ *    (inputs, outputs, workspace, the 4-byte status word); the library
+ *    allocates no memory and keeps no pointer after the call returns.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *    stream.  All work is enqueued on it and the call returns without waiting.
+ *  - Tensors are dense, row-major, in the element type `dims->dtype`
+ *    (MLA_BF16: bfloat16, MLA_FP32: float) unless stated otherwise.
+ *  - Return value: MLA_OK, or an error code for problems found on the host
+ *    before anything is enqueued (nothing runs in that case).  Problems only
+ *    the device can see (a bad length or position) are recorded in the status
+ *    word with an atomic "first error wins" update and never trap; read and
+ *    clear it with mla_get_status.
+ *  - Empty work (batch == 0, n_q == 0, n_new == 0, n_rows == 0) returns MLA_OK
+ *    and enqueues nothing.
+ */
+#ifndef MLA_H
+#define MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum mla_dtype { MLA_BF16 = 0, MLA_FP32 = 1 };
+
+enum mla_status {
+    MLA_OK = 0,
+    MLA_ERR_ARG = 1,          /* null pointer, non-positive or odd size, bad dtype */
+    MLA_ERR_ALIGN = 2,        /* a pointer the kernels load with TMA is not 16-byte aligned */
+    MLA_ERR_WORKSPACE = 3,    /* workspace_bytes below mla_decode_workspace_bytes() */
+    MLA_ERR_UNSUPPORTED = 4,  /* a valid request this build does not implement */
+    MLA_ERR_CUDA = 5,         /* a CUDA launch or API call failed */
+    MLA_ERR_LEN = 6,          /* device: len_b < n_q, len_b > capacity or len_b > max_len */
+    MLA_ERR_POS = 7,          /* device: an append position outside [0, capacity) */
+    MLA_ERR_TIMEOUT = 8       /* device: a bounded wait inside a kernel expired */
+};
+
+/* Model geometry.  The per-head query/key width is qk_nope + d_rope and the
+ * value width is v_dim ("Understanding MLA", Phase C step C1 and Phase D
+ * step D1).  softmax_scale is normally 1/sqrt(qk_nope + d_rope) (Phase D,
+ * step D2); rope_base is the RoPE base (10000). */
+typedef struct {
+    int32_t heads;
+    int32_t d_c;       /* latent width (512 for DeepSeek-V3) */
+    int32_t d_rope;    /* rope key width (64), even */
+    int32_t qk_nope;   /* content part of the query/key (128) */
+    int32_t v_dim;     /* value width per head (128) */
+    int32_t dtype;     /* enum mla_dtype */
+    float softmax_scale;
+    float rope_base;
+} mla_dims;
+
+/* Workspace regions of one mla_decode call (byte offsets from the workspace
+ * base; a size of 0 means the region is not used).  Exposed so tests can
+ * inspect the intermediate results of a call. */
+typedef struct {
+    size_t total;          /* bytes the call needs */
+    size_t q_lat;          /* absorbed queries [B][n_q][H][d_c + d_rope], compute dtype */
+    size_t q_lat_bytes;
+    size_t o_lat;          /* combined latent outputs [B][n_q][H][d_c], compute dtype */
+    size_t o_lat_bytes;
+    size_t part_o;         /* split-KV partial latent outputs, float */
+    size_t part_o_bytes;
+    size_t part_lse;       /* split-KV partial log-sum-exp values, float */
+    size_t part_lse_bytes;
+    size_t sched;          /* device-built work schedule */
+    size_t sched_bytes;
+    int32_t compute_dtype; /* enum mla_dtype of q_lat and o_lat */
+    int32_t splits;        /* key splits per query (generic path) or work items (tensor-core path) */
+} mla_ws_layout;
+
+/* Workspace needed by mla_decode for these sizes (0 on invalid arguments).
+ * max_len is a host-known upper bound on every len_b; splits as in
+ * mla_decode (0 = automatic). */
+MLA_API size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q,
+                                  int64_t max_len, int32_t splits);
+
+/* Same sizes as mla_decode_workspace_bytes, with the region offsets.
+ * Returns MLA_OK or MLA_ERR_ARG. */
+MLA_API int mla_decode_workspace_layout(const mla_dims* dims, int32_t batch, int32_t n_q,
+                                int64_t max_len, int32_t splits, mla_ws_layout* layout);
+
+/* In-place RoPE on strided rows ("Understanding MLA", Phase B step B2 and
+ * Phase C step C2): every interleaved pair (x[2i], x[2i+1]) of row r is
+ * rotated by the angle positions[r] * rope_base^(-2i/d_rope).
+ *   x          (device) first element of row 0; row r starts at x + r*row_stride
+ *              elements; d_rope elements per row are rotated.
+ *   row_stride elements between rows (>= d_rope).
+ *   positions  (device) int32[n_rows], each >= 0.
+ * Used to build a cache's rope keys from raw values (as the append step would
+ * have stored them); the decode and append kernels apply the same rotation
+ * internally. */
+MLA_API int mla_rope(const mla_dims* dims, int64_t n_rows, void* x, int64_t row_stride,
+             const int32_t* positions, void* stream);
+
+/* Append n_new tokens to each of `batch` sequences (aicassindra "Multi-head
+ * latent attention", "End-to-end flow"; "Understanding MLA", Phase A step A1):
+ * y = x W_dkv (float accumulation), latent = y[0:d_c], rope key =
+ * RoPE(y[d_c:d_c+d_rope], position), and cache[b][pos][:] = latent || rope key,
+ * rounded once to dims->dtype.
+ *   x          (device) [batch*n_new][hidden]; token i of sequence b is row b*n_new+i.
+ *   W_dkv      (device) [hidden][d_c + d_rope].
+ *   rms_gamma  must be NULL (latent RMSNorm is not implemented: MLA_ERR_UNSUPPORTED).
+ *   positions  (device) int32[batch*n_new]: slot of each new token.  A position
+ *              outside [0, capacity) sets MLA_ERR_POS and that row is not written.
+ *   cache      (device) [batch][capacity][d_c + d_rope]; only the addressed slots
+ *              are written, every other byte is left untouched.
+ *   status     (device) int32 status word. */
+MLA_API int mla_append(const mla_dims* dims, int32_t batch, int32_t n_new, int32_t hidden,
+               const void* x, const void* W_dkv, const float* rms_gamma,
+               const int32_t* positions, void* cache, int64_t capacity,
+               int32_t* status, void* stream);
+
+/* Absorbed MLA decode for n_q query tokens per sequence.
+ * For sequence b holding len_b cached tokens (its queries' own entries
+ * included), query j sits at position p = len_b - n_q + j and attends keys
+ * 0..p.  Per head h:
+ *   q_lat  = [ W_uk[h] q_nope  ||  RoPE(q_rope, p) ]            (width d_c + d_rope)
+ *   s_n    = softmax_scale * < q_lat , cache[b][n][:] >,  n <= p
+ *   o_lat  = sum_n softmax(s)_n * cache[b][n][0:d_c]
+ *   out    = o_lat W_uv[h]
+ * which equals softmax(Q K^T / sqrt(qk_nope + d_rope)) V with K = [c W_uk[h] ||
+ * rope key] and V = c W_uv[h] ("Understanding MLA", sections 3-4; "Multi-Head
+ * Latent Attention", section 2 "Computational complexity").
+ *   q_nope    (device) [batch][n_q][heads][qk_nope]
+ *   q_rope    (device) [batch][n_q][heads][d_rope], not yet rotated
+ *   W_uk      (device) [heads][d_c][qk_nope]   (K^(h) = c W_uk[h])
+ *   W_uv      (device) [heads][d_c][v_dim]     (V^(h) = c W_uv[h])
+ *   cache     (device) [batch][capacity][d_c + d_rope], rope keys already rotated
+ *   seq_lens  (device) int32[batch]; a length < n_q, > capacity or > max_len sets
+ *             MLA_ERR_LEN in the status word and that sequence's outputs are zero.
+ *   max_len   host-known bound on every len_b (n_q <= max_len <= capacity).
+ *   out       (device) [batch][n_q][heads][v_dim]
+ *   workspace (device) >= mla_decode_workspace_bytes(...) bytes, 256-byte aligned.
+ *   splits    0 = automatic; k > 0 asks for k key splits per query.
+ *   status    (device) int32 status word. */
+MLA_API int mla_decode(const mla_dims* dims, int32_t batch, int32_t n_q,
+               const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
+               const void* cache, int64_t capacity, const int32_t* seq_lens, int64_t max_len,
+               void* out, void* workspace, size_t workspace_bytes, int32_t splits,
+               int32_t* status, void* stream);
+
+/* Waits for `stream`, copies the status word to *host_status and resets it to
+ * MLA_OK.  Returns MLA_OK or MLA_ERR_CUDA. */
+MLA_API int mla_get_status(int32_t* status, void* stream, int32_t* host_status);
+
+/* Name of a status code ("MLA_OK", "MLA_ERR_LEN", ...). */
+MLA_API const char* mla_status_string(int code);
+
+/* Number of CUDA kernels the most recent mla_decode / mla_append call on this
+ * host thread enqueued (for launch accounting). */
+MLA_API int32_t mla_last_launch_count(void);
+
+/* Per-kernel timing on the launching stream.  mla_profile_enable(1) makes
+ * every later call record a CUDA event before and after each kernel it
+ * enqueues (events are created on first use and destroyed by
+ * mla_profile_enable(0); no device memory is involved).  mla_profile_read
+ * waits for the recorded events and returns, per kernel name, the launch
+ * count and the summed milliseconds since the previous read:
+ *   names      host buffer receiving NUL-separated kernel names
+ *   counts     host int32[max_kernels]; total_ms host float[max_kernels]
+ * Returns the number of kernel names written (>= 0), or -MLA_ERR_CUDA /
+ * -MLA_ERR_ARG. */
+MLA_API int mla_profile_enable(int on);
+MLA_API int mla_profile_read(char* names, size_t names_len, int32_t* counts, float* total_ms,
+                             int32_t max_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H */

@@ -1,0 +1,8 @@
+"""B200-native MLA absorbed decode: libmla (CUDA, sm_100a) and its Python binding.
+
+``binding`` is the ctypes layer over include/mla.h; ``runner`` moves a
+generated workload onto the GPU and drives the library; ``inputs`` holds the
+seeded synthetic inputs.  Importing the package loads nothing; the library is
+loaded on first use and a missing build raises.
+"""
+__all__ = ["binding", "inputs", "runner"]

@@ -1,0 +1,48 @@
+// Device helpers shared by every kernel of libmla: element conversion, the
+// status word, and the rotary embedding of one interleaved pair.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// First error wins: the word only changes while it still holds MLA_OK.
+__device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
+    if (status) atomicCAS(status, MLA_OK, code);
+}
+
+// Rotation of the interleaved pair (x0, x1) with index i of a d_rope-wide
+// rope vector at position pos: angle = pos * base^(-2i/d_rope).  The angle and
+// its sine/cosine are taken in double so that positions up to 2^31 keep the
+// rotation exact to float rounding; the result is rounded to float once.
+__device__ __forceinline__ void rope_pair(float x0, float x1, int64_t pos, int i, int d_rope,
+                                          float base, float* y0, float* y1) {
+    const double theta = pow((double)base, -2.0 * (double)i / (double)d_rope);
+    const double ang = (double)pos * theta;
+    double s, c;
+    sincos(ang, &s, &c);
+    *y0 = (float)((double)x0 * c - (double)x1 * s);
+    *y1 = (float)((double)x0 * s + (double)x1 * c);
+}
+
+// Query position of token j of a sequence holding len keys (its queries'
+// entries included): p = len - n_q + j.
+__device__ __forceinline__ int64_t query_pos(int64_t len, int n_q, int j) { return len - n_q + j; }
+
+__device__ __forceinline__ bool len_ok(int64_t len, int n_q, int64_t capacity, int64_t max_len) {
+    return len >= n_q && len <= capacity && len <= max_len;
+}
+
+}  // namespace mla

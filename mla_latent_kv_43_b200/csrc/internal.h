@@ -1,0 +1,56 @@
+// Internal interface between the C ABI (mla_api.cu) and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+struct DecodeCall {
+    mla_dims d;
+    int batch, n_q;
+    const void *q_nope, *q_rope, *W_uk, *W_uv, *cache;
+    int64_t capacity;
+    const int32_t* seq_lens;
+    int64_t max_len;
+    void* out;
+    char* ws;
+    mla_ws_layout L;
+    int32_t* status;
+    cudaStream_t stream;
+};
+
+struct AppendCall {
+    mla_dims d;
+    int batch, n_new, hidden;
+    const void *x, *W_dkv;
+    const int32_t* positions;
+    void* cache;
+    int64_t capacity;
+    int32_t* status;
+    cudaStream_t stream;
+};
+
+// True when the tensor-core path serves these dims: bf16 with the
+// DeepSeek-V3 head geometry (128 heads, latent 512, rope 64, nope 128, value 128).
+bool sm100_decode_supported(const mla_dims& d);
+bool sm100_append_supported(const mla_dims& d, int hidden);
+
+// Workspace layouts (offsets 256-byte aligned).
+void generic_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int splits,
+                    mla_ws_layout* L);
+void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int splits,
+                  mla_ws_layout* L);
+
+// Each returns MLA_OK or MLA_ERR_CUDA and adds the kernels it enqueued to *launches.
+int generic_decode(const DecodeCall& c, int* launches);
+int sm100_decode(const DecodeCall& c, int* launches);
+int generic_append(const AppendCall& c, int* launches);
+int sm100_append(const AppendCall& c, int* launches);
+int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
+              const int32_t* positions, cudaStream_t stream);
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace mla

@@ -1,0 +1,90 @@
+"""Algorithmic bytes and FLOPs of one decode step (what the roofline divides).
+
+Storage per cached token and layer is the latent plus the rope key, d_c +
+d_rope values ("Understanding MLA (Multi-head Latent Attention)", section 5:
+512 + 64 = 576; at 2 bytes that is 1152 B, and over DeepSeek-V3's 61 layers
+about 70 KB per token, as the akshathtiwari "MLA" blog states).
+
+Counting rules: every cache row a query can see is read once per sequence
+(all heads and all query tokens of a sequence share it); each weight is read
+once per step; queries are read and outputs written once.  Split-KV partial
+results are implementation traffic and are not counted.  FLOPs are 2 per
+multiply-add of the absorbed form: per visible key and query token,
+H * (d_c + d_rope) for the score and H * d_c for the weighted latent sum;
+per query token, H * qk_nope * d_c for the absorption and H * d_c * v_dim
+for the value up-projection; 2 * hidden * (d_c + d_rope) per appended token.
+"""
+from __future__ import annotations
+
+import json
+import os
+from typing import Dict, Sequence
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def cache_bytes_per_token(d_c: int, d_rope: int, elem_bytes: int, layers: int = 1) -> int:
+    return (d_c + d_rope) * elem_bytes * layers
+
+
+def load_peaks() -> Dict[str, float]:
+    """Measured peaks of this GPU pool, else the recorded fallback figures."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def step_work(w, lens: Sequence[int]) -> Dict[str, float]:
+    """Algorithmic bytes/FLOPs of one step of workload ``w`` with lengths ``lens``."""
+    es = 4 if w.dtype == "fp32" else 2
+    D = w.d_c + w.d_rope
+    H = w.heads
+    B = w.batch
+    qt = B * w.n_q                                     # query tokens
+    keys_per_seq = [int(L) for L in lens]
+    visible = sum(sum(L - w.n_q + j + 1 for j in range(w.n_q)) for L in keys_per_seq)
+    r = {}
+    r["cache_bytes"] = sum(keys_per_seq) * D * es
+    r["weight_bytes"] = H * w.d_c * (w.qk_nope + w.v_dim) * es
+    r["q_bytes"] = qt * H * (w.qk_nope + w.d_rope) * es
+    r["out_bytes"] = qt * H * w.v_dim * es
+    r["core_flops"] = visible * 2 * H * (D + w.d_c)
+    r["proj_flops"] = qt * 2 * H * w.d_c * (w.qk_nope + w.v_dim)
+    r["append_bytes"] = 0
+    r["append_flops"] = 0
+    if w.n_new:
+        m = B * w.n_new
+        r["append_bytes"] = (w.hidden * D + m * w.hidden + m * D) * es
+        r["append_flops"] = 2 * m * w.hidden * D
+    r["bytes"] = r["cache_bytes"] + r["weight_bytes"] + r["q_bytes"] + r["out_bytes"] + r["append_bytes"]
+    r["flops"] = r["core_flops"] + r["proj_flops"] + r["append_flops"]
+    r["query_tokens"] = qt
+    return r
+
+
+def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_elem: int) -> float:
+    """Algorithmic bytes of one launch of a kernel of the step.
+
+    The attention kernel moves the visible cache rows once per sequence, the
+    absorbed queries in and the latent outputs out; absorb/up-projection move
+    their weight and activations; append moves W_dkv, x and the new rows.
+    """
+    es = 4 if w.dtype == "fp32" else 2
+    D = w.d_c + w.d_rope
+    qt = w.batch * w.n_q
+    H = w.heads
+    if "attend" in kernel or "core" in kernel:
+        return sum(int(L) for L in lens) * D * es + qt * H * D * q_lat_elem + qt * H * w.d_c * o_lat_elem
+    if "absorb" in kernel:
+        return H * w.d_c * w.qk_nope * es + qt * H * (w.qk_nope + w.d_rope) * es + qt * H * D * q_lat_elem
+    if "upproj" in kernel:
+        return H * w.d_c * w.v_dim * es + qt * H * w.d_c * o_lat_elem + qt * H * w.v_dim * es
+    if "append" in kernel:
+        m = w.batch * w.n_new
+        return (w.hidden * D + m * w.hidden + m * D) * es
+    return 0.0

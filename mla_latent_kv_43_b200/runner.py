@@ -1,0 +1,80 @@
+"""Drive libmla on one GPU for a generated workload.
+
+A ``DeviceProblem`` holds a workload's tensors on the device, in the layout
+the library takes: the cache as [B][capacity][d_c + d_rope] with its rope
+keys rotated at their slot positions by ``mla_rope`` (what the append step
+would have stored), the weights, per-sequence lengths, and caller-owned
+output, workspace and status buffers.  ``step()`` runs one decode step
+(append of the new tokens when the workload has them, then attention).
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import binding as B
+from .inputs import Workload
+
+
+class DeviceProblem:
+    def __init__(self, w: Workload, host: Dict[str, torch.Tensor], device="cuda", splits: int = 0,
+                 stream: Optional[torch.cuda.Stream] = None, max_len: Optional[int] = None):
+        self.w = w
+        self.dims = B.dims_of(w)
+        self.splits = splits
+        self.stream = stream
+        dev = torch.device(device)
+        self.device = dev
+        to = lambda t: t.to(dev, non_blocking=False).contiguous()
+        self.q_nope = to(host["q_nope"])
+        self.q_rope = to(host["q_rope"])
+        self.W_uk = to(host["W_uk"])
+        self.W_uv = to(host["W_uv"])
+        self.seq_lens = to(host["seq_lens"])
+        self.max_len = int(host["seq_lens"].max()) if max_len is None else int(max_len)
+        # cache = [latent || raw rope key] per slot, then rotate every slot's rope
+        # key at its position inside the sequence.
+        self.cache = torch.empty(w.batch, w.capacity, w.d, dtype=w.torch_dtype, device=dev)
+        self.cache[..., : w.d_c].copy_(host["c_kv"])
+        self.cache[..., w.d_c:].copy_(host["k_rope"])
+        slot_pos = torch.arange(w.capacity, dtype=torch.int32, device=dev).repeat(w.batch)
+        B.mla_rope(self.dims, w.batch * w.capacity, self.cache, w.d, slot_pos, stream=stream,
+                   offset_elems=w.d_c)
+        del slot_pos
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.out = torch.empty(w.batch, w.n_q, w.heads, w.v_dim, dtype=w.torch_dtype, device=dev)
+        self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, self.max_len, splits)
+        self.workspace = torch.empty(max(self.layout["total"], 256), dtype=torch.uint8, device=dev)
+        self.has_append = w.n_new > 0
+        if self.has_append:
+            self.x = to(host["x"])
+            self.W_dkv = to(host["W_dkv"])
+            self.positions = to(host["positions"])
+
+    # --- the step -----------------------------------------------------------
+    def append(self):
+        B.mla_append(self.dims, self.x, self.W_dkv, self.positions, self.cache, self.status,
+                     batch=self.w.batch, n_new=self.w.n_new, stream=self.stream)
+
+    def decode(self):
+        B.mla_decode(self.dims, self.q_nope, self.q_rope, self.W_uk, self.W_uv, self.cache,
+                     self.seq_lens, self.max_len, self.out, self.workspace, self.status,
+                     splits=self.splits, stream=self.stream)
+
+    def step(self) -> int:
+        """One decode step; returns the number of kernels it enqueued."""
+        n = 0
+        if self.has_append:
+            self.append()
+            n += B.mla_last_launch_count()
+        self.decode()
+        return n + B.mla_last_launch_count()
+
+    def get_status(self) -> int:
+        return B.mla_get_status(self.status, stream=self.stream)
+
+    def workspace_view(self, region: str, shape, dtype) -> torch.Tensor:
+        off, nbytes = self.layout[region], self.layout[region + "_bytes"]
+        t = self.workspace[off: off + nbytes].view(dtype)
+        return t.view(*shape)

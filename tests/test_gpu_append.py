@@ -1,0 +1,77 @@
+"""The append step on the GPU: exactly the addressed cache slots change
+(bit-exact slot indexing against a sentinel pattern), their values match the
+oracle's fp64 rows, and positions outside the cache set MLA_ERR_POS."""
+import os
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+from gpu_common import TOL, rel_err  # noqa: E402
+from mla_latent_kv_43_b200 import binding as B  # noqa: E402
+from mla_latent_kv_43_b200 import inputs as gen  # noqa: E402
+from oracle import mla_oracle as O  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+SMALL = dict(heads=2, d_c=8, d_rope=4, qk_nope=6, v_dim=5)
+V3 = dict(heads=128, d_c=512, d_rope=64, qk_nope=128, v_dim=128)
+CASES = {"fp32_small": ("fp32", SMALL, 24), "bf16_small": ("bf16", SMALL, 40),
+         "bf16_v3": ("bf16", V3, 7168)}
+
+
+def run_append(case, positions, batch, n_new, capacity, seed=0):
+    dtype, g, hidden = CASES[case]
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    rng = np.random.default_rng(seed)
+    D = g["d_c"] + g["d_rope"]
+    x = torch.from_numpy(rng.standard_normal((batch * n_new, hidden), dtype=np.float32)).to(tdt)
+    W = torch.from_numpy((rng.standard_normal((hidden, D), dtype=np.float32) / np.sqrt(hidden)).astype(np.float32)).to(tdt)
+    # sentinel: a fixed byte pattern that is a finite value in both dtypes
+    cache = torch.empty(batch, capacity, D, dtype=tdt, device="cuda")
+    cache.view(torch.uint8).fill_(0x3C)
+    before = cache.clone()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dims = B.make_dims(dtype=dtype, **g)
+    pos = torch.tensor(positions, dtype=torch.int32)
+    B.mla_append(dims, x.cuda(), W.cuda(), pos.cuda(), cache, status, batch=batch, n_new=n_new)
+    code = B.mla_get_status(status)
+    return dims, x, W, pos, before, cache, code
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_append_writes_exactly_the_addressed_slots(case):
+    batch, n_new, cap = 3, 2, 70
+    positions = [5, 6, 0, 1, cap - 2, cap - 1]
+    dims, x, W, pos, before, cache, code = run_append(case, positions, batch, n_new, cap, seed=1)
+    assert code == 0
+    changed = (cache.view(torch.int16 if cache.element_size() == 2 else torch.int32)
+               != before.view(torch.int16 if cache.element_size() == 2 else torch.int32)).any(-1).cpu()
+    expect = torch.zeros(batch, cap, dtype=torch.bool)
+    for r, p in enumerate(positions):
+        expect[r // n_new, p] = True
+    assert torch.equal(changed, expect)
+    rows = O.append_rows(x, W, positions, dims.d_c, dims.rope_base)
+    got = np.stack([cache[r // n_new, p].double().cpu().numpy() for r, p in enumerate(positions)])
+    tol = TOL["fp32"] if case.startswith("fp32") else TOL["bf16"]
+    assert rel_err(got, rows) <= tol
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_append_rejects_positions_outside_the_cache(case):
+    batch, n_new, cap = 2, 2, 16
+    positions = [3, -1, cap, 15]
+    dims, x, W, pos, before, cache, code = run_append(case, positions, batch, n_new, cap, seed=2)
+    assert code == B.CODES["MLA_ERR_POS"]
+    rows = O.append_rows(x, W, positions, dims.d_c, dims.rope_base)
+    same = lambda b, p: torch.equal(cache[b, p], before[b, p])
+    assert not same(0, 3) and not same(1, 15)
+    # every other slot keeps the sentinel
+    mask = torch.ones(batch, cap, dtype=torch.bool)
+    mask[0, 3] = mask[1, 15] = False
+    assert torch.equal(cache[mask], before[mask])
+    tol = TOL["fp32"] if case.startswith("fp32") else TOL["bf16"]
+    assert rel_err(cache[0, 3].double().cpu().numpy(), rows[0]) <= tol
+    assert rel_err(cache[1, 15].double().cpu().numpy(), rows[3]) <= tol
