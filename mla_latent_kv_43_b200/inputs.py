@@ -162,11 +162,13 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
     return out
 
 
-def tiny(dtype: str = "fp32", *, batch=2, heads=3, d_c=8, d_rope=4, qk_nope=6,
+def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6,
          v_dim=5, n_q=1, lens=(5, 9), capacity=None, seed=0, latent_rms_norm=False,
          hidden=0, n_new=0) -> Workload:
-    """A small custom workload for pins and edge cases."""
+    """A small custom workload for pins and edge cases (batch = len(lens))."""
     cap = capacity if capacity is not None else max(lens)
+    if batch is None:
+        batch = len(lens)
     return Workload(name="custom", dtype=dtype, batch=batch, heads=heads, d_c=d_c,
                     d_rope=d_rope, qk_nope=qk_nope, v_dim=v_dim, n_q=n_q,
                     lens=tuple(lens), capacity=cap, latent_rms_norm=latent_rms_norm,
