@@ -1,0 +1,148 @@
+// Tensor-core decode path for the DeepSeek-V3 head geometry (bf16): workspace
+// layout, the split-KV combine kernel and the launch sequence
+//   absorb (+ q-RoPE + key-tile plan) -> attention -> combine -> up-projection.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "profile.h"
+#include "sm100_host.h"
+
+namespace mla {
+namespace sm100 {
+int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* launches);
+int launch_upproj(const DecodeCall& c, const __nv_bfloat16* o_lat, int* launches);
+int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
+                  float* part_o, float* part_lse, int pairs, int* launches);
+
+namespace {
+
+constexpr int kHeads = 128, kDc = 512;
+
+// Merge the pieces of query tokens whose key tiles were cut across clusters
+// (log-sum-exp weighting, base 2), and zero the latent output of tokens with
+// an invalid length.  Tokens finished inside one cluster are left untouched.
+// grid (BJ, 128 / 4): 4 heads per block, 128 threads, 16 columns each.
+__global__ void __launch_bounds__(128)
+combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* __restrict__ part_o,
+               const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat) {
+    const int bj = blockIdx.x;
+    const int T = cum[BJ];
+    const int c0 = cum[bj], c1 = cum[bj + 1];
+    const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+    const int col = (threadIdx.x & 31) * 16;
+    __nv_bfloat16* dst = o_lat + ((int64_t)bj * kHeads + h) * kDc + col;
+    if (c1 == c0) {
+        for (int i = 0; i < 16; ++i) dst[i] = __float2bfloat16_rn(0.f);
+        return;
+    }
+    auto start = [&](int p) { return (int)((int64_t)p * T / pairs); };
+    auto pair_of = [&](int t) {      // largest p with start(p) <= t
+        int lo = 0, hi = pairs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (start(mid) <= t) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    const int pf = pair_of(c0), pl = pair_of(c1 - 1);
+    if (pf == pl) return;            // finished inside one cluster
+    // clusters with an empty tile range between the first and the last piece hold nothing
+    auto empty = [&](int p) { return start(p) == (p + 1 < pairs ? start(p + 1) : T); };
+    float M = -INFINITY;
+    for (int p = pf; p <= pl; ++p) {
+        if (p != pf && empty(p)) continue;
+        const int slot = p == pf ? 2 * p + 1 : 2 * p;
+        M = fmaxf(M, part_lse[slot * kHeads + h]);
+    }
+    float acc[16];
+    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+    float wsum = 0.f;
+    for (int p = pf; p <= pl; ++p) {
+        if (p != pf && empty(p)) continue;
+        const int slot = p == pf ? 2 * p + 1 : 2 * p;
+        const float w = exp2f(part_lse[slot * kHeads + h] - M);
+        wsum += w;
+        const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slot * kHeads + h) * kDc + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v = src[i];
+            acc[4 * i] = fmaf(w, v.x, acc[4 * i]);
+            acc[4 * i + 1] = fmaf(w, v.y, acc[4 * i + 1]);
+            acc[4 * i + 2] = fmaf(w, v.z, acc[4 * i + 2]);
+            acc[4 * i + 3] = fmaf(w, v.w, acc[4 * i + 3]);
+        }
+    }
+    const float inv = 1.f / wsum;
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+        pk[i] = *reinterpret_cast<uint32_t*>(&v);
+    }
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+}
+
+int pairs_for(int splits) {
+    const int max_pairs = std::max(1, sm_count() / 2);
+    return splits > 0 ? std::min(splits, max_pairs) : max_pairs;
+}
+
+}  // namespace
+}  // namespace sm100
+
+bool sm100_decode_supported(const mla_dims& d) {
+    return d.dtype == MLA_BF16 && d.heads == 128 && d.d_c == 512 && d.d_rope == 64 && d.qk_nope == 128 &&
+           d.v_dim == 128;
+}
+
+bool sm100_append_supported(const mla_dims&, int) { return false; }
+
+void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int splits, mla_ws_layout* L) {
+    (void)max_len;
+    const int64_t BJ = (int64_t)batch * n_q;
+    const int P = sm100::pairs_for(splits);
+    *L = mla_ws_layout{};
+    size_t off = 0;
+    auto take = [&](size_t bytes, size_t* o, size_t* sz) {
+        *o = off;
+        *sz = bytes;
+        off = align_up(off + bytes, 256);
+    };
+    take(BJ * d.heads * (d.d_c + d.d_rope) * 2, &L->q_lat, &L->q_lat_bytes);
+    take(BJ * d.heads * d.d_c * 2, &L->o_lat, &L->o_lat_bytes);
+    take((size_t)2 * P * d.heads * d.d_c * 4, &L->part_o, &L->part_o_bytes);
+    take((size_t)2 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);
+    take((BJ + 1) * 4, &L->sched, &L->sched_bytes);
+    L->total = off;
+    L->compute_dtype = MLA_BF16;
+    L->splits = P;
+}
+
+int sm100_decode(const DecodeCall& c, int* launches) {
+    auto* q_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.q_lat);
+    auto* o_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.o_lat);
+    auto* part_o = reinterpret_cast<float*>(c.ws + c.L.part_o);
+    auto* part_lse = reinterpret_cast<float*>(c.ws + c.L.part_lse);
+    auto* cum = reinterpret_cast<int32_t*>(c.ws + c.L.sched);
+    const int P = c.L.splits;
+    const int BJ = c.batch * c.n_q;
+    int rc;
+    if ((rc = sm100::launch_absorb(c, q_lat, cum, launches))) return rc;
+    if ((rc = sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, P, launches))) return rc;
+    prof_begin(c.stream, "sm100_combine");
+    sm100::combine_kernel<<<dim3(BJ, 128 / 4), 128, 0, c.stream>>>(cum, BJ, P, part_o, part_lse, o_lat);
+    prof_end(c.stream);
+    if (launches) ++*launches;
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return sm100::launch_upproj(c, o_lat, launches);
+}
+
+int sm100_append(const AppendCall&, int*) { return MLA_ERR_UNSUPPORTED; }
+
+}  // namespace mla

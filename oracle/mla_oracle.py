@@ -132,31 +132,53 @@ def decode_naive(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, n_q: int,
     return out
 
 
+def absorbed_query(q_nope, q_rope, W_uk_h, p, base: float = 10000.0) -> np.ndarray:
+    """q_lat = [W_K^(h) q_nope || RoPE(q_rope, p)]: the key up-projection moved to
+    the query side ("Understanding MLA", section 4)."""
+    return np.concatenate([_f64(W_uk_h) @ _f64(q_nope), rope(q_rope, p, base)])
+
+
+def latent_attention(q_lat, c, k_rope_rot, scale: float):
+    """Softmax-weighted latent for one query against visible cache rows:
+    returns (o_lat, lse) with lse = log sum_n exp(s_n) (natural log)."""
+    s = (np.concatenate([_f64(c), _f64(k_rope_rot)], axis=1) @ q_lat) * scale
+    w = softmax(s)
+    mx = np.max(s)
+    return w @ _f64(c), mx + np.log(np.sum(np.exp(s - mx)))
+
+
 def decode_absorbed(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, n_q: int,
-                    scale: float, base: float = 10000.0):
+                    scale: float, base: float = 10000.0, *, batches=None, heads=None,
+                    return_intermediates: bool = False):
     """Absorbed form: score against the latent directly, up-project after.
 
-    q_lat = W_K^(h) q_nope moves the key up-projection to the query side
-    ("Understanding MLA", section 4); the value up-projection is applied to
-    the softmax-weighted latent ("Multi-head latent attention", aicassindra,
-    "End-to-end flow", producing the output).  Used only to check the algebra.
+    The value up-projection is applied to the softmax-weighted latent
+    ("Multi-head latent attention", aicassindra, "End-to-end flow").  Used to
+    check the algebra and to give the intermediate results of the absorbed
+    path (absorbed queries, latent outputs).
     """
     q_nope, q_rope = _f64(q_nope), _f64(q_rope)
     W_uk, W_uv = _f64(W_uk), _f64(W_uv)
     lens = [int(v) for v in np.asarray(lens).tolist()]
     B, _, H, _ = q_nope.shape
+    batches = range(B) if batches is None else batches
+    heads = range(H) if heads is None else heads
     out = np.zeros((B, n_q, H, W_uv.shape[-1]), dtype=np.float64)
-    for b in range(B):
+    inter = {}
+    for b in batches:
         L = lens[b]
         c = _f64(c_kv[b, :L])
         k_r = _f64(k_rope_rot[b, :L])
-        for h in range(H):
+        for h in heads:
             for j in range(n_q):
                 p = L - n_q + j
-                q_lat = W_uk[h] @ q_nope[b, j, h]                # [d_c]
-                s = (c[: p + 1] @ q_lat + k_r[: p + 1] @ rope(q_rope[b, j, h], p, base)) * scale
-                w = softmax(s)
-                out[b, j, h] = (w @ c[: p + 1]) @ W_uv[h]
+                q_lat = absorbed_query(q_nope[b, j, h], q_rope[b, j, h], W_uk[h], p, base)
+                o_lat, lse = latent_attention(q_lat, c[: p + 1], k_r[: p + 1], scale)
+                out[b, j, h] = o_lat @ W_uv[h]
+                if return_intermediates:
+                    inter[(b, j, h)] = (q_lat, o_lat, lse)
+    if return_intermediates:
+        return out, inter
     return out
 
 
