@@ -60,6 +60,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(gen.WORKLOADS))
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    ap.add_argument("--min-warmup-s", type=float, default=1.5, help="minimum warm-up wall time")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -229,10 +230,10 @@ def run_ours(a, rank, world, local):
     peaks = RF.load_peaks()
     sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
 
-    # warm-up: at least W steps and at least 1.5 s
+    # warm-up: at least W steps and at least --min-warmup-s seconds
     t_w = time.time()
     k = 0
-    while k < a.warmup or time.time() - t_w < 1.5:
+    while k < a.warmup or time.time() - t_w < a.min_warmup_s:
         flush.zero_()
         prob.step()
         k += 1

@@ -37,6 +37,20 @@ __device__ __forceinline__ void rope_pair(float x0, float x1, int64_t pos, int i
     *y1 = (float)((double)x0 * s + (double)x1 * c);
 }
 
+// Same rotation with the pair frequency theta = base^(-2i/d_rope) given:
+// the angle pos * theta is formed and reduced modulo 2*pi in double, so the
+// single-precision sincosf only sees |x| <= pi.
+__device__ __forceinline__ void rope_pair_theta(float x0, float x1, int64_t pos, double theta, float* y0,
+                                                float* y1) {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double ang = (double)pos * theta;
+    const double red = ang - rint(ang * (1.0 / two_pi)) * two_pi;
+    float s, c;
+    sincosf((float)red, &s, &c);
+    *y0 = x0 * c - x1 * s;
+    *y1 = x0 * s + x1 * c;
+}
+
 // Query position of token j of a sequence holding len keys (its queries'
 // entries included): p = len - n_q + j.
 __device__ __forceinline__ int64_t query_pos(int64_t len, int n_q, int j) { return len - n_q + j; }

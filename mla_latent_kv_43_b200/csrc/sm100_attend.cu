@@ -3,7 +3,7 @@
 // For one query token (b, j) and a range of 64-key tiles of its sequence,
 // with q_lat = [W_uk q_nope || RoPE(q_rope)] (576 wide, all 128 heads):
 //     S[h][n] = <q_lat[h], cache[b][n][0:576]>                    (score)
-//     online softmax over n (base 2, scale folded in), fp32
+//     online softmax over n (base 2, scale folded in), fp32 state
 //     O[h][0:512] += P[h][n] cache[b][n][0:512]                    (weighted latent)
 // i.e. the score of "Understanding MLA (Multi-head Latent Attention)",
 // section 4 (content part through the absorbed query, position part through
@@ -11,26 +11,34 @@
 // "Multi-head latent attention", "End-to-end flow".
 //
 // Work split.  All heads of a token share each cache row, so the 128 heads
-// are the M dimension of both contractions.  The fp32 accumulator of
-// 128 heads x 512 latent columns would fill all 512 TMEM columns, so a
-// cluster of two CTAs splits the latent: CTA r owns latent columns
-// [256r, 256r+256) and rope columns [512+32r, 512+32r+32).  Each CTA loads
-// only its 288 columns of every tile (each cache byte crosses HBM once, no
-// multicast), computes a partial score over its 288 columns with Q resident
-// in TMEM, and the two partials are exchanged through distributed shared
-// memory and added in the same order on both CTAs, so both run the identical
-// softmax.  Each CTA then accumulates its half of O from the same smem tile
-// read as an MN-major operand.
+// are the M dimension of both contractions.  A 128 x 512 fp32 accumulator
+// would fill all of TMEM, so a cluster of two CTAs splits the latent: CTA r
+// owns latent columns [256r, 256r+256) and rope columns [512+32r, +32).
+// Each CTA loads only its 288 columns of every tile (each cache byte crosses
+// HBM once, no multicast) and computes a partial score over them.  The
+// exchange warps round their partial to fp16 and store it straight into the
+// peer's shared memory (two buffers, so the exchange runs up to two tiles
+// ahead); each softmax thread adds its own fp32 partial to the peer's.  The
+// two CTAs' scores thus differ only by that fp16 rounding; each CTA keeps its
+// own running max and sum and normalises its own half of O with them, so each
+// half is self-consistent.  Each CTA accumulates its half of O from the same
+// smem tile read as an MN-major operand.
 //
-// Roles (192 threads): warp 0 issues TMA, warp 1 issues MMAs, warps 2-5 run
-// the softmax (thread <-> head <-> TMEM lane) and the epilogues.
+// TMEM (512 columns): O [0,256), S double buffer [256,384), Q latent slice
+// [384,512) (A operand of the score GEMM); the 32 rope columns of Q are an
+// smem operand.
+//
+// Roles (448 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 "exchange"
+// (score tile -> fp16 -> peer smem, query loads; thread <-> head <-> TMEM lane),
+// warps 6-13 "softmax" (P, O rescale, epilogue; two threads per head row).
 //
 // Work items.  The key tiles of all query tokens are concatenated and cut
 // into one contiguous range per cluster.  A token whose tiles all fall in one
 // cluster's range is finished there (normalised latent output, bf16); a token
 // cut across clusters leaves fp32 partial outputs plus log2-sum-exp per piece
-// for the combine kernel.
+// for the combine step.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "common.cuh"
@@ -42,23 +50,21 @@
 namespace mla {
 namespace sm100 {
 
-constexpr int kAttnKeys = 64;
-
 namespace {
 
-constexpr int kStages = 3;
+constexpr int kKeys = 64;
+constexpr int kStages = 4;
 constexpr int kLatBox = 8192;                      // 64 keys x 64 columns x 2 B
 constexpr int kRopeBox = 4096;                     // 64 keys x 32 columns x 2 B
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;
-constexpr int kPBytes = 128 * 128;                 // 128 heads x 64 keys bf16
-constexpr int kXRow = 272;                         // 64 floats + 16 B pad (bank-conflict free)
-constexpr int kXBytes = 128 * kXRow;
-constexpr int kOffP = kStages * kStageBytes;
-constexpr int kOffX = kOffP + 2 * kPBytes;
-constexpr int kSmemBytes = kOffX + 2 * kXBytes;
-constexpr int kThreads = 192;
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 320, kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;          // log2 units: rescale O only when the max grows by > 2^8
+constexpr int kTileBytes = 128 * 128;              // 128 rows x 64 x 2 B (P, exchange tiles)
+constexpr int kOffP = kStages * kStageBytes;       // two P buffers
+constexpr int kOffXin = kOffP + 2 * kTileBytes;    // two buffers, written by the peer
+constexpr int kOffQr = kOffXin + 2 * kTileBytes;   // 128 heads x 32 rope columns, SW64
+constexpr int kSmemBytes = kOffQr + 128 * 64;
+constexpr int kThreads = 448;
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
 struct AttnArgs {
     const __nv_bfloat16* q_lat;   // [BJ][128][576]
@@ -76,11 +82,11 @@ struct Item {
     int bj, t0, t1, n_vis, slot;  // slot < 0: finished here
 };
 
-// Iterates the pieces of the concatenated tile range [s0, s1) of one cluster.
+// Pieces of the concatenated tile range [s0, s1) of one cluster, in order.
 struct ItemIter {
     const int32_t* cum;
-    int BJ, n_q, bj, s0, s1, pair;
     const int32_t* lens;
+    int BJ, n_q, bj, s0, s1, pair;
     __device__ void init(const AttnArgs& a, int p) {
         cum = a.cum;
         BJ = a.BJ;
@@ -117,23 +123,48 @@ struct ItemIter {
     }
 };
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
-
-__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
                  : "memory");
     return v;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Asynchronous 16-byte store into the peer CTA's shared memory; its bytes are
+// counted (complete_tx) on the peer's mbarrier `bar` (both shared::cluster).
+__device__ __forceinline__ void st_async_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     addr),
+                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
                  : "memory");
+}
+
+// Relaxed arrive on a barrier of the peer CTA (no ordering of this thread's
+// earlier memory operations is implied).
+__device__ __forceinline__ void mbar_arrive_peer_relaxed(uint32_t peer_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_addr) : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[16];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        tmem_ld16(taddr + 16 * c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[16 * c + i] = __uint_as_float(r[i]);
+    }
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
@@ -142,10 +173,14 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kStages], empty[kStages];
-    __shared__ uint64_t s_full, s_free, q_ready, drain;
-    __shared__ uint64_t p_ready[2], p_free[2], x_full[2];
+    __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, drain;
+    __shared__ uint64_t p_ready[2], xin_full[2], rx_done[2];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
+    // per-warpgroup decisions, each written by the leader before a named barrier
+    // and read after it; a barrier separates every read from the next write
+    __shared__ int ex_stop, sm_stop, sm_stop2, sm_top;
+    __shared__ float row_max[2][128], row_sum[2][128];   // softmax half-row exchange
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -157,15 +192,18 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(&s_full, 1);
-        mbar_init(&s_free, 128);
-        mbar_init(&q_ready, 128);
-        mbar_init(&drain, 1);
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&p_ready[i], 128);
-            mbar_init(&p_free[i], 1);
-            mbar_init(&x_full[i], 128);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 5);       // 4 exchange warps + the softmax leader
+            mbar_init(&xin_full[i], 1);     // my softmax leader's expect_tx + the peer's bytes
+            mbar_init(&rx_done[i], 1);      // the peer's softmax leader
         }
+        mbar_init(&o_done[0], 1);           // O GEMMs of even / odd global tiles
+        mbar_init(&o_done[1], 1);
+        mbar_init(&q_ready, 1);
+        mbar_init(&drain, 1);
+        mbar_init(&p_ready[0], 1);          // P tile of even / odd global tiles written
+        mbar_init(&p_ready[1], 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -175,9 +213,10 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();          // the peer's barriers are initialised before any remote arrive
+    cluster_sync();          // the peer's barriers are initialised before any remote access
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    const uint32_t sbase = smem_u32(smem);
     volatile int* abort = &abort_flag;
     auto fail = [&]() {
         *abort = 1;
@@ -204,7 +243,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     }
                     uint8_t* st = smem + s * kStageBytes;
                     mbar_expect_tx(&full[s], kStageBytes);
-                    const int key0 = t * kAttnKeys;
+                    const int key0 = t * kKeys;
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         tma_load_3d(st + i * kLatBox, &map_lat, &full[s], 256 * rank + 64 * i, key0, b);
@@ -212,229 +251,359 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 }
             }
             if (!ok) fail();
-            // let every issued load land before the CTA can exit
             const uint32_t first = it > kStages ? it - kStages : 0;
             for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Two streams in tile order: score GEMMs S(g) and latent GEMMs O(g).
+        // Each is issued as soon as its inputs are ready, so S runs ahead of O
+        // as far as the two S buffers allow.
         if (elect_one()) {
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
-            const uint32_t sbase = smem_u32(smem);
-            const uint32_t pbase = sbase + kOffP;
-            ItemIter iter;
-            iter.init(a, pair);
-            Item item;
-            uint32_t it = 0, n_items = 0;
+            const uint32_t qr = sbase + kOffQr;
+            ItemIter iterS, iterO;
+            iterS.init(a, pair);
+            iterO.init(a, pair);
+            Item itS, itO;
+            bool haveS = iterS.next(itS), haveO = iterO.next(itO);
+            int kS = 0, kO = 0;
+            uint32_t gS = 0, gO = 0, nItemsS = 0;
+            bool qS = false;                       // q_ready observed for the current S item
+            int sStep = -1;                        // K-step of the score GEMM in progress (-1: none)
+            uint64_t t_last = globaltimer();
             bool ok = true;
-            auto issue_o = [&](uint32_t g, bool first) -> bool {
-                const int pb = g & 1;
-                if (!mbar_wait(&p_ready[pb], (g >> 1) & 1, abort)) return false;
-                tc_fence_after();
-                const uint32_t st = sbase + (g % kStages) * kStageBytes;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = sdesc(pbase + pb * kPBytes + ks * 32, 16, 1024, kSwizzle128);
-                    const uint64_t bd = sdesc(st + ks * 2048, kLatBox, 1024, kSwizzle128);
-                    mma_ss(tmem + kColO, ad, bd, idO, (first && ks == 0) ? 0u : 1u);
-                }
-                mma_commit(&empty[g % kStages]);
-                mma_commit(&p_free[pb]);
-                return true;
-            };
-            while (ok && iter.next(item)) {
-                if (!mbar_wait(&q_ready, n_items & 1, abort)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int T = item.t1 - item.t0;
-                for (int k = 0; k < T && ok; ++k) {
-                    const uint32_t g = it + k;
-                    const int s = g % kStages;
-                    if (!mbar_wait(&full[s], (g / kStages) & 1, abort)) { ok = false; break; }
-                    if (g > 0 && !mbar_wait(&s_free, (g - 1) & 1, abort)) { ok = false; break; }
+            while (ok && haveO) {
+                bool progressed = false;
+                // O GEMMs first: they release the stage and unblock the softmax two tiles later
+                if (gO < gS - (sStep >= 0 ? 1u : 0u) && mbar_ready(&p_ready[gO & 1], (gO >> 1) & 1)) {
                     tc_fence_after();
+                    const int s = gO % kStages;
                     const uint32_t st = sbase + s * kStageBytes;
 #pragma unroll
-                    for (int ks = 0; ks < 16; ++ks) {
-                        const uint64_t bd = sdesc(st + (ks >> 2) * kLatBox + (ks & 3) * 32, 16, 1024, kSwizzle128);
-                        mma_ts(tmem + kColS, tmem + kColQ + 8 * ks, bd, idS, ks ? 1u : 0u);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sdesc(sbase + kOffP + (gO & 1) * kTileBytes + ks * 32, 16, 1024, kSwizzle128);
+                        const uint64_t bd = sdesc(st + ks * 2048, kLatBox, 1024, kSwizzle128);
+                        mma_ss(tmem + kColO, ad, bd, idO, (kO == 0 && ks == 0) ? 0u : 1u);
                     }
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        const uint64_t bd = sdesc(st + 4 * kLatBox + ks * 32, 16, 512, kSwizzle64);
-                        mma_ts(tmem + kColS, tmem + kColQ + 8 * (16 + ks), bd, idS, 1u);
+                    mma_commit(&empty[s]);
+                    mma_commit(&o_done[gO & 1]);
+                    ++gO;
+                    if (++kO == itO.t1 - itO.t0) {
+                        kO = 0;
+                        haveO = iterO.next(itO);
                     }
-                    mma_commit(&s_full);
-                    if (k > 0 && !issue_o(g - 1, k == 1)) ok = false;
+                    progressed = true;
                 }
-                if (ok && T > 0 && !issue_o(it + T - 1, T == 1)) ok = false;
-                it += T;
-                ++n_items;
+                // score GEMM S(gS), issued 6 K-steps at a time so a ready O is never held back long
+                if (haveS && sStep < 0) {
+                    const int s = gS % kStages, sb = gS & 1;
+                    if (!qS) qS = mbar_ready(&q_ready, nItemsS & 1);
+                    if (qS && mbar_ready(&full[s], (gS / kStages) & 1) &&
+                        (gS < 2 || mbar_ready(&s_free[sb], ((gS >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        sStep = 0;
+                        ++gS;                      // S(gS - 1) now in progress
+                    }
+                }
+                if (sStep >= 0) {
+                    const uint32_t g = gS - 1;
+                    const int s = g % kStages, sb = g & 1;
+                    const uint32_t st = sbase + s * kStageBytes;
+                    const uint32_t dS = tmem + kColS + 64 * sb;
+                    const int end = sStep + 6;
+                    for (; sStep < end; ++sStep) {
+                        if (sStep < 16) {
+                            const uint64_t bd = sdesc(st + (sStep >> 2) * kLatBox + (sStep & 3) * 32, 16, 1024, kSwizzle128);
+                            mma_ts(dS, tmem + kColQ + 8 * sStep, bd, idS, sStep ? 1u : 0u);
+                        } else {
+                            const uint64_t ad = sdesc(qr + (sStep - 16) * 32, 16, 512, kSwizzle64);
+                            const uint64_t bd = sdesc(st + 4 * kLatBox + (sStep - 16) * 32, 16, 512, kSwizzle64);
+                            mma_ss(dS, ad, bd, idS, 1u);
+                        }
+                    }
+                    if (sStep == 18) {
+                        mma_commit(&s_full[sb]);
+                        sStep = -1;
+                        if (++kS == itS.t1 - itS.t0) {
+                            kS = 0;
+                            qS = false;
+                            ++nItemsS;
+                            haveS = iterS.next(itS);
+                        }
+                    }
+                    progressed = true;
+                }
+                if (progressed) {
+                    t_last = globaltimer();
+                } else if (*abort || globaltimer() - t_last > kWaitLimitNs) {
+                    ok = false;
+                }
             }
             if (!ok) fail();
             mma_commit(&drain);
             mbar_wait(&drain, 0, nullptr);
         }
-    } else {
-        // ------------------------------------------------------------ softmax / epilogue
-        const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int h = q * 32 + lane;            // head == TMEM lane
-        const int tid = threadIdx.x - 64;       // 0..127
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ exchange warpgroup
+        // One leader does every mbarrier wait (bounded) and a named barrier
+        // broadcasts the outcome, so the warpgroup never diverges on a timeout.
+        const int q = warp & 3;
+        const int h = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const uint32_t sbase = smem_u32(smem);
-        const uint32_t x_local = sbase + kOffX;
-        const uint32_t x_peer = map_peer(x_local, peer);
-        const uint32_t xbar_peer[2] = {map_peer(smem_u32(&x_full[0]), peer), map_peer(smem_u32(&x_full[1]), peer)};
-        uint32_t o_seen[2] = {0, 0};            // completed O GEMMs observed per P buffer
-        auto wait_o = [&](uint32_t g) -> bool { // O GEMM of global tile g has completed
-            const int pb = g & 1;
-            const uint32_t n = g >> 1;
-            if (o_seen[pb] > n) return true;
-            if (!mbar_wait(&p_free[pb], n & 1, abort)) return false;
-            o_seen[pb] = n + 1;
-            return true;
-        };
+        const uint32_t xin_peer = map_peer(sbase + kOffXin, peer);
+        const uint32_t xbar_peer[2] = {map_peer(smem_u32(&xin_full[0]), peer), map_peer(smem_u32(&xin_full[1]), peer)};
+        const bool leader = (warp == 2) && lane == 0;
         ItemIter iter;
         iter.init(a, pair);
         Item item;
         uint32_t it = 0;
-        bool ok = true;
-        while (ok && iter.next(item)) {
-            // Q slice of this token into TMEM (A operand of the score GEMM)
+        while (iter.next(item)) {
+            if (leader) ex_stop = *abort;
+            named_barrier(1, 128);
+            if (ex_stop) break;
+            // query slice of this token: latent part -> TMEM, rope part -> smem (SW64 rows).
+            // Every score GEMM of the previous item has completed: its last
+            // score tile was read below before we got here.
             {
                 const uint4* src = reinterpret_cast<const uint4*>(a.q_lat + ((int64_t)item.bj * 128 + h) * 576);
                 uint32_t w[16];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {     // latent columns 256r + 32c .. +31 (16 words)
-                    const uint4 v0 = src[(256 * rank + 32 * c) / 8 + 0];
-                    const uint4 v1 = src[(256 * rank + 32 * c) / 8 + 1];
-                    const uint4 v2 = src[(256 * rank + 32 * c) / 8 + 2];
-                    const uint4 v3 = src[(256 * rank + 32 * c) / 8 + 3];
-                    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-                    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-                    w[8] = v2.x; w[9] = v2.y; w[10] = v2.z; w[11] = v2.w;
-                    w[12] = v3.x; w[13] = v3.y; w[14] = v3.z; w[15] = v3.w;
-                    tmem_st16(tmem + lane_off + kColQ + 16 * c, w);
-                }
-                {
-                    const uint4 v0 = src[(512 + 32 * rank) / 8 + 0];
-                    const uint4 v1 = src[(512 + 32 * rank) / 8 + 1];
-                    const uint4 v2 = src[(512 + 32 * rank) / 8 + 2];
-                    const uint4 v3 = src[(512 + 32 * rank) / 8 + 3];
-                    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-                    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-                    w[8] = v2.x; w[9] = v2.y; w[10] = v2.z; w[11] = v2.w;
-                    w[12] = v3.x; w[13] = v3.y; w[14] = v3.z; w[15] = v3.w;
-                    tmem_st16(tmem + lane_off + kColQ + 128, w);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&q_ready);
-            }
-            float m = -INFINITY, l = 0.f;
-            const int T = item.t1 - item.t0;
-            for (int k = 0; k < T && ok; ++k) {
-                const uint32_t g = it + k;
-                const int key0 = (item.t0 + k) * kAttnKeys;
-                const int valid = min(kAttnKeys, item.n_vis - key0);
-                if (!mbar_wait(&s_full, g & 1, abort)) { ok = false; break; }
-                tc_fence_after();
-                float sc[64];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColS + 16 * c, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) sc[16 * c + i] = __uint_as_float(r[i]);
-                }
-                tc_fence_before();
-                mbar_arrive(&s_free);
-                // partial scores to the peer, then the peer's partial for this row
-                const uint32_t xb = (g & 1) * kXBytes + h * kXRow;
-#pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    st_cluster_v4(x_peer + xb + 16 * c, sc[4 * c], sc[4 * c + 1], sc[4 * c + 2], sc[4 * c + 3]);
-                mbar_arrive_peer(xbar_peer[g & 1]);
-                if (!mbar_wait<true>(&x_full[g & 1], (g >> 1) & 1, abort)) { ok = false; break; }
-                float mx = -INFINITY;
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const float4 v = ld_shared_v4(x_local + xb + 16 * c);
-                    const float t4[4] = {v.x, v.y, v.z, v.w};
+                for (int c = 0; c < 8; ++c) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int n = 4 * c + i;
-                        const float s = (sc[n] + t4[i]) * a.scale_log2;
-                        sc[n] = n < valid ? s : -INFINITY;
-                        mx = fmaxf(mx, sc[n]);
+                        const uint4 v = src[32 * rank + 4 * c + i];
+                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                    }
+                    tmem_st16(tmem + lane_off + kColQ + 16 * c, w);
+                }
+                const uint32_t qrow = sbase + kOffQr + h * 64;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 v = src[64 + 4 * rank + c];
+                    st_shared_u4(qrow + ((c ^ ((h >> 1) & 3)) << 4), v.x, v.y, v.z, v.w);
+                }
+                tmem_wait_st();
+                fence_async_smem();
+                tc_fence_before();
+                named_barrier(1, 128);
+                if (leader) mbar_arrive(&q_ready);
+            }
+            const int T = item.t1 - item.t0;
+            bool stop = false;
+            for (int k = 0; k < T; ++k) {
+                const uint32_t g = it + k;
+                const int sb = g & 1;
+                if (leader) {
+                    // score tile g ready; the peer's buffer sb was read (tile g - 2)
+                    bool ok = mbar_wait(&s_full[sb], (g >> 1) & 1, abort);
+                    if (ok && g >= 2) ok = mbar_wait<true>(&rx_done[sb], ((g >> 1) - 1) & 1, abort);
+                    if (!ok) fail();
+                    ex_stop = *abort;
+                }
+                named_barrier(1, 128);
+                if (ex_stop) { stop = true; break; }
+                tc_fence_after();
+                // my raw partial scores rounded to fp16, stored straight into the peer's
+                // buffer (the peer adds exactly these values; so do I)
+                const uint32_t row = xin_peer + sb * kTileBytes + h * 128;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32 * half, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t hw[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            __half2 v = __floats2half2_rn(__uint_as_float(r[8 * c + 2 * i]), __uint_as_float(r[8 * c + 2 * i + 1]));
+                            hw[i] = *reinterpret_cast<uint32_t*>(&v);
+                        }
+                        const int chunk = 4 * half + c;
+                        st_async_u4(row + ((chunk ^ (h & 7)) << 4), hw[0], hw[1], hw[2], hw[3], xbar_peer[sb]);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sb]);
+            }
+            if (stop) break;
+            it += T;
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warpgroups
+        // Two threads per head row: warp w serves TMEM lane quarter w % 4 and
+        // score columns [32c, 32c + 32) with c = (w - 6) / 4.  The two halves
+        // share the row maximum through smem each tile and keep separate
+        // running sums, combined once per item.
+        const int q = warp & 3;
+        const int ch = (warp - 6) >> 2;               // column half
+        const int h = q * 32 + lane;
+        const int tid = threadIdx.x - 192;            // 0..255
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t rx_peer[2] = {map_peer(smem_u32(&rx_done[0]), peer), map_peer(smem_u32(&rx_done[1]), peer)};
+        const bool leader = (warp == 6) && lane == 0;
+        // O GEMM of global tile n has completed.  Completions alternate between two
+        // barriers, and the next completion on o_done[n & 1] (tile n + 2) needs a P
+        // tile not yet written whenever this is called, so the phase parity is exact.
+        auto wait_o = [&](uint32_t n) -> bool { return mbar_wait(&o_done[n & 1], (n >> 1) & 1, abort); };
+        ItemIter iter;
+        iter.init(a, pair);
+        Item item;
+        uint32_t it = 0;
+        while (iter.next(item)) {
+            if (leader) sm_top = *abort;
+            named_barrier(2, 256);
+            if (sm_top) break;
+            float m = -INFINITY, l = 0.f;             // l: this thread's half of the row sum
+            const int T = item.t1 - item.t0;
+            bool stop = false;
+            for (int k = 0; k < T; ++k) {
+                const uint32_t g = it + k;
+                const int sb = g & 1;
+                const int key0 = (item.t0 + k) * kKeys;
+                const int valid = min(kKeys, item.n_vis - key0);
+                if (leader) {
+                    mbar_expect_tx(&xin_full[sb], kTileBytes);
+                    if (!(mbar_wait<true>(&xin_full[sb], (g >> 1) & 1, abort) && mbar_wait(&s_full[sb], (g >> 1) & 1, abort)))
+                        fail();
+                    sm_stop = *abort;
+                }
+                named_barrier(2, 256);
+                if (sm_stop) { stop = true; break; }
+                // own partial (TMEM, rounded to fp16 exactly as sent to the peer) and the
+                // peer's fp16 partial for this row half (chunks 4c .. 4c + 3)
+                tc_fence_after();
+                uint32_t own[32];
+                tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32 * ch, own);
+                tmem_wait_ld();
+                tc_fence_before();
+                uint4 oth[4];
+                const uint32_t prow = sbase + kOffXin + sb * kTileBytes + h * 128;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) oth[c] = ld_shared_u4(prow + (((4 * ch + c) ^ (h & 7)) << 4));
+                // raw score = own fp32 partial + the peer's fp16 partial
+                float x[32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t pw[4] = {oth[c].x, oth[c].y, oth[c].z, oth[c].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = 8 * c + 2 * i;
+                        const float2 b2 = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
+                        x[n] = __uint_as_float(own[n]) + b2.x;
+                        x[n + 1] = __uint_as_float(own[n + 1]) + b2.y;
+                    }
+                }
+                if (valid < kKeys) {
+#pragma unroll
+                    for (int n = 0; n < 32; ++n) x[n] = (32 * ch + n) < valid ? x[n] : -INFINITY;
+                }
+                float mx8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24]));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
+                // softmax in base 2: scores scaled by scale * log2(e) (> 0, so the raw max serves)
+                const float mx_half = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
+                row_max[ch][h] = mx_half;
+                // everyone has read the exchange buffers and published its half maximum;
+                // P buffer g & 1 is free once O GEMM g-2 completed
+                if (leader) {
+                    if (g >= 2 && !wait_o(g - 2)) fail();
+                    sm_stop2 = *abort;
+                }
+                named_barrier(2, 256);
+                if (sm_stop2) { stop = true; break; }
+                if (leader) {
+                    // every thread's reads of the exchange buffer returned before the barrier
+                    mbar_arrive(&s_free[sb]);
+                    mbar_arrive_peer_relaxed(rx_peer[sb]);
+                }
+                tc_fence_after();
+                const float mx = fmaxf(mx_half, row_max[ch ^ 1][h]);
                 const float m_new = fmaxf(m, mx);
-                if (m_new > m + kRescaleThreshold) {
-                    const float alpha = exp2f(m - m_new);
-                    if (k > 0) {
-                        if (!wait_o(g - 1)) { ok = false; break; }
+                // Lazy rescaling: only when the row maximum grew by more than 2^8.
+                // The TMEM accesses are warp-collective, so the decision is made per
+                // warp; lanes that need no rescale multiply by 1.
+                const bool need = m_new > m + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need) && k > 0) {
+                        // O must hold every earlier tile: O GEMM g-1 has to be complete.
+                    int ok = 1;
+                    if (lane == 0) {
+                        ok = wait_o(g - 1) ? 1 : 0;
+                        if (!ok) fail();
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (ok) {
                         tc_fence_after();
+                        const float alpha = need ? ex2(m - m_new) : 1.f;
 #pragma unroll 1
-                        for (int c = 0; c < 16; ++c) {
+                        for (int c = 0; c < 8; ++c) {
                             uint32_t r[16];
-                            tmem_ld16(tmem + lane_off + kColO + 16 * c, r);
+                            const uint32_t ta = tmem + lane_off + kColO + 128 * ch + 16 * c;
+                            tmem_ld16(ta, r);
                             tmem_wait_ld();
 #pragma unroll
                             for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                            tmem_st16(tmem + lane_off + kColO + 16 * c, r);
+                            tmem_st16(ta, r);
                         }
                         tmem_wait_st();
                     }
-                    l *= alpha;
+                }
+                if (need) {
+                    l *= ex2(m - m_new);
                     m = m_new;
                 }
-                // P buffer (g & 1) is free once the O GEMM of tile g - 2 completed
-                if (g >= 2 && !wait_o(g - 2)) { ok = false; break; }
-                if (valid < kAttnKeys) {
+                if (valid < kKeys) {
                     // rows past the visible keys may hold anything: zero them for the O GEMM
                     const uint32_t st = sbase + (g % kStages) * kStageBytes;
-                    const int nchunks = (kAttnKeys - valid) * 32;
-                    for (int i = tid; i < nchunks; i += 128) {
-                        const int row = valid + (i >> 5), box = (i >> 3) & 3, ch = i & 7;
-                        st_shared_v4(st + box * kLatBox + row * 128 + ch * 16, 0u, 0u, 0u, 0u);
+                    const int nchunks = (kKeys - valid) * 32;
+                    for (int i = tid; i < nchunks; i += 256) {
+                        const int r = valid + (i >> 5), box = (i >> 3) & 3, c = i & 7;
+                        st_shared_u4(st + box * kLatBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
                     }
                 }
-                const uint32_t prow = sbase + kOffP + (g & 1) * kPBytes + h * 128;
-                float psum = 0.f;
+                const uint32_t pr = sbase + kOffP + (g & 1) * kTileBytes + h * 128;
+                float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) {
                     uint32_t pw[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const __nv_bfloat162 p2 =
-                            __floats2bfloat162_rn(exp2f(sc[8 * c + 2 * i] - m), exp2f(sc[8 * c + 2 * i + 1] - m));
-                        const float2 f2 = __bfloat1622float2(p2);
-                        psum += f2.x + f2.y;
-                        pw[i] = *reinterpret_cast<const uint32_t*>(&p2);
+                        const float p0 = ex2(fmaf(x[8 * c + 2 * i], a.scale_log2, -m));
+                        const float p1 = ex2(fmaf(x[8 * c + 2 * i + 1], a.scale_log2, -m));
+                        ps[i] += p0 + p1;
+                        pw[i] = pack_bf16(p0, p1);
                     }
-                    st_shared_v4(prow + ((c ^ (h & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                    st_shared_u4(pr + (((4 * ch + c) ^ (h & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                 }
-                l += psum;
+                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
                 fence_async_smem();
-                mbar_arrive(&p_ready[g & 1]);
+                tc_fence_before();
+                named_barrier(2, 256);
+                if (leader) mbar_arrive(&p_ready[g & 1]);
             }
-            if (!ok) break;
+            if (stop) break;
             // epilogue: normalised latent half (or partial + log2-sum-exp)
-            const uint32_t g_last = it + T - 1;
-            if (!wait_o(g_last)) { ok = false; break; }
+            row_sum[ch][h] = l;
+            if (leader) {
+                if (!wait_o(it + T - 1)) fail();
+                sm_stop = *abort;
+            }
+            named_barrier(2, 256);
+            if (sm_stop) break;
             tc_fence_after();
-            const float inv = 1.f / l;
+            const float lsum = row_sum[0][h] + row_sum[1][h];
+            const float inv = 1.f / lsum;
             if (item.slot < 0) {
-                uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ((int64_t)item.bj * 128 + h) * 512 + 256 * rank);
+                uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ((int64_t)item.bj * 128 + h) * 512 + 256 * rank + 128 * ch);
 #pragma unroll 1
-                for (int c = 0; c < 16; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColO + 16 * c, r);
+                    tmem_ld16(tmem + lane_off + kColO + 128 * ch + 16 * c, r);
                     tmem_wait_ld();
                     uint32_t pk[8];
 #pragma unroll
@@ -444,11 +613,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     dst[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
             } else {
-                float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)item.slot * 128 + h) * 512 + 256 * rank);
+                float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)item.slot * 128 + h) * 512 + 256 * rank +
+                                                        128 * ch);
 #pragma unroll 1
-                for (int c = 0; c < 16; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColO + 16 * c, r);
+                    tmem_ld16(tmem + lane_off + kColO + 128 * ch + 16 * c, r);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -456,12 +626,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                                                      __uint_as_float(r[4 * i + 2]) * inv,
                                                      __uint_as_float(r[4 * i + 3]) * inv);
                 }
-                if (rank == 0) a.part_lse[item.slot * 128 + h] = m + log2f(l);
+                if (rank == 0 && ch == 0) a.part_lse[item.slot * 128 + h] = m + __log2f(lsum);
             }
             tc_fence_before();
             it += T;
         }
-        if (!ok) fail();
     }
 
     tc_fence_before();
@@ -470,7 +639,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    cluster_sync();          // no CTA leaves while its peer may still write to it
+    cluster_sync();          // no CTA leaves while its peer may still access it
 }
 
 }  // namespace

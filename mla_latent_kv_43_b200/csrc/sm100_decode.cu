@@ -52,28 +52,43 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
     if (pf == pl) return;            // finished inside one cluster
     // clusters with an empty tile range between the first and the last piece hold nothing
     auto empty = [&](int p) { return start(p) == (p + 1 < pairs ? start(p + 1) : T); };
-    float M = -INFINITY;
-    for (int p = pf; p <= pl; ++p) {
-        if (p != pf && empty(p)) continue;
-        const int slot = p == pf ? 2 * p + 1 : 2 * p;
-        M = fmaxf(M, part_lse[slot * kHeads + h]);
-    }
+    constexpr int kMaxPieces = 16;
+    int slots[kMaxPieces];
+    int np = 0;
     float acc[16];
     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
     float wsum = 0.f;
-    for (int p = pf; p <= pl; ++p) {
-        if (p != pf && empty(p)) continue;
-        const int slot = p == pf ? 2 * p + 1 : 2 * p;
-        const float w = exp2f(part_lse[slot * kHeads + h] - M);
-        wsum += w;
-        const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slot * kHeads + h) * kDc + col);
+    float M = -INFINITY;
+    // pieces in batches of up to kMaxPieces: log-sum-exps first (independent loads), then rows
+    for (int p0 = pf; p0 <= pl;) {
+        np = 0;
+        for (; p0 <= pl && np < kMaxPieces; ++p0)
+            if (p0 == pf || !empty(p0)) slots[np++] = p0 == pf ? 2 * p0 + 1 : 2 * p0;
+        float lse[kMaxPieces];
+        float Mb = M;
+        for (int i = 0; i < np; ++i) {
+            lse[i] = part_lse[slots[i] * kHeads + h];
+            Mb = fmaxf(Mb, lse[i]);
+        }
+        // rescale what was accumulated so far to the new maximum
+        const float r = (M == -INFINITY) ? 0.f : exp2f(M - Mb);
+        wsum *= r;
+        for (int i = 0; i < 16; ++i) acc[i] *= r;
+        M = Mb;
+        for (int i = 0; i < np; ++i) {
+            const float w = exp2f(lse[i] - M);
+            wsum += w;
+            const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slots[i] * kHeads + h) * kDc + col);
+            float4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float4 v = src[i];
-            acc[4 * i] = fmaf(w, v.x, acc[4 * i]);
-            acc[4 * i + 1] = fmaf(w, v.y, acc[4 * i + 1]);
-            acc[4 * i + 2] = fmaf(w, v.z, acc[4 * i + 2]);
-            acc[4 * i + 3] = fmaf(w, v.w, acc[4 * i + 3]);
+            for (int k = 0; k < 4; ++k) v[k] = src[k];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                acc[4 * k] = fmaf(w, v[k].x, acc[4 * k]);
+                acc[4 * k + 1] = fmaf(w, v[k].y, acc[4 * k + 1]);
+                acc[4 * k + 2] = fmaf(w, v[k].z, acc[4 * k + 2]);
+                acc[4 * k + 3] = fmaf(w, v[k].w, acc[4 * k + 3]);
+            }
         }
     }
     const float inv = 1.f / wsum;

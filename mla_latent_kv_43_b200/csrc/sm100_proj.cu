@@ -27,8 +27,6 @@ namespace sm100 {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kStages = 4;
-constexpr int kStageBytes = 32768;   // A k-block (16 KB) + B k-block (<= 16 KB)
 constexpr int kKeysPerTile = 64;
 
 struct ProjArgs {
@@ -43,11 +41,6 @@ struct ProjArgs {
     // upproj
     __nv_bfloat16* out;
     int32_t* status;
-};
-
-template <int MODE>  // 0: absorb, 1: upproj
-struct ProjShape {
-    static constexpr int kBlocks = MODE == 0 ? 2 : 8;   // K / 64
 };
 
 __device__ void plan_tiles(const ProjArgs& a, int tid) {
@@ -83,28 +76,41 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
     }
 }
 
-template <int MODE>
+__host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
+    return n <= 32 ? 32u : (n <= 64 ? 64u : (n <= 128 ? 128u : (n <= 256 ? 256u : 512u)));
+}
+
+// Thread 0 waits for `bar` (bounded); the block learns the outcome through
+// smem after a __syncthreads, so no warp diverges on a timeout.
+__device__ bool block_wait(uint64_t* bar, int* flag, int32_t* status) {
+    if (threadIdx.x == 0) {
+        *flag = mbar_wait(bar, 0, nullptr) ? 1 : 0;
+        if (!*flag) set_status(status, MLA_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
+// One CTA per (head, token tile): the whole W_uk[h] (4 row tiles x 2 k-blocks,
+// 128 KB) and the token tile's q_nope arrive in one batch of TMA loads; the 4
+// row tiles accumulate side by side in TMEM (4 x N columns).
 __global__ void __launch_bounds__(kThreads, 1)
-proj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, ProjArgs a) {
-    constexpr int KB = ProjShape<MODE>::kBlocks;
+absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, ProjArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[kStages], empty[kStages], done;
+    __shared__ uint64_t full, done;
     __shared__ uint32_t tmem_base;
-    __shared__ int abort_flag;
-
-    const int h = blockIdx.x, mt = blockIdx.y, nt = blockIdx.z;
+    __shared__ int flag;
+    const int h = blockIdx.x, nt = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = a.n_tile;
-    const uint32_t ncols = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+    const uint32_t ncols = tmem_cols_for(4 * N);
+    uint8_t* sA = smem;                    // [mt][kb] 16 KB boxes
+    uint8_t* sB = smem + 8 * 16384;        // [kb] N x 128 B
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
+        mbar_init(&full, 1);
         mbar_init(&done, 1);
-        abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -115,98 +121,84 @@ proj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
-    const uint32_t a_bytes = 16384, b_bytes = (uint32_t)N * 128;
 
-    if (warp == 0) {
-        if (elect_one()) {
-            tma_prefetch(&mapA);
-            tma_prefetch(&mapB);
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages;
-                if (kb >= kStages && !mbar_wait(&empty[s], ((kb / kStages) - 1) & 1, &abort_flag)) {
-                    abort_flag = 1;
-                    break;
-                }
-                uint8_t* sa = smem + s * kStageBytes;
-                uint8_t* sb = sa + 16384;
-                mbar_expect_tx(&full[s], a_bytes + b_bytes);
-                if (MODE == 0) {
-                    tma_load_2d(sa, &mapA, &full[s], kb * 64, h * 512 + mt * 128);
-                } else {
-                    tma_load_2d(sa, &mapA, &full[s], 0, h * 512 + kb * 64);
-                    tma_load_2d(sa + 8192, &mapA, &full[s], 64, h * 512 + kb * 64);
-                }
-                tma_load_3d(sb, &mapB, &full[s], kb * 64, h, nt * N);
-            }
+    if (warp == 0 && elect_one()) {
+        mbar_expect_tx(&full, 8 * 16384 + 2 * N * 128);
+        for (int kb = 0; kb < 2; ++kb) {
+            tma_load_3d(sB + kb * N * 128, &mapB, &full, kb * 64, h, nt * N);
+            for (int mt = 0; mt < 4; ++mt)
+                tma_load_2d(sA + (mt * 2 + kb) * 16384, &mapA, &full, kb * 64, h * 512 + mt * 128);
         }
-    } else if (warp == 1) {
-        if (elect_one()) {
-            const uint32_t idesc = idesc_bf16(128, N, MODE == 1, false);
-            bool ok = true;
-            for (int kb = 0; kb < KB && ok; ++kb) {
-                const int s = kb % kStages;
-                if (!mbar_wait(&full[s], (kb / kStages) & 1, &abort_flag)) {
-                    abort_flag = 1;
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t sa = smem_u32(smem + s * kStageBytes), sb = sa + 16384;
+    } else if (warp == 1 && elect_one()) {
+        if (mbar_wait(&full, 0, nullptr)) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, N, false, false);
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+            for (int mt = 0; mt < 4; ++mt)
+                for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = MODE == 0 ? sdesc(sa + ks * 32, 16, 1024, kSwizzle128)
-                                                  : sdesc(sa + ks * 2048, 8192, 1024, kSwizzle128);
-                    const uint64_t bd = sdesc(sb + ks * 32, 16, 1024, kSwizzle128);
-                    mma_ss(tmem, ad, bd, idesc, (kb | ks) ? 1u : 0u);
-                }
-                mma_commit(&empty[s]);
-            }
-            mma_commit(&done);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(tmem + mt * N, sdesc(a0 + (mt * 2 + kb) * 16384 + ks * 32, 16, 1024, kSwizzle128),
+                               sdesc(b0 + kb * N * 128 + ks * 32, 16, 1024, kSwizzle128), idesc,
+                               (kb | ks) ? 1u : 0u);
         }
+        mma_commit(&done);
     }
     __syncwarp();
 
-    // absorb extras while the MMAs run: query RoPE and the key-tile plan
-    if (MODE == 0) {
-        if (mt == 0) {
-            for (int t = threadIdx.x; t < N * 32; t += kThreads) {
-                const int n = nt * N + t / 32, r = t % 32;
-                if (n >= a.BJ) continue;
-                const int b = n / a.n_q, j = n % a.n_q;
-                const int64_t p = query_pos(a.seq_lens[b], a.n_q, j);
-                const __nv_bfloat16* qr = a.q_rope + ((int64_t)n * a.H + h) * 64;
+    // query RoPE (one thread per token row, vector loads/stores) and the
+    // key-tile plan while the MMAs run
+    __shared__ double theta[32];
+    if (threadIdx.x < 32) theta[threadIdx.x] = pow((double)a.rope_base, -2.0 * threadIdx.x / 64.0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < N; t += kThreads) {
+        const int n = nt * N + t;
+        if (n >= a.BJ) break;
+        const int b = n / a.n_q, j = n % a.n_q;
+        const int64_t p = query_pos(a.seq_lens[b], a.n_q, j);
+        const uint4* src = reinterpret_cast<const uint4*>(a.q_rope + ((int64_t)n * a.H + h) * 64);
+        uint4* dst = reinterpret_cast<uint4*>(a.q_lat + ((int64_t)n * a.H + h) * 576 + 512);
+        uint4 v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = src[c];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
                 float y0, y1;
-                rope_pair(__bfloat162float(qr[2 * r]), __bfloat162float(qr[2 * r + 1]), p, r, 64, a.rope_base, &y0,
-                          &y1);
-                __nv_bfloat16* dst = a.q_lat + ((int64_t)n * a.H + h) * 576 + 512 + 2 * r;
-                dst[0] = __float2bfloat16_rn(y0);
-                dst[1] = __float2bfloat16_rn(y1);
+                rope_pair_theta(x.x, x.y, p, theta[4 * c + i], &y0, &y1);
+                w[i] = pack_bf16(y0, y1);
+            }
+            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+    if (h == 0 && nt == 0) plan_tiles(a, threadIdx.x);
+
+    if (block_wait(&done, &flag, a.status)) {
+        // TMEM row m of tile mt holds q_lat[n][h][128 mt + m] for the N tokens;
+        // stage as [n][512] bf16 in smem (the operand area is free now), then
+        // write each token's 1 KB row with 16-byte stores.
+        tc_fence_after();
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);
+        const int m = warp * 32 + lane;
+        for (int mt = 0; mt < 4; ++mt) {
+            for (int c0 = 0; c0 < N; c0 += 16) {
+                uint32_t r[16];
+                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + mt * N + c0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    stage[(c0 + c) * 512 + mt * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[c]));
             }
         }
-        if (h == 0 && mt == 0 && nt == 0) plan_tiles(a, threadIdx.x);
-    }
-
-    // epilogue: TMEM row (32*warp + lane) -> bf16 outputs
-    const bool ok = mbar_wait(&done, 0, &abort_flag);
-    tc_fence_after();
-    if (!ok) {
-        if (threadIdx.x == 0) set_status(a.status, MLA_ERR_TIMEOUT);
-    } else {
-        const int m = warp * 32 + lane;
-        for (int c0 = 0; c0 < N; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const int n = nt * N + c0 + c;
-                if (c0 + c >= N || n >= a.BJ) continue;
-                const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(r[c]));
-                if (MODE == 0)
-                    a.q_lat[((int64_t)n * a.H + h) * 576 + mt * 128 + m] = v;
-                else
-                    a.out[((int64_t)n * a.H + h) * 128 + m] = v;
-            }
+        __syncthreads();
+        const int nvalid = min(N, a.BJ - nt * N);
+        for (int i = threadIdx.x; i < nvalid * 64; i += kThreads) {
+            const int n = i >> 6, c = i & 63;
+            reinterpret_cast<uint4*>(a.q_lat + ((int64_t)(nt * N + n) * a.H + h) * 576)[c] =
+                reinterpret_cast<const uint4*>(stage + n * 512)[c];
         }
     }
     tc_fence_before();
@@ -214,21 +206,97 @@ proj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CU
     if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
-int round_n(int bj) {
-    int n = bj < 128 ? bj : 128;
+// One CTA per (head, token tile of <= 64): out[n][h][v] = sum_i W_uv[h][i][v] o_lat[n][h][i].
+// A = W_uv[h] read MN-major (v contiguous), 8 k-blocks of 64 rows, all in flight.
+__global__ void __launch_bounds__(kThreads, 1)
+upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, ProjArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[8], done;
+    __shared__ uint32_t tmem_base;
+    __shared__ int flag;
+    const int h = blockIdx.x, nt = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int N = a.n_tile;
+    const uint32_t ncols = tmem_cols_for(N);
+    const int stage = 16384 + N * 128;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 8; ++i) mbar_init(&full[i], 1);
+        mbar_init(&done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0 && elect_one()) {
+        for (int kb = 0; kb < 8; ++kb) {
+            uint8_t* st = smem + kb * stage;
+            mbar_expect_tx(&full[kb], 16384 + N * 128);
+            tma_load_2d(st, &mapA, &full[kb], 0, h * 512 + kb * 64);
+            tma_load_2d(st + 8192, &mapA, &full[kb], 64, h * 512 + kb * 64);
+            tma_load_3d(st + 16384, &mapB, &full[kb], kb * 64, h, nt * N);
+        }
+    } else if (warp == 1 && elect_one()) {
+        const uint32_t idesc = idesc_bf16(128, N, true, false);
+        bool ok = true;
+        for (int kb = 0; kb < 8 && ok; ++kb) {
+            if (!mbar_wait(&full[kb], 0, nullptr)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sa = smem_u32(smem + kb * stage), sb = sa + 16384;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ss(tmem, sdesc(sa + ks * 2048, 8192, 1024, kSwizzle128), sdesc(sb + ks * 32, 16, 1024, kSwizzle128),
+                       idesc, (kb | ks) ? 1u : 0u);
+        }
+        mma_commit(&done);
+    }
+    __syncwarp();
+
+    if (block_wait(&done, &flag, a.status)) {
+        // stage out[n][h][0:128] as [n][128] bf16 in smem, then 16-byte stores
+        tc_fence_after();
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);
+        const int m = warp * 32 + lane;
+        for (int c0 = 0; c0 < N; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) stage[(c0 + c) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[c]));
+        }
+        __syncthreads();
+        const int nvalid = min(N, a.BJ - nt * N);
+        for (int i = threadIdx.x; i < nvalid * 16; i += kThreads) {
+            const int n = i >> 4, c = i & 15;
+            reinterpret_cast<uint4*>(a.out + ((int64_t)(nt * N + n) * a.H + h) * 128)[c] =
+                reinterpret_cast<const uint4*>(stage + n * 128)[c];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, ncols);
+}
+
+int round_n(int bj, int cap) {
+    int n = bj < cap ? bj : cap;
     n = (n + 15) / 16 * 16;
     return n < 16 ? 16 : n;
 }
 
-template <int MODE>
-int launch(const CUtensorMap& A, const CUtensorMap& B, const ProjArgs& a, dim3 grid, cudaStream_t st,
-           const char* name, int* launches) {
-    const size_t smem = kStages * kStageBytes + 1024;
-    if (cudaFuncSetAttribute(proj_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+template <typename K>
+int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs& a, dim3 grid, size_t smem,
+           cudaStream_t st, const char* name, int* launches) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(st, name);
-    proj_kernel<MODE><<<grid, kThreads, smem, st>>>(A, B, a);
+    kernel<<<grid, kThreads, smem, st>>>(A, B, a);
     prof_end(st);
     if (launches) ++*launches;
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
@@ -238,7 +306,7 @@ int launch(const CUtensorMap& A, const CUtensorMap& B, const ProjArgs& a, dim3 g
 
 // absorb + q-RoPE + plan.  q_nope [BJ][H][128], W_uk [H][512][128], q_rope [BJ][H][64]
 int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* launches) {
-    const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ);
+    const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 128);
     CUtensorMap A, B;
     {
         const uint64_t dims[2] = {128, (uint64_t)H * 512}, str[1] = {128 * 2};
@@ -263,13 +331,13 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* 
     a.q_lat = q_lat;
     a.cum = cum;
     a.status = c.status;
-    const dim3 grid(H, 4, (BJ + N - 1) / N);
-    return launch<0>(A, B, a, grid, c.stream, "sm100_absorb", launches);
+    const dim3 grid(H, 1, (BJ + N - 1) / N);
+    return launch(absorb_kernel, A, B, a, grid, 8 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches);
 }
 
 // up-projection.  o_lat [BJ][H][512] bf16, W_uv [H][512][128], out [BJ][H][128]
 int launch_upproj(const DecodeCall& c, const __nv_bfloat16* o_lat, int* launches) {
-    const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ);
+    const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 64);
     CUtensorMap A, B;
     {
         const uint64_t dims[2] = {128, (uint64_t)H * 512}, str[1] = {128 * 2};
@@ -289,7 +357,7 @@ int launch_upproj(const DecodeCall& c, const __nv_bfloat16* o_lat, int* launches
     a.out = (__nv_bfloat16*)c.out;
     a.status = c.status;
     const dim3 grid(H, 1, (BJ + N - 1) / N);
-    return launch<1>(A, B, a, grid, c.stream, "sm100_upproj", launches);
+    return launch(upproj_kernel, A, B, a, grid, 8 * (16384 + N * 128) + 1024, c.stream, "sm100_upproj", launches);
 }
 
 }  // namespace sm100
