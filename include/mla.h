@@ -162,6 +162,35 @@ MLA_API int mla_decode(const mla_dims* dims, int32_t batch, int32_t n_q,
                void* out, void* workspace, size_t workspace_bytes, int32_t splits,
                int32_t* status, void* stream);
 
+/* Size of the fixed scratch area behind mla_decode_noalloc. */
+#define MLA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* mla_decode without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code that runs where cudaMalloc is not allowed or
+ * must not block (inside an allocator-free serving loop, a plugin that may
+ * only use memory its host framework hands it, a real-time thread that cannot
+ * risk the device-wide synchronisation an allocation may cause).  It has no
+ * counterpart on the pages; it is a packaging variant of mla_decode.
+ *
+ * Arguments and results are those of mla_decode minus workspace and
+ * workspace_bytes.  The workspace is a fixed MLA_NOALLOC_SCRATCH_BYTES static
+ * device array inside the library: every GPU that loads the library holds it
+ * until the process exits, and the call allocates nothing.  A request whose
+ * workspace (mla_decode_workspace_bytes with the same sizes and splits) would
+ * exceed it returns MLA_ERR_WORKSPACE; pass a small `splits` (for example 4)
+ * to fit larger batches, since split-KV partial results dominate the size.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents (no
+ * region needs clearing: each is written before it is read), so calls whose
+ * execution overlaps on the GPU -- on different streams, or from different
+ * host threads -- race with each other; serialise them. */
+MLA_API int mla_decode_noalloc(const mla_dims* dims, int32_t batch, int32_t n_q,
+                               const void* q_nope, const void* q_rope, const void* W_uk,
+                               const void* W_uv, const void* cache, int64_t capacity,
+                               const int32_t* seq_lens, int64_t max_len, void* out,
+                               int32_t splits, int32_t* status, void* stream);
+
 /* Waits for `stream`, copies the status word to *host_status and resets it to
  * MLA_OK.  Returns MLA_OK or MLA_ERR_CUDA. */
 MLA_API int mla_get_status(int32_t* status, void* stream, int32_t* host_status);

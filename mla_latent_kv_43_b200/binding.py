@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.mla_status_string.restype = ctypes.c_char_p
         L.mla_last_launch_count.argtypes = []
         L.mla_last_launch_count.restype = ctypes.c_int32
+        L.mla_decode_noalloc.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, I32, P, P]
+        L.mla_decode_noalloc.restype = ctypes.c_int
         L.mla_profile_enable.argtypes = [ctypes.c_int]
         L.mla_profile_enable.restype = ctypes.c_int
         L.mla_profile_read.argtypes = [ctypes.c_char_p, SZ, ctypes.POINTER(ctypes.c_int32),
@@ -147,6 +149,19 @@ def mla_decode(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: 
                             _ptr(W_uv), _ptr(cache), cache.shape[1], _ptr(seq_lens), max_len,
                             _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             splits, _ptr(status), _stream(stream)), "mla_decode")
+
+
+def mla_decode_noalloc(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor,
+                       W_uv: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor, max_len: int,
+                       out: torch.Tensor, status: torch.Tensor, splits: int, stream=None):
+    """mla_decode with the library's fixed scratch area instead of a workspace."""
+    batch, n_q = q_nope.shape[0], q_nope.shape[1]
+    _check(lib().mla_decode_noalloc(ctypes.byref(dims), batch, n_q, _ptr(q_nope), _ptr(q_rope), _ptr(W_uk),
+                                    _ptr(W_uv), _ptr(cache), cache.shape[1], _ptr(seq_lens), max_len,
+                                    _ptr(out), splits, _ptr(status), _stream(stream)), "mla_decode_noalloc")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def mla_get_status(status: torch.Tensor, stream=None) -> int:
