@@ -94,8 +94,8 @@ struct ItemIter {
         lens = a.seq_lens;
         pair = p;
         const int T = cum[BJ];
-        s0 = (int)((int64_t)p * T / a.pairs);
-        s1 = (int)((int64_t)(p + 1) * T / a.pairs);
+        s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
+        s1 = (int)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
         int lo = 0, hi = BJ;          // first bj with cum[bj + 1] > s0
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
@@ -215,6 +215,8 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     __syncthreads();
     cluster_sync();          // the peer's barriers are initialised before any remote access
     tc_fence_after();
+    grid_dep_wait();         // q_lat and the tile plan come from the previous kernel
+    grid_dep_trigger();
     const uint32_t tmem = tmem_base;
     const uint32_t sbase = smem_u32(smem);
     volatile int* abort = &abort_flag;
@@ -668,10 +670,10 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
     if (cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(c.stream, "sm100_attend");
-    attend_kernel<<<2 * pairs, kThreads, smem, c.stream>>>(ml, mr, a);
+    const cudaError_t e = launch_pdl(attend_kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, ml, mr, a);
     prof_end(c.stream);
     if (launches) ++*launches;
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace sm100

@@ -10,6 +10,7 @@
 #include "internal.h"
 #include "profile.h"
 #include "sm100_host.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace sm100 {
@@ -29,6 +30,8 @@ constexpr int kHeads = 128, kDc = 512;
 __global__ void __launch_bounds__(128)
 combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* __restrict__ part_o,
                const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat) {
+    grid_dep_wait();
+    grid_dep_trigger();
     const int bj = blockIdx.x;
     const int T = cum[BJ];
     const int c0 = cum[bj], c1 = cum[bj + 1];
@@ -39,7 +42,8 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
         for (int i = 0; i < 16; ++i) dst[i] = __float2bfloat16_rn(0.f);
         return;
     }
-    auto start = [&](int p) { return (int)((int64_t)p * T / pairs); };
+    // cluster p covers key tiles [start(p), start(p + 1)); T * pairs fits 32 bits
+    auto start = [&](int p) { return (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)pairs); };
     auto pair_of = [&](int t) {      // largest p with start(p) <= t
         int lo = 0, hi = pairs - 1;
         while (lo < hi) {
@@ -151,10 +155,12 @@ int sm100_decode(const DecodeCall& c, int* launches) {
     if ((rc = sm100::launch_absorb(c, q_lat, cum, launches))) return rc;
     if ((rc = sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, P, launches))) return rc;
     prof_begin(c.stream, "sm100_combine");
-    sm100::combine_kernel<<<dim3(BJ, 128 / 4), 128, 0, c.stream>>>(cum, BJ, P, part_o, part_lse, o_lat);
+    const cudaError_t e = sm100::launch_pdl(sm100::combine_kernel, dim3(BJ, 128 / 4), dim3(128), 0, c.stream,
+                                            (const int32_t*)cum, BJ, P, (const float*)part_o,
+                                            (const float*)part_lse, o_lat);
     prof_end(c.stream);
     if (launches) ++*launches;
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return sm100::launch_upproj(c, o_lat, launches);
 }
 

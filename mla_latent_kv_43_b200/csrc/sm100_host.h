@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace mla {
 namespace sm100 {
 
@@ -15,6 +17,24 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims
 
 // Streaming multiprocessors of the current device (148 on B200 when unknown).
 int sm_count();
+
+// Launch with programmatic stream serialisation (the kernel overlaps its
+// prologue with the previous kernel and calls griddepcontrol.wait itself).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace sm100
 }  // namespace mla

@@ -122,6 +122,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = tmem_base;
 
+    // W_uk and q_nope are inputs: load and multiply before waiting for the
+    // previous kernel; the workspace (q_lat, plan) is written only after it.
     if (warp == 0 && elect_one()) {
         mbar_expect_tx(&full, 8 * 16384 + 2 * N * 128);
         for (int kb = 0; kb < 2; ++kb) {
@@ -146,6 +148,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     }
     __syncwarp();
 
+    grid_dep_wait();
+    grid_dep_trigger();
     // query RoPE (one thread per token row, vector loads/stores) and the
     // key-tile plan while the MMAs run
     __shared__ double theta[32];
@@ -236,13 +240,16 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     const uint32_t tmem = tmem_base;
 
     if (warp == 0 && elect_one()) {
+        // W_uv is an input: fetch it before waiting for the previous kernel
         for (int kb = 0; kb < 8; ++kb) {
             uint8_t* st = smem + kb * stage;
             mbar_expect_tx(&full[kb], 16384 + N * 128);
             tma_load_2d(st, &mapA, &full[kb], 0, h * 512 + kb * 64);
             tma_load_2d(st + 8192, &mapA, &full[kb], 64, h * 512 + kb * 64);
-            tma_load_3d(st + 16384, &mapB, &full[kb], kb * 64, h, nt * N);
         }
+        grid_dep_wait();         // o_lat comes from the previous kernels
+        for (int kb = 0; kb < 8; ++kb)
+            tma_load_3d(smem + kb * stage + 16384, &mapB, &full[kb], kb * 64, h, nt * N);
     } else if (warp == 1 && elect_one()) {
         const uint32_t idesc = idesc_bf16(128, N, true, false);
         bool ok = true;
@@ -258,6 +265,8 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
         mma_commit(&done);
     }
     __syncwarp();
+    grid_dep_wait();
+    grid_dep_trigger();
 
     if (block_wait(&done, &flag, a.status)) {
         // stage out[n][h][0:128] as [n][128] bf16 in smem, then 16-byte stores
@@ -296,10 +305,10 @@ int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs&
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(st, name);
-    kernel<<<grid, kThreads, smem, st>>>(A, B, a);
+    const cudaError_t e = launch_pdl(kernel, grid, dim3(kThreads), smem, st, A, B, a);
     prof_end(st);
     if (launches) ++*launches;
-    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace
