@@ -113,19 +113,31 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- helpers
-def barrier(world):
+def barrier(world, device="cuda"):
     if world > 1:
-        t = torch.ones(1, device="cuda")
+        t = torch.ones(1, device=device)
         dist.all_reduce(t)
-    torch.cuda.synchronize()
+    if device == "cuda":
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
+    """The slowest rank's value (every rank gets it)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_workload(w, rank: int):
+    """Rank r's shard: the same shapes, its own sequences (seed offset)."""
+    return w.with_(seed=w.seed + 1000 * rank) if rank else w
+
+
+def job_throughput(query_tokens_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job query tokens per second: every rank's tokens over the slowest rank's time."""
+    return query_tokens_per_rank * world / (ms_per_step_max * 1e-3)
 
 
 def source_sha(path: str) -> str:
@@ -220,7 +232,7 @@ def run_ours(a, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = gen.WORKLOADS[a.workload]
-    w_rank = w.with_(seed=w.seed + 1000 * rank) if rank else w
+    w_rank = shard_workload(w, rank)
     host = gen.generate(w_rank)
     stream = torch.cuda.current_stream()
     prob = DeviceProblem(w_rank, host, device=dev, splits=a.splits)
@@ -309,7 +321,7 @@ def run_ours(a, rank, world, local):
 
     ms_step = total_ms / a.steps
     qtok = work["query_tokens"] * world
-    value = qtok / (ms_step * 1e-3)
+    value = job_throughput(work["query_tokens"], world, ms_step)
     step_s = ms_step * 1e-3
     # dominant kernel
     kern = max(prof.items(), key=lambda kv: kv[1][1])
