@@ -17,8 +17,10 @@
 // Each CTA loads only its 288 columns of every tile (each cache byte crosses
 // HBM once, no multicast) and computes a partial score over them.  The
 // exchange warps round their partial to fp16 and store it straight into the
-// peer's shared memory (two buffers, so the exchange runs up to two tiles
-// ahead); each softmax thread adds its own fp32 partial to the peer's.  The
+// peer's shared memory (three buffers); each softmax thread adds its own
+// fp32 partial to the peer's, then writes its P values over the very chunks
+// it read, so the same buffer is the A operand of the O GEMM and returns to
+// the peer when that GEMM completes.  The
 // two CTAs' scores thus differ only by that fp16 rounding; each CTA keeps its
 // own running max and sum and normalises its own half of O with them, so each
 // half is self-consistent.  Each CTA accumulates its half of O from the same
@@ -57,10 +59,10 @@ constexpr int kStages = 4;
 constexpr int kLatBox = 8192;                      // 64 keys x 64 columns x 2 B
 constexpr int kRopeBox = 4096;                     // 64 keys x 32 columns x 2 B
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;
-constexpr int kTileBytes = 128 * 128;              // 128 rows x 64 x 2 B (P, exchange tiles)
-constexpr int kOffP = kStages * kStageBytes;       // two P buffers
-constexpr int kOffXin = kOffP + 2 * kTileBytes;    // two buffers, written by the peer
-constexpr int kOffQr = kOffXin + 2 * kTileBytes;   // 128 heads x 32 rope columns, SW64
+constexpr int kTileBytes = 128 * 128;              // 128 rows x 64 x 2 B (exchange / P tiles)
+constexpr int kXBufs = 3;                          // exchange buffers
+constexpr int kOffXin = kStages * kStageBytes;     // the peer's partial scores, then P
+constexpr int kOffQr = kOffXin + kXBufs * kTileBytes;  // 128 heads x 32 rope columns, SW64
 constexpr int kSmemBytes = kOffQr + 128 * 64;
 constexpr int kThreads = 448;
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kTmemCols = 512;
@@ -144,12 +146,6 @@ __device__ __forceinline__ void st_async_u4(uint32_t addr, uint32_t a, uint32_t 
                  : "memory");
 }
 
-// Relaxed arrive on a barrier of the peer CTA (no ordering of this thread's
-// earlier memory operations is implied).
-__device__ __forceinline__ void mbar_arrive_peer_relaxed(uint32_t peer_addr) {
-    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_addr) : "memory");
-}
-
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -174,12 +170,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kStages], empty[kStages];
     __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, drain;
-    __shared__ uint64_t p_ready[2], xin_full[2], rx_done[2];
+    __shared__ uint64_t p_ready[kXBufs], xin_full[kXBufs], rx_done[kXBufs];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
     // per-warpgroup decisions, each written by the leader before a named barrier
     // and read after it; a barrier separates every read from the next write
-    __shared__ int ex_stop, sm_stop, sm_stop2, sm_top;
+    __shared__ int ex_stop, sm_stop, sm_top;
     __shared__ float row_max[2][128], row_sum[2][128];   // softmax half-row exchange
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -195,15 +191,16 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&s_free[i], 5);       // 4 exchange warps + the softmax leader
+        }
+        for (int i = 0; i < kXBufs; ++i) {
             mbar_init(&xin_full[i], 1);     // my softmax leader's expect_tx + the peer's bytes
-            mbar_init(&rx_done[i], 1);      // the peer's softmax leader
+            mbar_init(&rx_done[i], 1);      // the peer's O GEMM has read the buffer (its commit)
+            mbar_init(&p_ready[i], 1);      // P tile written over the exchange buffer
         }
         mbar_init(&o_done[0], 1);           // O GEMMs of even / odd global tiles
         mbar_init(&o_done[1], 1);
         mbar_init(&q_ready, 1);
         mbar_init(&drain, 1);
-        mbar_init(&p_ready[0], 1);          // P tile of even / odd global tiles written
-        mbar_init(&p_ready[1], 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -260,93 +257,90 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         // ------------------------------------------------------------ MMA issuer
         // Two streams in tile order: score GEMMs S(g) and latent GEMMs O(g).
         // Each is issued as soon as its inputs are ready, so S runs ahead of O
-        // as far as the two S buffers allow.
-        if (elect_one()) {
-            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
-            const uint32_t qr = sbase + kOffQr;
-            ItemIter iterS, iterO;
-            iterS.init(a, pair);
-            iterO.init(a, pair);
-            Item itS, itO;
-            bool haveS = iterS.next(itS), haveO = iterO.next(itO);
-            int kS = 0, kO = 0;
-            uint32_t gS = 0, gO = 0, nItemsS = 0;
-            bool qS = false;                       // q_ready observed for the current S item
-            int sStep = -1;                        // K-step of the score GEMM in progress (-1: none)
-            uint64_t t_last = globaltimer();
-            bool ok = true;
-            while (ok && haveO) {
-                bool progressed = false;
-                // O GEMMs first: they release the stage and unblock the softmax two tiles later
-                if (gO < gS - (sStep >= 0 ? 1u : 0u) && mbar_ready(&p_ready[gO & 1], (gO >> 1) & 1)) {
-                    tc_fence_after();
-                    const int s = gO % kStages;
-                    const uint32_t st = sbase + s * kStageBytes;
+        // as far as the two S buffers allow.  The whole warp runs this loop
+        // (every decision is lane 0's observation, broadcast) and one elected
+        // lane issues each instruction.
+        constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
+        constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
+        // descriptors of stage 0 / P buffer 0; other stages and steps are byte offsets
+        const uint64_t dLatK = sdesc(sbase, 16, 1024, kSwizzle128);          // cache tile, K-major (score)
+        const uint64_t dLatN = sdesc(sbase, kLatBox, 1024, kSwizzle128);     // cache tile, MN-major (latent)
+        const uint64_t dRope = sdesc(sbase + 4 * kLatBox, 16, 512, kSwizzle64);
+        const uint64_t dQr = sdesc(sbase + kOffQr, 16, 512, kSwizzle64);
+        const uint64_t dP = sdesc(sbase + kOffXin, 16, 1024, kSwizzle128);
+        ItemIter iterS, iterO;
+        iterS.init(a, pair);
+        iterO.init(a, pair);
+        Item itS, itO;
+        bool haveS = iterS.next(itS), haveO = iterO.next(itO);
+        int kS = 0, kO = 0;
+        uint32_t gS = 0, gO = 0, nItemsS = 0;
+        bool qS = false;                           // q_ready observed for the current S item
+        uint32_t idle = 0;                         // consecutive passes without progress
+        uint64_t t_idle = 0;                       // timer at the 256th of them
+        bool ok = true;
+        while (ok && haveO) {
+            bool progressed = false;
+            // O GEMMs first: they release the stage and unblock the softmax two tiles later
+            if (gO < gS && mbar_ready_w(&p_ready[gO % kXBufs], (gO / kXBufs) & 1)) {
+                tc_fence_after();
+                const int s = gO % kStages;
+                const uint32_t so = s * kStageBytes, po = (gO % kXBufs) * kTileBytes;
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = sdesc(sbase + kOffP + (gO & 1) * kTileBytes + ks * 32, 16, 1024, kSwizzle128);
-                        const uint64_t bd = sdesc(st + ks * 2048, kLatBox, 1024, kSwizzle128);
-                        mma_ss(tmem + kColO, ad, bd, idO, (kO == 0 && ks == 0) ? 0u : 1u);
-                    }
-                    mma_commit(&empty[s]);
-                    mma_commit(&o_done[gO & 1]);
-                    ++gO;
-                    if (++kO == itO.t1 - itO.t0) {
-                        kO = 0;
-                        haveO = iterO.next(itO);
-                    }
-                    progressed = true;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ss_w(tmem + kColO, sdesc_add(dP, po + ks * 32), sdesc_add(dLatN, so + ks * 2048), idO,
+                             (kO == 0 && ks == 0) ? 0u : 1u);
+                mma_commit_w(&empty[s]);
+                mma_commit_w(&o_done[gO & 1]);
+                // P buffer gO % 3 is free again: the peer may send its tile gO + 3 into it
+                mma_commit_mc_w(&rx_done[gO % kXBufs], (uint16_t)(1u << peer));
+                ++gO;
+                if (++kO == itO.t1 - itO.t0) {
+                    kO = 0;
+                    haveO = iterO.next(itO);
                 }
-                // score GEMM S(gS), issued 6 K-steps at a time so a ready O is never held back long
-                if (haveS && sStep < 0) {
-                    const int s = gS % kStages, sb = gS & 1;
-                    if (!qS) qS = mbar_ready(&q_ready, nItemsS & 1);
-                    if (qS && mbar_ready(&full[s], (gS / kStages) & 1) &&
-                        (gS < 2 || mbar_ready(&s_free[sb], ((gS >> 1) - 1) & 1))) {
-                        tc_fence_after();
-                        sStep = 0;
-                        ++gS;                      // S(gS - 1) now in progress
-                    }
-                }
-                if (sStep >= 0) {
-                    const uint32_t g = gS - 1;
-                    const int s = g % kStages, sb = g & 1;
-                    const uint32_t st = sbase + s * kStageBytes;
+                progressed = true;
+            }
+            // score GEMM S(gS): 16 K-steps of latent (A = query slice in TMEM), 2 of rope
+            if (haveS) {
+                const int s = gS % kStages, sb = gS & 1;
+                if (!qS) qS = mbar_ready_w(&q_ready, nItemsS & 1);
+                if (qS && mbar_ready_w(&full[s], (gS / kStages) & 1) &&
+                    (gS < 2 || mbar_ready_w(&s_free[sb], ((gS >> 1) - 1) & 1))) {
+                    tc_fence_after();
+                    const uint32_t so = s * kStageBytes;
                     const uint32_t dS = tmem + kColS + 64 * sb;
-                    const int end = sStep + 6;
-                    for (; sStep < end; ++sStep) {
-                        if (sStep < 16) {
-                            const uint64_t bd = sdesc(st + (sStep >> 2) * kLatBox + (sStep & 3) * 32, 16, 1024, kSwizzle128);
-                            mma_ts(dS, tmem + kColQ + 8 * sStep, bd, idS, sStep ? 1u : 0u);
-                        } else {
-                            const uint64_t ad = sdesc(qr + (sStep - 16) * 32, 16, 512, kSwizzle64);
-                            const uint64_t bd = sdesc(st + 4 * kLatBox + (sStep - 16) * 32, 16, 512, kSwizzle64);
-                            mma_ss(dS, ad, bd, idS, 1u);
-                        }
-                    }
-                    if (sStep == 18) {
-                        mma_commit(&s_full[sb]);
-                        sStep = -1;
-                        if (++kS == itS.t1 - itS.t0) {
-                            kS = 0;
-                            qS = false;
-                            ++nItemsS;
-                            haveS = iterS.next(itS);
-                        }
+#pragma unroll
+                    for (int ks = 0; ks < 16; ++ks)
+                        mma_ts_w(dS, tmem + kColQ + 8 * ks, sdesc_add(dLatK, so + (ks >> 2) * kLatBox + (ks & 3) * 32),
+                                 idS, ks ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)
+                        mma_ss_w(dS, sdesc_add(dQr, ks * 32), sdesc_add(dRope, so + ks * 32), idS, 1u);
+                    mma_commit_w(&s_full[sb]);
+                    ++gS;
+                    if (++kS == itS.t1 - itS.t0) {
+                        kS = 0;
+                        qS = false;
+                        ++nItemsS;
+                        haveS = iterS.next(itS);
                     }
                     progressed = true;
-                }
-                if (progressed) {
-                    t_last = globaltimer();
-                } else if (*abort || globaltimer() - t_last > kWaitLimitNs) {
-                    ok = false;
                 }
             }
-            if (!ok) fail();
-            mma_commit(&drain);
-            mbar_wait(&drain, 0, nullptr);
+            // bounded idle time: the timer is read once per 256 idle passes
+            if (progressed) {
+                idle = 0;
+            } else if ((++idle & 255u) == 0) {
+                const uint64_t now = globaltimer();
+                if (idle == 256) t_idle = now;
+                const int quit = (*abort || now - t_idle > kWaitLimitNs) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, quit, 0)) ok = false;
+            }
         }
+        if (!ok && lane == 0) fail();
+        mma_commit_w(&drain);
+        mbar_wait(&drain, 0, nullptr);
     } else if (warp < 6) {
         // ------------------------------------------------------------ exchange warpgroup
         // One leader does every mbarrier wait (bounded) and a named barrier
@@ -355,7 +349,9 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         const int h = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const uint32_t xin_peer = map_peer(sbase + kOffXin, peer);
-        const uint32_t xbar_peer[2] = {map_peer(smem_u32(&xin_full[0]), peer), map_peer(smem_u32(&xin_full[1]), peer)};
+        uint32_t xbar_peer[kXBufs];
+#pragma unroll
+        for (int i = 0; i < kXBufs; ++i) xbar_peer[i] = map_peer(smem_u32(&xin_full[i]), peer);
         const bool leader = (warp == 2) && lane == 0;
         ItemIter iter;
         iter.init(a, pair);
@@ -396,11 +392,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             bool stop = false;
             for (int k = 0; k < T; ++k) {
                 const uint32_t g = it + k;
-                const int sb = g & 1;
+                const int sb = g & 1, xb = g % kXBufs;
                 if (leader) {
-                    // score tile g ready; the peer's buffer sb was read (tile g - 2)
+                    // score tile g ready; the peer's buffer xb is free (its O GEMM of tile g - 3 is done)
                     bool ok = mbar_wait(&s_full[sb], (g >> 1) & 1, abort);
-                    if (ok && g >= 2) ok = mbar_wait<true>(&rx_done[sb], ((g >> 1) - 1) & 1, abort);
+                    if (ok && g >= kXBufs) ok = mbar_wait<true>(&rx_done[xb], ((g / kXBufs) - 1) & 1, abort);
                     if (!ok) fail();
                     ex_stop = *abort;
                 }
@@ -409,7 +405,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 tc_fence_after();
                 // my raw partial scores rounded to fp16, stored straight into the peer's
                 // buffer (the peer adds exactly these values; so do I)
-                const uint32_t row = xin_peer + sb * kTileBytes + h * 128;
+                const uint32_t row = xin_peer + xb * kTileBytes + h * 128;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[32];
@@ -424,7 +420,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                             hw[i] = *reinterpret_cast<uint32_t*>(&v);
                         }
                         const int chunk = 4 * half + c;
-                        st_async_u4(row + ((chunk ^ (h & 7)) << 4), hw[0], hw[1], hw[2], hw[3], xbar_peer[sb]);
+                        st_async_u4(row + ((chunk ^ (h & 7)) << 4), hw[0], hw[1], hw[2], hw[3], xbar_peer[xb]);
                     }
                 }
                 tc_fence_before();
@@ -445,11 +441,13 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         const int h = q * 32 + lane;
         const int tid = threadIdx.x - 192;            // 0..255
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const uint32_t rx_peer[2] = {map_peer(smem_u32(&rx_done[0]), peer), map_peer(smem_u32(&rx_done[1]), peer)};
         const bool leader = (warp == 6) && lane == 0;
         // O GEMM of global tile n has completed.  Completions alternate between two
         // barriers, and the next completion on o_done[n & 1] (tile n + 2) needs a P
         // tile not yet written whenever this is called, so the phase parity is exact.
+        // Exchange buffer g % 3 holds the peer's partial scores of tile g, then
+        // this CTA's P tile g (each thread overwrites exactly the chunks it read);
+        // the commit of O GEMM g hands it back to the peer (for its tile g + 3).
         auto wait_o = [&](uint32_t n) -> bool { return mbar_wait(&o_done[n & 1], (n >> 1) & 1, abort); };
         ItemIter iter;
         iter.init(a, pair);
@@ -464,13 +462,14 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             bool stop = false;
             for (int k = 0; k < T; ++k) {
                 const uint32_t g = it + k;
-                const int sb = g & 1;
+                const int sb = g & 1, xb = g % kXBufs;
                 const int key0 = (item.t0 + k) * kKeys;
                 const int valid = min(kKeys, item.n_vis - key0);
                 if (leader) {
-                    mbar_expect_tx(&xin_full[sb], kTileBytes);
-                    if (!(mbar_wait<true>(&xin_full[sb], (g >> 1) & 1, abort) && mbar_wait(&s_full[sb], (g >> 1) & 1, abort)))
-                        fail();
+                    mbar_expect_tx(&xin_full[xb], kTileBytes);
+                    const bool ok = mbar_wait<true>(&xin_full[xb], (g / kXBufs) & 1, abort) &&
+                                    mbar_wait(&s_full[sb], (g >> 1) & 1, abort);
+                    if (!ok) fail();
                     sm_stop = *abort;
                 }
                 named_barrier(2, 256);
@@ -483,7 +482,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 tmem_wait_ld();
                 tc_fence_before();
                 uint4 oth[4];
-                const uint32_t prow = sbase + kOffXin + sb * kTileBytes + h * 128;
+                const uint32_t prow = sbase + kOffXin + xb * kTileBytes + h * 128;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) oth[c] = ld_shared_u4(prow + (((4 * ch + c) ^ (h & 7)) << 4));
                 // raw score = own fp32 partial + the peer's fp16 partial
@@ -511,19 +510,9 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 // softmax in base 2: scores scaled by scale * log2(e) (> 0, so the raw max serves)
                 const float mx_half = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
                 row_max[ch][h] = mx_half;
-                // everyone has read the exchange buffers and published its half maximum;
-                // P buffer g & 1 is free once O GEMM g-2 completed
-                if (leader) {
-                    if (g >= 2 && !wait_o(g - 2)) fail();
-                    sm_stop2 = *abort;
-                }
+                // every half maximum published; every read of score buffer sb done
                 named_barrier(2, 256);
-                if (sm_stop2) { stop = true; break; }
-                if (leader) {
-                    // every thread's reads of the exchange buffer returned before the barrier
-                    mbar_arrive(&s_free[sb]);
-                    mbar_arrive_peer_relaxed(rx_peer[sb]);
-                }
+                if (leader) mbar_arrive(&s_free[sb]);
                 tc_fence_after();
                 const float mx = fmaxf(mx_half, row_max[ch ^ 1][h]);
                 const float m_new = fmaxf(m, mx);
@@ -568,7 +557,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                         st_shared_u4(st + box * kLatBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
                     }
                 }
-                const uint32_t pr = sbase + kOffP + (g & 1) * kTileBytes + h * 128;
+                const uint32_t pr = prow;             // P over the chunks read above
                 float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -586,7 +575,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 fence_async_smem();
                 tc_fence_before();
                 named_barrier(2, 256);
-                if (leader) mbar_arrive(&p_ready[g & 1]);
+                if (leader) mbar_arrive(&p_ready[xb]);
             }
             if (stop) break;
             // epilogue: normalised latent half (or partial + log2-sum-exp)

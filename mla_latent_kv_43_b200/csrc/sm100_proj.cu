@@ -131,20 +131,25 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
             for (int mt = 0; mt < 4; ++mt)
                 tma_load_2d(sA + (mt * 2 + kb) * 16384, &mapA, &full, kb * 64, h * 512 + mt * 128);
         }
-    } else if (warp == 1 && elect_one()) {
-        if (mbar_wait(&full, 0, nullptr)) {
+    } else if (warp == 1) {
+        // whole warp, one elected lane issues (warp-uniform descriptors)
+        int ready = 0;
+        if (lane == 0) ready = mbar_wait(&full, 0, nullptr) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, ready, 0)) {
             tc_fence_after();
             const uint32_t idesc = idesc_bf16(128, N, false, false);
-            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+            const uint64_t da = sdesc(smem_u32(sA), 16, 1024, kSwizzle128);
+            const uint64_t db = sdesc(smem_u32(sB), 16, 1024, kSwizzle128);
+#pragma unroll
             for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(tmem + mt * N, sdesc(a0 + (mt * 2 + kb) * 16384 + ks * 32, 16, 1024, kSwizzle128),
-                               sdesc(b0 + kb * N * 128 + ks * 32, 16, 1024, kSwizzle128), idesc,
-                               (kb | ks) ? 1u : 0u);
+                        mma_ss_w(tmem + mt * N, sdesc_add(da, (mt * 2 + kb) * 16384 + ks * 32),
+                                 sdesc_add(db, kb * N * 128 + ks * 32), idesc, (kb | ks) ? 1u : 0u);
         }
-        mma_commit(&done);
+        mma_commit_w(&done);
     }
     __syncwarp();
 
@@ -250,19 +255,22 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
         grid_dep_wait();         // o_lat comes from the previous kernels
         for (int kb = 0; kb < 8; ++kb)
             tma_load_3d(smem + kb * stage + 16384, &mapB, &full[kb], kb * 64, h, nt * N);
-    } else if (warp == 1 && elect_one()) {
+    } else if (warp == 1) {
+        // whole warp, one elected lane issues (warp-uniform descriptors)
         const uint32_t idesc = idesc_bf16(128, N, true, false);
-        bool ok = true;
-        for (int kb = 0; kb < 8 && ok; ++kb) {
-            if (!mbar_wait(&full[kb], 0, nullptr)) { ok = false; break; }
+        const uint64_t da = sdesc(smem_u32(smem), 8192, 1024, kSwizzle128);
+        const uint64_t db = sdesc(smem_u32(smem) + 16384, 16, 1024, kSwizzle128);
+        for (int kb = 0; kb < 8; ++kb) {
+            int ready = 0;
+            if (lane == 0) ready = mbar_wait(&full[kb], 0, nullptr) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ready, 0)) break;
             tc_fence_after();
-            const uint32_t sa = smem_u32(smem + kb * stage), sb = sa + 16384;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_ss(tmem, sdesc(sa + ks * 2048, 8192, 1024, kSwizzle128), sdesc(sb + ks * 32, 16, 1024, kSwizzle128),
-                       idesc, (kb | ks) ? 1u : 0u);
+                mma_ss_w(tmem, sdesc_add(da, kb * stage + ks * 2048), sdesc_add(db, kb * stage + ks * 32), idesc,
+                         (kb | ks) ? 1u : 0u);
         }
-        mma_commit(&done);
+        mma_commit_w(&done);
     }
     __syncwarp();
     grid_dep_wait();

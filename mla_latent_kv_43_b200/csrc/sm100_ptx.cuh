@@ -226,6 +226,67 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// Warp-collective forms of the three issue instructions: every lane of a
+// converged warp executes the call and one lane, chosen by elect.sync inside
+// the same asm block, issues the instruction.  Keeping the issuing loop
+// warp-uniform (instead of running it in one divergent thread) lets the
+// descriptors stay warp-uniform values, which makes issue several times
+// cheaper.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+        : "memory");
+}
+
+// Commit whose arrive lands on the barrier at the same shared-memory offset
+// in every CTA of `cta_mask` (the CTAs of this cluster, by rank), e.g. to
+// release a buffer that another CTA of the cluster fills.  Warp-collective,
+// one elected lane issues.
+__device__ __forceinline__ void mma_commit_mc_w(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+// mbar_ready for a converged warp: lane 0's observation, broadcast, so every
+// lane takes the same branch.
+__device__ __forceinline__ bool mbar_ready_w(uint64_t* bar, uint32_t parity) {
+    return __shfl_sync(0xffffffffu, mbar_ready(bar, parity) ? 1 : 0, 0) != 0;
+}
+
+// A descriptor for the same matrix layout starting `bytes` further on: the
+// start address field holds address >> 4 in its low 14 bits, and every shared
+// address of a CTA fits there, so adding never carries into the next field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) { return desc + (bytes >> 4); }
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
