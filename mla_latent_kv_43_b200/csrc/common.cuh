@@ -37,16 +37,17 @@ __device__ __forceinline__ void rope_pair(float x0, float x1, int64_t pos, int i
     *y1 = (float)((double)x0 * s + (double)x1 * c);
 }
 
-// Same rotation with the pair frequency theta = base^(-2i/d_rope) given:
-// the angle pos * theta is formed and reduced modulo 2*pi in double, so the
-// single-precision sincosf only sees |x| <= pi.
-__device__ __forceinline__ void rope_pair_theta(float x0, float x1, int64_t pos, double theta, float* y0,
-                                                float* y1) {
-    const double two_pi = 6.283185307179586476925286766559;
-    const double ang = (double)pos * theta;
-    const double red = ang - rint(ang * (1.0 / two_pi)) * two_pi;
+// Same rotation with the pair frequency given as a fraction of a turn in
+// 64-bit fixed point, turn = round(theta / (2 pi) * 2^64) (rope_turn_table).
+// pos * turn modulo 2^64 is frac(pos * theta / (2 pi)) exactly up to the
+// table's rounding (< 2^-33 of a turn for pos < 2^31), so the angle reaches
+// sincosf already reduced to [-pi, pi); only integer multiplies, no double.
+__device__ __forceinline__ void rope_pair_turn(float x0, float x1, int64_t pos, uint64_t turn, float* y0,
+                                               float* y1) {
+    const uint64_t t = (uint64_t)pos * turn;
+    const float ang = (float)(int32_t)(uint32_t)(t >> 32) * 1.46291807926715968e-9f;   // 2 pi / 2^32
     float s, c;
-    sincosf((float)red, &s, &c);
+    sincosf(ang, &s, &c);
     *y0 = x0 * c - x1 * s;
     *y1 = x0 * s + x1 * c;
 }

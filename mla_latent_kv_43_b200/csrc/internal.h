@@ -53,4 +53,9 @@ int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// RoPE pair frequencies theta_i = base^(-2i/d_rope), i < d_rope / 2, as
+// fractions of a turn in 64-bit fixed point: turn[i] = round(theta_i / (2 pi) * 2^64),
+// computed in long double (rope_pair_turn in common.cuh uses them).
+void rope_turn_table(float base, int d_rope, uint64_t* turn);
+
 }  // namespace mla

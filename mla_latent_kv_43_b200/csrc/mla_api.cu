@@ -41,6 +41,18 @@ int layout_for(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len
 
 }  // namespace
 
+namespace mla {
+
+void rope_turn_table(float base, int d_rope, uint64_t* turn) {
+    const long double two_pi = 6.283185307179586476925286766559005768L;
+    for (int i = 0; i < d_rope / 2; ++i) {
+        const long double theta = powl((long double)base, -2.0L * i / d_rope);
+        turn[i] = (uint64_t)llroundl(theta / two_pi * 18446744073709551616.0L);   // 2^64
+    }
+}
+
+}  // namespace mla
+
 extern "C" {
 
 size_t mla_decode_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len,

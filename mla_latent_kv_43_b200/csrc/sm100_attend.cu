@@ -152,17 +152,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-    uint32_t r[16];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        tmem_ld16(taddr + 16 * c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 * c + i] = __uint_as_float(r[i]);
-    }
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
               AttnArgs a) {

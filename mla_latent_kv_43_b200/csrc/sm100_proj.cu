@@ -35,7 +35,7 @@ struct ProjArgs {
     const __nv_bfloat16* q_rope;
     const int32_t* seq_lens;
     int64_t capacity, max_len;
-    float rope_base;
+    uint64_t rope_turn[32];  // pair frequencies, fractions of a turn (rope_turn_table)
     __nv_bfloat16* q_lat;
     int32_t* cum;            // [BJ + 1] key tiles prefix of each query token
     // upproj
@@ -45,7 +45,7 @@ struct ProjArgs {
 
 __device__ void plan_tiles(const ProjArgs& a, int tid) {
     // Tiles of 64 keys each query token attends; 0 for an invalid length.
-    __shared__ int32_t part[kThreads + 1];
+    __shared__ int32_t part[kThreads / 32];
     const int per = (a.BJ + kThreads - 1) / kThreads;
     const int lo = min(a.BJ, tid * per), hi = min(a.BJ, lo + per);
     int32_t sum = 0;
@@ -59,13 +59,19 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
             bad = true;
     }
     if (bad) set_status(a.status, MLA_ERR_LEN);
-    part[tid + 1] = sum;
-    if (tid == 0) part[0] = 0;
+    // exclusive prefix of the per-thread sums: shuffle scan in each warp, then
+    // the four warp totals
+    const int lane = tid & 31, warp = tid >> 5;
+    int32_t incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    if (lane == 31) part[warp] = incl;
     __syncthreads();
-    if (tid == 0)
-        for (int i = 1; i <= kThreads; ++i) part[i] += part[i - 1];
-    __syncthreads();
-    int32_t run = part[tid];
+    int32_t run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += part[w];
     if (tid == 0) a.cum[0] = 0;
     for (int bj = lo; bj < hi; ++bj) {
         const int b = bj / a.n_q, j = bj % a.n_q;
@@ -91,22 +97,25 @@ __device__ bool block_wait(uint64_t* bar, int* flag, int32_t* status) {
     return *flag != 0;
 }
 
-// One CTA per (head, token tile): the whole W_uk[h] (4 row tiles x 2 k-blocks,
-// 128 KB) and the token tile's q_nope arrive in one batch of TMA loads; the 4
-// row tiles accumulate side by side in TMEM (4 x N columns).
-__global__ void __launch_bounds__(kThreads, 1)
+// One CTA per (head h, row tile mt of W_uk[h], token tile): the 128 latent
+// rows [128 mt, 128 mt + 128) against the tile's tokens, M = 128, N = tokens,
+// K = 128 (2 boxes of 64).  Four CTAs of 48 KB fit on an SM, so one CTA's
+// loads overlap another's MMAs and epilogue.  This is the first kernel of a
+// decode call and is launched without programmatic dependence: its TMA loads
+// read the caller's inputs.
+__global__ void __launch_bounds__(kThreads, 4)
 absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB, ProjArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full, done;
     __shared__ uint32_t tmem_base;
     __shared__ int flag;
-    const int h = blockIdx.x, nt = blockIdx.z;
+    const int h = blockIdx.x, mt = blockIdx.y, nt = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = a.n_tile;
-    const uint32_t ncols = tmem_cols_for(4 * N);
-    uint8_t* sA = smem;                    // [mt][kb] 16 KB boxes
-    uint8_t* sB = smem + 8 * 16384;        // [kb] N x 128 B
+    const uint32_t ncols = tmem_cols_for(N);
+    uint8_t* sA = smem;                    // [kb] 16 KB boxes: 128 rows x 64 k
+    uint8_t* sB = smem + 2 * 16384;        // [kb] N x 128 B
 
     if (threadIdx.x == 0) {
         mbar_init(&full, 1);
@@ -121,15 +130,13 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base;
+    grid_dep_wait();         // no-op under a plain launch
 
-    // W_uk and q_nope are inputs: load and multiply before waiting for the
-    // previous kernel; the workspace (q_lat, plan) is written only after it.
     if (warp == 0 && elect_one()) {
-        mbar_expect_tx(&full, 8 * 16384 + 2 * N * 128);
+        mbar_expect_tx(&full, 2 * 16384 + 2 * N * 128);
         for (int kb = 0; kb < 2; ++kb) {
+            tma_load_2d(sA + kb * 16384, &mapA, &full, kb * 64, h * 512 + mt * 128);
             tma_load_3d(sB + kb * N * 128, &mapB, &full, kb * 64, h, nt * N);
-            for (int mt = 0; mt < 4; ++mt)
-                tma_load_2d(sA + (mt * 2 + kb) * 16384, &mapA, &full, kb * 64, h * 512 + mt * 128);
         }
     } else if (warp == 1) {
         // whole warp, one elected lane issues (warp-uniform descriptors)
@@ -141,73 +148,63 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
             const uint64_t da = sdesc(smem_u32(sA), 16, 1024, kSwizzle128);
             const uint64_t db = sdesc(smem_u32(sB), 16, 1024, kSwizzle128);
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
+            for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-                for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss_w(tmem + mt * N, sdesc_add(da, (mt * 2 + kb) * 16384 + ks * 32),
-                                 sdesc_add(db, kb * N * 128 + ks * 32), idesc, (kb | ks) ? 1u : 0u);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ss_w(tmem, sdesc_add(da, kb * 16384 + ks * 32), sdesc_add(db, kb * N * 128 + ks * 32), idesc,
+                             (kb | ks) ? 1u : 0u);
         }
         mma_commit_w(&done);
     }
     __syncwarp();
-
-    grid_dep_wait();
     grid_dep_trigger();
-    // query RoPE (one thread per token row, vector loads/stores) and the
-    // key-tile plan while the MMAs run
-    __shared__ double theta[32];
-    if (threadIdx.x < 32) theta[threadIdx.x] = pow((double)a.rope_base, -2.0 * threadIdx.x / 64.0);
-    __syncthreads();
-    for (int t = threadIdx.x; t < N; t += kThreads) {
-        const int n = nt * N + t;
-        if (n >= a.BJ) break;
-        const int b = n / a.n_q, j = n % a.n_q;
+
+    // query RoPE (CTAs of row tile 0; one thread per token row, N <= kThreads)
+    // and the key-tile plan while the MMAs run
+    const int n_row = nt * N + threadIdx.x;
+    if (mt == 0 && threadIdx.x < N && n_row < a.BJ) {
+        const int b = n_row / a.n_q, j = n_row % a.n_q;
         const int64_t p = query_pos(a.seq_lens[b], a.n_q, j);
-        const uint4* src = reinterpret_cast<const uint4*>(a.q_rope + ((int64_t)n * a.H + h) * 64);
-        uint4* dst = reinterpret_cast<uint4*>(a.q_lat + ((int64_t)n * a.H + h) * 576 + 512);
-        uint4 v[8];
+        const uint4* src = reinterpret_cast<const uint4*>(a.q_rope + ((int64_t)n_row * a.H + h) * 64);
+        uint4* dst = reinterpret_cast<uint4*>(a.q_lat + ((int64_t)n_row * a.H + h) * 576 + 512);
+        uint4 rot[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = src[c];
+        for (int c = 0; c < 8; ++c) rot[c] = src[c];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+            uint32_t w[4] = {rot[c].x, rot[c].y, rot[c].z, rot[c].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
                 float y0, y1;
-                rope_pair_theta(x.x, x.y, p, theta[4 * c + i], &y0, &y1);
+                rope_pair_turn(x.x, x.y, p, a.rope_turn[4 * c + i], &y0, &y1);
                 w[i] = pack_bf16(y0, y1);
             }
             dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
-    if (h == 0 && nt == 0) plan_tiles(a, threadIdx.x);
+    if (h == 0 && mt == 0 && nt == 0) plan_tiles(a, threadIdx.x);
 
     if (block_wait(&done, &flag, a.status)) {
-        // TMEM row m of tile mt holds q_lat[n][h][128 mt + m] for the N tokens;
-        // stage as [n][512] bf16 in smem (the operand area is free now), then
-        // write each token's 1 KB row with 16-byte stores.
+        // TMEM row m holds q_lat[n][h][128 mt + m] for the N tokens; stage as
+        // [n][128] bf16 in smem (the operand area is free now), then write each
+        // token's 256-byte segment with 16-byte stores.
         tc_fence_after();
         __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(smem);
         const int m = warp * 32 + lane;
-        for (int mt = 0; mt < 4; ++mt) {
-            for (int c0 = 0; c0 < N; c0 += 16) {
-                uint32_t r[16];
-                tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + mt * N + c0, r);
-                tmem_wait_ld();
+        for (int c0 = 0; c0 < N; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+            tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    stage[(c0 + c) * 512 + mt * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[c]));
-            }
+            for (int c = 0; c < 16; ++c) stage[(c0 + c) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[c]));
         }
         __syncthreads();
         const int nvalid = min(N, a.BJ - nt * N);
-        for (int i = threadIdx.x; i < nvalid * 64; i += kThreads) {
-            const int n = i >> 6, c = i & 63;
-            reinterpret_cast<uint4*>(a.q_lat + ((int64_t)(nt * N + n) * a.H + h) * 576)[c] =
-                reinterpret_cast<const uint4*>(stage + n * 512)[c];
+        for (int i = threadIdx.x; i < nvalid * 16; i += kThreads) {
+            const int n = i >> 4, c = i & 15;
+            reinterpret_cast<uint4*>(a.q_lat + ((int64_t)(nt * N + n) * a.H + h) * 576 + 128 * mt)[c] =
+                reinterpret_cast<const uint4*>(stage + n * 128)[c];
         }
     }
     tc_fence_before();
@@ -309,11 +306,12 @@ int round_n(int bj, int cap) {
 
 template <typename K>
 int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs& a, dim3 grid, size_t smem,
-           cudaStream_t st, const char* name, int* launches) {
+           cudaStream_t st, const char* name, int* launches, bool pdl = true) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(st, name);
-    const cudaError_t e = launch_pdl(kernel, grid, dim3(kThreads), smem, st, A, B, a);
+    const cudaError_t e = pdl ? launch_pdl(kernel, grid, dim3(kThreads), smem, st, A, B, a)
+                              : launch_plain(kernel, grid, dim3(kThreads), smem, st, A, B, a);
     prof_end(st);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
@@ -344,12 +342,13 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* 
     a.seq_lens = c.seq_lens;
     a.capacity = c.capacity;
     a.max_len = c.max_len;
-    a.rope_base = c.d.rope_base;
+    rope_turn_table(c.d.rope_base, 64, a.rope_turn);
     a.q_lat = q_lat;
     a.cum = cum;
     a.status = c.status;
-    const dim3 grid(H, 1, (BJ + N - 1) / N);
-    return launch(absorb_kernel, A, B, a, grid, 8 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches);
+    const dim3 grid(H, 4, (BJ + N - 1) / N);
+    return launch(absorb_kernel, A, B, a, grid, 2 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches,
+                  false);
 }
 
 // up-projection.  o_lat [BJ][H][512] bf16, W_uv [H][512][128], out [BJ][H][128]
