@@ -32,7 +32,8 @@
 //
 // Roles (448 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 "exchange"
 // (score tile -> fp16 -> peer smem, query loads; thread <-> head <-> TMEM lane),
-// warps 6-13 "softmax" (P, O rescale, epilogue; two threads per head row).
+// warps 6-13 "softmax" (P, O rescale, epilogue): two groups of four warps that
+// take alternate tiles, one thread per head row.
 //
 // Work items.  The key tiles of all query tokens are concatenated and cut
 // into one contiguous range per cluster.  A token whose tiles all fall in one
@@ -56,6 +57,7 @@ namespace {
 
 constexpr int kKeys = 64;
 constexpr int kStages = 4;
+constexpr int kPrefetchTiles = 4;                  // L2 prefetch distance beyond the loads
 constexpr int kLatBox = 8192;                      // 64 keys x 64 columns x 2 B
 constexpr int kRopeBox = 4096;                     // 64 keys x 32 columns x 2 B
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;
@@ -164,8 +166,13 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     __shared__ int abort_flag;
     // per-warpgroup decisions, each written by the leader before a named barrier
     // and read after it; a barrier separates every read from the next write
-    __shared__ int ex_stop, sm_stop, sm_top;
-    __shared__ float row_max[2][128], row_sum[2][128];   // softmax half-row exchange
+    __shared__ int ex_stop;
+    // softmax: the running row maximum after tile g (slot g & 1) and its
+    // per-quarter barriers; per-item meeting of the two groups' row sums
+    __shared__ uint64_t m_ready[2][4], ep_ready[4];
+    __shared__ float m_pub[2][128];
+    __shared__ float ep_m[2][2][128], ep_l[2][2][128];
+    __shared__ __align__(16) uint32_t ep_scratch[8][32 * 16];   // per softmax warp: 32 rows x 64 bytes
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -179,16 +186,21 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 5);       // 4 exchange warps + the softmax leader
+            mbar_init(&s_free[i], 8);       // 4 exchange warps + the 4 warps of the tile's softmax group
         }
         for (int i = 0; i < kXBufs; ++i) {
             mbar_init(&xin_full[i], 1);     // my softmax leader's expect_tx + the peer's bytes
             mbar_init(&rx_done[i], 1);      // the peer's O GEMM has read the buffer (its commit)
-            mbar_init(&p_ready[i], 1);      // P tile written over the exchange buffer
+            mbar_init(&p_ready[i], 4);      // P tile written over the exchange buffer (4 warps)
         }
         mbar_init(&o_done[0], 1);           // O GEMMs of even / odd global tiles
         mbar_init(&o_done[1], 1);
         mbar_init(&q_ready, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&m_ready[0][i], 1);   // warp of lane quarter i in the group of an even tile
+            mbar_init(&m_ready[1][i], 1);   // ... of an odd tile
+            mbar_init(&ep_ready[i], 2);     // the two groups' warps of lane quarter i, once per item
+        }
         mbar_init(&drain, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -219,11 +231,40 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             ItemIter iter;
             iter.init(a, pair);
             Item item;
+            // L2 prefetch runs kPrefetchTiles tiles ahead of the shared-memory loads,
+            // so a stage that frees up is refilled from L2 rather than from HBM
+            ItemIter pf_iter;
+            pf_iter.init(a, pair);
+            Item pf_item;
+            bool pf_have = pf_iter.next(pf_item);
+            int pf_t = pf_have ? pf_item.t0 : 0;
+            auto prefetch_skip_next = [&]() {      // advance without prefetching
+                if (!pf_have) return;
+                if (++pf_t == pf_item.t1) {
+                    pf_have = pf_iter.next(pf_item);
+                    if (pf_have) pf_t = pf_item.t0;
+                }
+            };
+            auto prefetch_next = [&]() {
+                if (!pf_have) return;
+                const int pb = pf_item.bj / a.n_q;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tma_prefetch_l2_3d(&map_lat, 256 * rank + 64 * i, pf_t * kKeys, pb);
+                tma_prefetch_l2_3d(&map_rope, 512 + 32 * rank, pf_t * kKeys, pb);
+                if (++pf_t == pf_item.t1) {
+                    pf_have = pf_iter.next(pf_item);
+                    if (pf_have) pf_t = pf_item.t0;
+                }
+            };
+            // the prefetch starts once the ring has cycled: the first stages' loads
+            // are not made to share the start-up burst with it
+            for (int i = 0; i < kStages + kPrefetchTiles; ++i) prefetch_skip_next();
             uint32_t it = 0;
             bool ok = true;
             while (ok && iter.next(item)) {
                 const int b = item.bj / a.n_q;
                 for (int t = item.t0; t < item.t1; ++t, ++it) {
+                    if (it >= kStages) prefetch_next();
                     const int s = it % kStages;
                     if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, abort)) {
                         ok = false;
@@ -420,196 +461,230 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             it += T;
         }
     } else {
-        // ------------------------------------------------------------ softmax warpgroups
-        // Two threads per head row: warp w serves TMEM lane quarter w % 4 and
-        // score columns [32c, 32c + 32) with c = (w - 6) / 4.  The two halves
-        // share the row maximum through smem each tile and keep separate
-        // running sums, combined once per item.
+        // ------------------------------------------------------------ softmax groups
+        // Two groups of four warps take alternate global tiles (group 0 even g,
+        // warps 6-9; group 1 odd g, warps 10-13).  One thread per head row (its
+        // TMEM lane) handles all 64 score columns of its group's tiles.  The
+        // running row maximum is handed from each tile to the next through m_pub
+        // and a per-quarter mbarrier, so a group spends two tile periods on each
+        // of its tiles while the other group works on the next one.  Each group
+        // keeps its own part of the row sum, relative to the maximum it last
+        // used; the two parts meet at the end of every item.
+        const int grp = (warp - 6) >> 2;
         const int q = warp & 3;
-        const int ch = (warp - 6) >> 2;               // column half
         const int h = q * 32 + lane;
-        const int tid = threadIdx.x - 192;            // 0..255
+        const int gtid = (warp - 6 - 4 * grp) * 32 + lane;   // 0..127 within the group
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const bool leader = (warp == 6) && lane == 0;
+        const bool xleader = (warp == 6 + 4 * grp) && lane == 0;   // the expect_tx of this group's tiles
         // O GEMM of global tile n has completed.  Completions alternate between two
-        // barriers, and the next completion on o_done[n & 1] (tile n + 2) needs a P
-        // tile not yet written whenever this is called, so the phase parity is exact.
-        // Exchange buffer g % 3 holds the peer's partial scores of tile g, then
-        // this CTA's P tile g (each thread overwrites exactly the chunks it read);
-        // the commit of O GEMM g hands it back to the peer (for its tile g + 3).
+        // barriers; the next completion on o_done[n & 1] (tile n + 2) needs a P tile
+        // that cannot have been written when this is called, so the parity is exact.
+        // Exchange buffer g % 3 holds the peer's partial scores of tile g, then this
+        // CTA's P tile g (each thread overwrites exactly the chunks it read); the
+        // commit of O GEMM g hands it back to the peer (for its tile g + 3).
         auto wait_o = [&](uint32_t n) -> bool { return mbar_wait(&o_done[n & 1], (n >> 1) & 1, abort); };
+        // lane 0 waits (bounded), the warp follows its outcome
+        auto lane0 = [&](bool ok) -> bool { return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0; };
         ItemIter iter;
         iter.init(a, pair);
         Item item;
-        uint32_t it = 0;
-        while (iter.next(item)) {
-            if (leader) sm_top = *abort;
-            named_barrier(2, 256);
-            if (sm_top) break;
-            float m = -INFINITY, l = 0.f;             // l: this thread's half of the row sum
+        uint32_t it = 0, n_item = 0;
+        bool stop = false;
+        while (!stop && iter.next(item)) {
             const int T = item.t1 - item.t0;
-            bool stop = false;
-            for (int k = 0; k < T; ++k) {
+            float m_used = -INFINITY, l = 0.f;        // this group's part of the row sum, relative to m_used
+            for (int k = 0; k < T && !stop; ++k) {
                 const uint32_t g = it + k;
+                if ((int)(g & 1) != grp) continue;
                 const int sb = g & 1, xb = g % kXBufs;
                 const int key0 = (item.t0 + k) * kKeys;
                 const int valid = min(kKeys, item.n_vis - key0);
-                if (leader) {
-                    mbar_expect_tx(&xin_full[xb], kTileBytes);
-                    const bool ok = mbar_wait<true>(&xin_full[xb], (g / kXBufs) & 1, abort) &&
-                                    mbar_wait(&s_full[sb], (g >> 1) & 1, abort);
-                    if (!ok) fail();
-                    sm_stop = *abort;
+                bool ok = true;
+                if (lane == 0) {
+                    if (xleader) mbar_expect_tx(&xin_full[xb], kTileBytes);
+                    ok = mbar_wait<true>(&xin_full[xb], (g / kXBufs) & 1, abort) &&
+                         mbar_wait(&s_full[sb], (g >> 1) & 1, abort);
                 }
-                named_barrier(2, 256);
-                if (sm_stop) { stop = true; break; }
-                // own partial (TMEM, rounded to fp16 exactly as sent to the peer) and the
-                // peer's fp16 partial for this row half (chunks 4c .. 4c + 3)
+                if (!lane0(ok)) { stop = true; break; }
+                // own fp32 partial (TMEM) plus the peer's fp16 partial (smem)
                 tc_fence_after();
-                uint32_t own[32];
-                tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32 * ch, own);
-                tmem_wait_ld();
+                float x[64];
+                {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[32 + i] = __uint_as_float(r[i]);
+                }
                 tc_fence_before();
-                uint4 oth[4];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sb]);      // this warp is done with score buffer sb
                 const uint32_t prow = sbase + kOffXin + xb * kTileBytes + h * 128;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) oth[c] = ld_shared_u4(prow + (((4 * ch + c) ^ (h & 7)) << 4));
-                // raw score = own fp32 partial + the peer's fp16 partial
-                float x[32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t pw[4] = {oth[c].x, oth[c].y, oth[c].z, oth[c].w};
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = ld_shared_u4(prow + ((c ^ (h & 7)) << 4));
+                    const uint32_t pw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int n = 8 * c + 2 * i;
                         const float2 b2 = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
-                        x[n] = __uint_as_float(own[n]) + b2.x;
-                        x[n + 1] = __uint_as_float(own[n + 1]) + b2.y;
+                        x[8 * c + 2 * i] += b2.x;
+                        x[8 * c + 2 * i + 1] += b2.y;
                     }
                 }
                 if (valid < kKeys) {
 #pragma unroll
-                    for (int n = 0; n < 32; ++n) x[n] = (32 * ch + n) < valid ? x[n] : -INFINITY;
+                    for (int n = 0; n < 64; ++n) x[n] = n < valid ? x[n] : -INFINITY;
                 }
                 float mx8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24]));
+                for (int i = 0; i < 8; ++i)
+                    mx8[i] = fmaxf(fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24])),
+                                   fmaxf(fmaxf(x[i + 32], x[i + 40]), fmaxf(x[i + 48], x[i + 56])));
 #pragma unroll
                 for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
                 // softmax in base 2: scores scaled by scale * log2(e) (> 0, so the raw max serves)
-                const float mx_half = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
-                row_max[ch][h] = mx_half;
-                // every half maximum published; every read of score buffer sb done
-                named_barrier(2, 256);
-                if (leader) mbar_arrive(&s_free[sb]);
-                tc_fence_after();
-                const float mx = fmaxf(mx_half, row_max[ch ^ 1][h]);
-                const float m_new = fmaxf(m, mx);
-                // Lazy rescaling: only when the row maximum grew by more than 2^8.
-                // The TMEM accesses are warp-collective, so the decision is made per
-                // warp; lanes that need no rescale multiply by 1.
-                const bool need = m_new > m + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need) && k > 0) {
-                        // O must hold every earlier tile: O GEMM g-1 has to be complete.
-                    int ok = 1;
-                    if (lane == 0) {
-                        ok = wait_o(g - 1) ? 1 : 0;
-                        if (!ok) fail();
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (ok) {
-                        tc_fence_after();
-                        const float alpha = need ? ex2(m - m_new) : 1.f;
-#pragma unroll 1
-                        for (int c = 0; c < 8; ++c) {
-                            uint32_t r[16];
-                            const uint32_t ta = tmem + lane_off + kColO + 128 * ch + 16 * c;
-                            tmem_ld16(ta, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                            tmem_st16(ta, r);
-                        }
-                        tmem_wait_st();
-                    }
+                const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
+                // the running maximum after tile g - 1 (ignored at an item's first tile)
+                float m_prev = -INFINITY;
+                if (g >= 1) {
+                    const int pb = (g - 1) & 1;
+                    if (lane == 0) ok = mbar_wait(&m_ready[pb][q], ((g - 1) >> 1) & 1, abort);
+                    if (!lane0(ok)) { stop = true; break; }
+                    if (k > 0) m_prev = m_pub[pb][h];
                 }
-                if (need) {
-                    l *= ex2(m - m_new);
-                    m = m_new;
+                // Lazy rescaling: the maximum moves only when it grew by more than 2^8.
+                const float m_cand = fmaxf(m_prev, mx);
+                const float m = m_cand > m_prev + kRescaleThreshold ? m_cand : m_prev;
+                m_pub[g & 1][h] = m;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&m_ready[g & 1][q]);
+                // O holds the tiles before g relative to m_prev: rescale it when m moved.
+                // TMEM accesses are warp-collective, so lanes that need none multiply by 1.
+                const bool need = k > 0 && m > m_prev;
+                if (__any_sync(0xffffffffu, need)) {
+                    if (lane == 0) ok = wait_o(g - 1);
+                    if (!lane0(ok)) { stop = true; break; }
+                    tc_fence_after();
+                    const float alpha = need ? ex2(m_prev - m) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < 16; ++c) {
+                        uint32_t r[16];
+                        const uint32_t ta = tmem + lane_off + kColO + 16 * c;
+                        tmem_ld16(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st16(ta, r);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+                if (m > m_used) {
+                    if (m_used != -INFINITY) l *= ex2(m_used - m);
+                    m_used = m;
                 }
                 if (valid < kKeys) {
                     // rows past the visible keys may hold anything: zero them for the O GEMM
                     const uint32_t st = sbase + (g % kStages) * kStageBytes;
                     const int nchunks = (kKeys - valid) * 32;
-                    for (int i = tid; i < nchunks; i += 256) {
+                    for (int i = gtid; i < nchunks; i += 128) {
                         const int r = valid + (i >> 5), box = (i >> 3) & 3, c = i & 7;
                         st_shared_u4(st + box * kLatBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
                     }
                 }
-                const uint32_t pr = prow;             // P over the chunks read above
-                float ps[4] = {0.f, 0.f, 0.f, 0.f};
+                float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t pw[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const float p0 = ex2(fmaf(x[8 * c + 2 * i], a.scale_log2, -m));
                         const float p1 = ex2(fmaf(x[8 * c + 2 * i + 1], a.scale_log2, -m));
-                        ps[i] += p0 + p1;
+                        ps4[i] += p0 + p1;
                         pw[i] = pack_bf16(p0, p1);
                     }
-                    st_shared_u4(pr + (((4 * ch + c) ^ (h & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                    // P over the chunk read above
+                    st_shared_u4(prow + ((c ^ (h & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                 }
-                l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+                l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
                 fence_async_smem();
-                tc_fence_before();
-                named_barrier(2, 256);
-                if (leader) mbar_arrive(&p_ready[xb]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_ready[xb]);
             }
             if (stop) break;
-            // epilogue: normalised latent half (or partial + log2-sum-exp)
-            row_sum[ch][h] = l;
-            if (leader) {
-                if (!wait_o(it + T - 1)) fail();
-                sm_stop = *abort;
+            // epilogue: both groups' sums meet; group c writes O columns [128c, 128c + 128)
+            // of this CTA's latent half (normalised, or a partial plus log2-sum-exp)
+            bool ok = true;
+            if (lane == 0) ok = wait_o(it + T - 1);
+            if (!lane0(ok)) break;
+            const int eb = n_item & 1;
+            ep_m[eb][grp][h] = m_used;
+            ep_l[eb][grp][h] = l;
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&ep_ready[q]);
+                ok = mbar_wait(&ep_ready[q], eb, abort);
             }
-            named_barrier(2, 256);
-            if (sm_stop) break;
+            if (!lane0(ok)) break;
+            const float m0 = ep_m[eb][0][h], m1 = ep_m[eb][1][h];
+            const float mf = fmaxf(m0, m1);
+            const float lsum = (m0 == -INFINITY ? 0.f : ep_l[eb][0][h] * ex2(m0 - mf)) +
+                               (m1 == -INFINITY ? 0.f : ep_l[eb][1][h] * ex2(m1 - mf));
             tc_fence_after();
-            const float lsum = row_sum[0][h] + row_sum[1][h];
             const float inv = 1.f / lsum;
-            if (item.slot < 0) {
-                uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ((int64_t)item.bj * 128 + h) * 512 + 256 * rank + 128 * ch);
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColO + 128 * ch + 16 * c, r);
-                    tmem_wait_ld();
-                    uint32_t pk[8];
+            // Rows leave TMEM one per thread; each 32-row x 64-byte block goes through
+            // this warp's smem scratch so that a store instruction covers eight
+            // contiguous 64-byte row segments instead of 32 scattered 16-byte pieces.
+            const uint32_t scr = smem_u32(&ep_scratch[warp - 6][0]);
+            auto put_rows = [&](const uint32_t (&w)[16], auto&& row_ptr) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                    dst[2 * c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                for (int j = 0; j < 4; ++j)
+                    st_shared_u4(scr + lane * 64 + ((j ^ (lane & 3)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int r = 8 * k + (lane >> 2), pc = lane & 3;
+                    const uint4 v = ld_shared_u4(scr + r * 64 + ((pc ^ (r & 3)) << 4));
+                    *reinterpret_cast<uint4*>(row_ptr(q * 32 + r) + 16 * pc) = v;
+                }
+                __syncwarp();
+            };
+            if (item.slot < 0) {
+                // bf16, 32 columns (64 bytes) per row and block
+                char* base = reinterpret_cast<char*>(a.o_lat + (int64_t)item.bj * 128 * 512 + 256 * rank + 128 * grp);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + kColO + 128 * grp + 32 * c, r);
+                    tmem_wait_ld();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                    put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 32 * c) * 2; });
                 }
             } else {
-                float4* dst = reinterpret_cast<float4*>(a.part_o + ((int64_t)item.slot * 128 + h) * 512 + 256 * rank +
-                                                        128 * ch);
+                // fp32 partial, 16 columns (64 bytes) per row and block
+                char* base = reinterpret_cast<char*>(a.part_o + (int64_t)item.slot * 128 * 512 + 256 * rank + 128 * grp);
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
                     uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColO + 128 * ch + 16 * c, r);
+                    tmem_ld16(tmem + lane_off + kColO + 128 * grp + 16 * c, r);
                     tmem_wait_ld();
+                    uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[4 * c + i] = make_float4(__uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                                                     __uint_as_float(r[4 * i + 2]) * inv,
-                                                     __uint_as_float(r[4 * i + 3]) * inv);
+                    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(__uint_as_float(r[i]) * inv);
+                    put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 16 * c) * 4; });
                 }
-                if (rank == 0 && ch == 0) a.part_lse[item.slot * 128 + h] = m + __log2f(lsum);
+                if (rank == 0 && grp == 0) a.part_lse[item.slot * 128 + h] = mf + __log2f(lsum);
             }
             tc_fence_before();
             it += T;
+            ++n_item;
         }
     }
 
