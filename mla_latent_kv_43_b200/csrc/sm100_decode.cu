@@ -56,42 +56,51 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
     if (pf == pl) return;            // finished inside one cluster
     // clusters with an empty tile range between the first and the last piece hold nothing
     auto empty = [&](int p) { return start(p) == (p + 1 < pairs ? start(p + 1) : T); };
-    constexpr int kMaxPieces = 16;
-    int slots[kMaxPieces];
-    int np = 0;
+    // pieces in batches of kBatch: every load of a batch (log-sum-exps and partial
+    // rows) is issued before any is used, so a batch costs one memory round trip
+    constexpr int kBatch = 4;
     float acc[16];
     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
     float wsum = 0.f;
     float M = -INFINITY;
-    // pieces in batches of up to kMaxPieces: log-sum-exps first (independent loads), then rows
-    for (int p0 = pf; p0 <= pl;) {
-        np = 0;
-        for (; p0 <= pl && np < kMaxPieces; ++p0)
+    int p0 = pf;
+    while (p0 <= pl) {
+        int slots[kBatch];
+        int np = 0;
+        for (; p0 <= pl && np < kBatch; ++p0)
             if (p0 == pf || !empty(p0)) slots[np++] = p0 == pf ? 2 * p0 + 1 : 2 * p0;
-        float lse[kMaxPieces];
-        float Mb = M;
-        for (int i = 0; i < np; ++i) {
-            lse[i] = part_lse[slots[i] * kHeads + h];
-            Mb = fmaxf(Mb, lse[i]);
+        float lse[kBatch];
+        float4 v[kBatch][4];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            if (i < np) {
+                lse[i] = part_lse[slots[i] * kHeads + h];
+                const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slots[i] * kHeads + h) * kDc + col);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) v[i][k] = src[k];
+            }
         }
+        float Mb = M;
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i)
+            if (i < np) Mb = fmaxf(Mb, lse[i]);
         // rescale what was accumulated so far to the new maximum
         const float r = (M == -INFINITY) ? 0.f : exp2f(M - Mb);
         wsum *= r;
         for (int i = 0; i < 16; ++i) acc[i] *= r;
         M = Mb;
-        for (int i = 0; i < np; ++i) {
-            const float w = exp2f(lse[i] - M);
-            wsum += w;
-            const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slots[i] * kHeads + h) * kDc + col);
-            float4 v[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) v[k] = src[k];
+        for (int i = 0; i < kBatch; ++i) {
+            if (i < np) {
+                const float w = exp2f(lse[i] - M);
+                wsum += w;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                acc[4 * k] = fmaf(w, v[k].x, acc[4 * k]);
-                acc[4 * k + 1] = fmaf(w, v[k].y, acc[4 * k + 1]);
-                acc[4 * k + 2] = fmaf(w, v[k].z, acc[4 * k + 2]);
-                acc[4 * k + 3] = fmaf(w, v[k].w, acc[4 * k + 3]);
+                for (int k = 0; k < 4; ++k) {
+                    acc[4 * k] = fmaf(w, v[i][k].x, acc[4 * k]);
+                    acc[4 * k + 1] = fmaf(w, v[i][k].y, acc[4 * k + 1]);
+                    acc[4 * k + 2] = fmaf(w, v[i][k].z, acc[4 * k + 2]);
+                    acc[4 * k + 3] = fmaf(w, v[i][k].w, acc[4 * k + 3]);
+                }
             }
         }
     }
