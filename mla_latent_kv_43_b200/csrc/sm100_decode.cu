@@ -129,8 +129,6 @@ bool sm100_decode_supported(const mla_dims& d) {
            d.v_dim == 128;
 }
 
-bool sm100_append_supported(const mla_dims&, int) { return false; }
-
 void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int splits, mla_ws_layout* L) {
     (void)max_len;
     const int64_t BJ = (int64_t)batch * n_q;
@@ -173,6 +171,5 @@ int sm100_decode(const DecodeCall& c, int* launches) {
     return sm100::launch_upproj(c, o_lat, launches);
 }
 
-int sm100_append(const AppendCall&, int*) { return MLA_ERR_UNSUPPORTED; }
 
 }  // namespace mla

@@ -75,3 +75,29 @@ def test_append_rejects_positions_outside_the_cache(case):
     tol = TOL["fp32"] if case.startswith("fp32") else TOL["bf16"]
     assert rel_err(cache[0, 3].double().cpu().numpy(), rows[0]) <= tol
     assert rel_err(cache[1, 15].double().cpu().numpy(), rows[3]) <= tol
+
+
+@pytest.mark.parametrize("hidden", [256, 7168])
+@pytest.mark.parametrize("tokens", [1, 37, 300])
+def test_tensor_core_append_shapes(hidden, tokens):
+    """DeepSeek-V3 latent/rope widths (the tensor-core append): fewer K blocks
+    than the cluster's CTAs (hidden 256), a single token, a ragged token count
+    and more tokens than one launch tile (300 > 256); every slot written once,
+    the rest untouched."""
+    CASES["bf16_v3_h"] = ("bf16", V3, hidden)
+    try:
+        batch, n_new, cap = tokens, 1, 9
+        rng = np.random.default_rng(tokens + hidden)
+        positions = [int(p) for p in rng.integers(0, cap, size=tokens)]
+        dims, x, W, pos, before, cache, code = run_append("bf16_v3_h", positions, batch, n_new, cap, seed=3)
+    finally:
+        del CASES["bf16_v3_h"]
+    assert code == 0
+    changed = (cache.view(torch.int16) != before.view(torch.int16)).any(-1).cpu()
+    expect = torch.zeros(batch, cap, dtype=torch.bool)
+    for r, p in enumerate(positions):
+        expect[r, p] = True
+    assert torch.equal(changed, expect)
+    rows = O.append_rows(x, W, positions, dims.d_c, dims.rope_base)
+    got = np.stack([cache[r, p].double().cpu().numpy() for r, p in enumerate(positions)])
+    assert rel_err(got, rows) <= TOL["bf16"]
