@@ -395,23 +395,32 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             // Every score GEMM of the previous item has completed: its last
             // score tile was read below before we got here.
             {
+                // loads in two batches of 16 (plus the rope chunks), each batch issued
+                // before any TMEM store, so the slice costs two memory round trips
                 const uint4* src = reinterpret_cast<const uint4*>(a.q_lat + ((int64_t)item.bj * 128 + h) * 576);
-                uint32_t w[16];
+                uint4 rq[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 4; ++c) rq[c] = src[64 + 4 * rank + c];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint4 v = src[32 * rank + 4 * c + i];
-                        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                for (int half = 0; half < 2; ++half) {
+                    uint4 v[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = src[32 * rank + 16 * half + i];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            w[4 * i] = v[4 * c + i].x; w[4 * i + 1] = v[4 * c + i].y;
+                            w[4 * i + 2] = v[4 * c + i].z; w[4 * i + 3] = v[4 * c + i].w;
+                        }
+                        tmem_st16(tmem + lane_off + kColQ + 16 * (4 * half + c), w);
                     }
-                    tmem_st16(tmem + lane_off + kColQ + 16 * c, w);
                 }
                 const uint32_t qrow = sbase + kOffQr + h * 64;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint4 v = src[64 + 4 * rank + c];
-                    st_shared_u4(qrow + ((c ^ ((h >> 1) & 3)) << 4), v.x, v.y, v.z, v.w);
-                }
+                for (int c = 0; c < 4; ++c)
+                    st_shared_u4(qrow + ((c ^ ((h >> 1) & 3)) << 4), rq[c].x, rq[c].y, rq[c].z, rq[c].w);
                 tmem_wait_st();
                 fence_async_smem();
                 tc_fence_before();

@@ -116,9 +116,18 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
     d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
-int pairs_for(int splits) {
-    const int max_pairs = std::max(1, sm_count() / 2);
-    return splits > 0 ? std::min(splits, max_pairs) : max_pairs;
+constexpr int kMaxPairs = 256;              // clusters per launch
+
+// Clusters per launch.  splits > 0 asks for that many; 0 (auto) gives every
+// cluster at least kMinTiles key tiles of the largest possible total
+// (batch * n_q * ceil(max_len / 64)): fewer, longer pieces when there are few
+// long sequences, all 74 clusters otherwise.
+constexpr int64_t kMinTiles = 8;
+int pairs_for(int splits, int64_t BJ, int64_t max_len) {
+    const int max_pairs = std::max(1, std::min(sm_count() / 2, kMaxPairs));
+    if (splits > 0) return std::min(splits, max_pairs);
+    const int64_t tiles = BJ * ((max_len + 63) / 64);
+    return (int)std::max<int64_t>(1, std::min<int64_t>(max_pairs, (tiles + kMinTiles - 1) / kMinTiles));
 }
 
 }  // namespace
@@ -130,9 +139,8 @@ bool sm100_decode_supported(const mla_dims& d) {
 }
 
 void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int splits, mla_ws_layout* L) {
-    (void)max_len;
     const int64_t BJ = (int64_t)batch * n_q;
-    const int P = sm100::pairs_for(splits);
+    const int P = sm100::pairs_for(splits, BJ, max_len);
     *L = mla_ws_layout{};
     size_t off = 0;
     auto take = [&](size_t bytes, size_t* o, size_t* sz) {
