@@ -81,13 +81,14 @@ typedef struct {
     size_t q_lat_bytes;
     size_t o_lat;          /* combined latent outputs [B][n_q][H][d_c], compute dtype */
     size_t o_lat_bytes;
-    size_t part_o;         /* split-KV partial latent outputs, float */
+    size_t part_o;         /* split-KV partial latent outputs, each normalised by its own sum:
+                              compute dtype on the tensor-core path, float otherwise */
     size_t part_o_bytes;
     size_t part_lse;       /* split-KV partial log-sum-exp values, float */
     size_t part_lse_bytes;
     size_t sched;          /* device-built work schedule */
     size_t sched_bytes;
-    int32_t compute_dtype; /* enum mla_dtype of q_lat and o_lat */
+    int32_t compute_dtype; /* enum mla_dtype of q_lat, o_lat (and part_o on the tensor-core path) */
     int32_t splits;        /* key splits per query (generic path) or work items (tensor-core path) */
 } mla_ws_layout;
 

@@ -73,11 +73,12 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units
 struct AttnArgs {
     const __nv_bfloat16* q_lat;   // [BJ][128][576]
     const int32_t* cum;           // [BJ + 1] tile prefix
+    const int32_t* first_bj;      // [pairs] first query token of each cluster's range
     const int32_t* seq_lens;
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* o_lat;         // [BJ][128][512]
-    float* part_o;                // [2 * pairs][128][512]
+    __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
     float* part_lse;              // [2 * pairs][128], log2 domain
     int32_t* status;
 };
@@ -100,12 +101,7 @@ struct ItemIter {
         const int T = cum[BJ];
         s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
         s1 = (int)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
-        int lo = 0, hi = BJ;          // first bj with cum[bj + 1] > s0
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (cum[mid + 1] > s0) hi = mid; else lo = mid + 1;
-        }
-        bj = lo;
+        bj = a.first_bj[p];           // first bj with cum[bj + 1] > s0 (from the plan)
     }
     __device__ bool next(Item& it) {
         while (bj < BJ) {
@@ -267,6 +263,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     if (it >= kStages) prefetch_next();
                     const int s = it % kStages;
                     if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    // start-up: the first stage is requested alone, so every SM's first
+                    // tile lands before the rest of the start-up burst
+                    if (it == 1 && !mbar_wait(&full[0], 0, abort)) {
                         ok = false;
                         break;
                     }
@@ -662,9 +664,13 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 }
                 __syncwarp();
             };
-            if (item.slot < 0) {
-                // bf16, 32 columns (64 bytes) per row and block
-                char* base = reinterpret_cast<char*>(a.o_lat + (int64_t)item.bj * 128 * 512 + 256 * rank + 128 * grp);
+            {
+                // bf16, 32 columns (64 bytes) per row and block: the normalised output of a
+                // token finished here, or this piece's normalised partial (plus its
+                // log2-sum-exp) for the combine step
+                __nv_bfloat16* dst = item.slot < 0 ? a.o_lat + (int64_t)item.bj * 128 * 512
+                                                   : a.part_o + (int64_t)item.slot * 128 * 512;
+                char* base = reinterpret_cast<char*>(dst + 256 * rank + 128 * grp);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
@@ -676,20 +682,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                         w[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
                     put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 32 * c) * 2; });
                 }
-            } else {
-                // fp32 partial, 16 columns (64 bytes) per row and block
-                char* base = reinterpret_cast<char*>(a.part_o + (int64_t)item.slot * 128 * 512 + 256 * rank + 128 * grp);
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(tmem + lane_off + kColO + 128 * grp + 16 * c, r);
-                    tmem_wait_ld();
-                    uint32_t w[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) w[i] = __float_as_uint(__uint_as_float(r[i]) * inv);
-                    put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 16 * c) * 4; });
-                }
-                if (rank == 0 && grp == 0) a.part_lse[item.slot * 128 + h] = mf + __log2f(lsum);
+                if (item.slot >= 0 && rank == 0 && grp == 0) a.part_lse[item.slot * 128 + h] = mf + __log2f(lsum);
             }
             tc_fence_before();
             it += T;
@@ -709,7 +702,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 }  // namespace
 
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                  float* part_o, float* part_lse, int pairs, int* launches) {
+                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches) {
     CUtensorMap ml, mr;
     const uint64_t dims[3] = {576, (uint64_t)c.capacity, (uint64_t)c.batch};
     const uint64_t str[2] = {576 * 2, (uint64_t)c.capacity * 576 * 2};
@@ -719,6 +712,7 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
     AttnArgs a{};
     a.q_lat = q_lat;
     a.cum = cum;
+    a.first_bj = first_bj;
     a.seq_lens = c.seq_lens;
     a.BJ = c.batch * c.n_q;
     a.n_q = c.n_q;

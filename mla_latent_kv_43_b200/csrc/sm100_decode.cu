@@ -14,10 +14,11 @@
 
 namespace mla {
 namespace sm100 {
-int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* launches);
+int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32_t* first_bj, int pairs,
+                  int* launches);
 int launch_upproj(const DecodeCall& c, const __nv_bfloat16* o_lat, int* launches);
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                  float* part_o, float* part_lse, int pairs, int* launches);
+                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches);
 
 namespace {
 
@@ -28,7 +29,7 @@ constexpr int kHeads = 128, kDc = 512;
 // an invalid length.  Tokens finished inside one cluster are left untouched.
 // grid (BJ, 128 / 4): 4 heads per block, 128 threads, 16 columns each.
 __global__ void __launch_bounds__(128)
-combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* __restrict__ part_o,
+combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const __nv_bfloat16* __restrict__ part_o,
                const float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o_lat) {
     grid_dep_wait();
     grid_dep_trigger();
@@ -65,19 +66,26 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
     float M = -INFINITY;
     int p0 = pf;
     while (p0 <= pl) {
-        int slots[kBatch];
+        int slots[kBatch] = {0, 0, 0, 0};
         int np = 0;
-        for (; p0 <= pl && np < kBatch; ++p0)
-            if (p0 == pf || !empty(p0)) slots[np++] = p0 == pf ? 2 * p0 + 1 : 2 * p0;
+        for (; p0 <= pl && np < kBatch; ++p0) {
+            if (p0 == pf || !empty(p0)) {
+                const int sl = p0 == pf ? 2 * p0 + 1 : 2 * p0;
+#pragma unroll
+                for (int i = 0; i < kBatch; ++i)
+                    if (i == np) slots[i] = sl;        // register-indexed, no local memory
+                ++np;
+            }
+        }
         float lse[kBatch];
-        float4 v[kBatch][4];
+        uint4 v[kBatch][2];               // 16 bf16 columns per piece
 #pragma unroll
         for (int i = 0; i < kBatch; ++i) {
             if (i < np) {
                 lse[i] = part_lse[slots[i] * kHeads + h];
-                const float4* src = reinterpret_cast<const float4*>(part_o + ((int64_t)slots[i] * kHeads + h) * kDc + col);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) v[i][k] = src[k];
+                const uint4* src = reinterpret_cast<const uint4*>(part_o + ((int64_t)slots[i] * kHeads + h) * kDc + col);
+                v[i][0] = src[0];
+                v[i][1] = src[1];
             }
         }
         float Mb = M;
@@ -95,11 +103,14 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const float* 
                 const float w = exp2f(lse[i] - M);
                 wsum += w;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    acc[4 * k] = fmaf(w, v[i][k].x, acc[4 * k]);
-                    acc[4 * k + 1] = fmaf(w, v[i][k].y, acc[4 * k + 1]);
-                    acc[4 * k + 2] = fmaf(w, v[i][k].z, acc[4 * k + 2]);
-                    acc[4 * k + 3] = fmaf(w, v[i][k].w, acc[4 * k + 3]);
+                for (int k = 0; k < 2; ++k) {
+                    const uint32_t pw[4] = {v[i][k].x, v[i][k].y, v[i][k].z, v[i][k].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
+                        acc[8 * k + 2 * j] = fmaf(w, f.x, acc[8 * k + 2 * j]);
+                        acc[8 * k + 2 * j + 1] = fmaf(w, f.y, acc[8 * k + 2 * j + 1]);
+                    }
                 }
             }
         }
@@ -150,9 +161,9 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
     };
     take(BJ * d.heads * (d.d_c + d.d_rope) * 2, &L->q_lat, &L->q_lat_bytes);
     take(BJ * d.heads * d.d_c * 2, &L->o_lat, &L->o_lat_bytes);
-    take((size_t)2 * P * d.heads * d.d_c * 4, &L->part_o, &L->part_o_bytes);
+    take((size_t)2 * P * d.heads * d.d_c * 2, &L->part_o, &L->part_o_bytes);   // bf16
     take((size_t)2 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);
-    take((BJ + 1) * 4, &L->sched, &L->sched_bytes);
+    take((BJ + 1 + P) * 4, &L->sched, &L->sched_bytes);   // tile prefix, then each cluster's first token
     L->total = off;
     L->compute_dtype = MLA_BF16;
     L->splits = P;
@@ -161,17 +172,18 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
 int sm100_decode(const DecodeCall& c, int* launches) {
     auto* q_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.q_lat);
     auto* o_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.o_lat);
-    auto* part_o = reinterpret_cast<float*>(c.ws + c.L.part_o);
+    auto* part_o = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.part_o);
     auto* part_lse = reinterpret_cast<float*>(c.ws + c.L.part_lse);
     auto* cum = reinterpret_cast<int32_t*>(c.ws + c.L.sched);
     const int P = c.L.splits;
     const int BJ = c.batch * c.n_q;
     int rc;
-    if ((rc = sm100::launch_absorb(c, q_lat, cum, launches))) return rc;
-    if ((rc = sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, P, launches))) return rc;
+    int32_t* first_bj = cum + BJ + 1;
+    if ((rc = sm100::launch_absorb(c, q_lat, cum, first_bj, P, launches))) return rc;
+    if ((rc = sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, P, launches))) return rc;
     prof_begin(c.stream, "sm100_combine");
     const cudaError_t e = sm100::launch_pdl(sm100::combine_kernel, dim3(BJ, 128 / 4), dim3(128), 0, c.stream,
-                                            (const int32_t*)cum, BJ, P, (const float*)part_o,
+                                            (const int32_t*)cum, BJ, P, (const __nv_bfloat16*)part_o,
                                             (const float*)part_lse, o_lat);
     prof_end(c.stream);
     if (launches) ++*launches;

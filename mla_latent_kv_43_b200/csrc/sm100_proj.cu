@@ -38,6 +38,8 @@ struct ProjArgs {
     uint64_t rope_turn[32];  // pair frequencies, fractions of a turn (rope_turn_table)
     __nv_bfloat16* q_lat;
     int32_t* cum;            // [BJ + 1] key tiles prefix of each query token
+    int32_t* first_bj;       // [pairs] first query token of each attention cluster's tile range
+    int pairs;
     // upproj
     __nv_bfloat16* out;
     int32_t* status;
@@ -79,6 +81,20 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
         if (len_ok(len, a.n_q, a.capacity, a.max_len))
             run += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
         a.cum[bj + 1] = run;
+    }
+    // first query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
+    // the first bj with cum[bj + 1] > p T / pairs (the attention kernel reads it
+    // instead of searching the prefix itself)
+    __syncthreads();
+    const int T = a.cum[a.BJ];
+    for (int p = tid; p < a.pairs; p += kThreads) {
+        const int s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
+        int lo = 0, hi = a.BJ;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (a.cum[mid + 1] > s0) hi = mid; else lo = mid + 1;
+        }
+        a.first_bj[p] = lo;
     }
 }
 
@@ -320,7 +336,8 @@ int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs&
 }  // namespace
 
 // absorb + q-RoPE + plan.  q_nope [BJ][H][128], W_uk [H][512][128], q_rope [BJ][H][64]
-int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* launches) {
+int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32_t* first_bj, int pairs,
+                  int* launches) {
     const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 128);
     CUtensorMap A, B;
     {
@@ -345,6 +362,8 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int* 
     rope_turn_table(c.d.rope_base, 64, a.rope_turn);
     a.q_lat = q_lat;
     a.cum = cum;
+    a.first_bj = first_bj;
+    a.pairs = pairs;
     a.status = c.status;
     const dim3 grid(H, 4, (BJ + N - 1) / N);
     return launch(absorb_kernel, A, B, a, grid, 2 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches,
