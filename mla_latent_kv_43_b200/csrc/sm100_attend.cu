@@ -57,7 +57,6 @@ namespace {
 
 constexpr int kKeys = 64;
 constexpr int kStages = 4;
-constexpr int kPrefetchTiles = 4;                  // L2 prefetch distance beyond the loads
 constexpr int kLatBox = 8192;                      // 64 keys x 64 columns x 2 B
 constexpr int kRopeBox = 4096;                     // 64 keys x 32 columns x 2 B
 constexpr int kStageBytes = 4 * kLatBox + kRopeBox;
@@ -227,40 +226,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             ItemIter iter;
             iter.init(a, pair);
             Item item;
-            // L2 prefetch runs kPrefetchTiles tiles ahead of the shared-memory loads,
-            // so a stage that frees up is refilled from L2 rather than from HBM
-            ItemIter pf_iter;
-            pf_iter.init(a, pair);
-            Item pf_item;
-            bool pf_have = pf_iter.next(pf_item);
-            int pf_t = pf_have ? pf_item.t0 : 0;
-            auto prefetch_skip_next = [&]() {      // advance without prefetching
-                if (!pf_have) return;
-                if (++pf_t == pf_item.t1) {
-                    pf_have = pf_iter.next(pf_item);
-                    if (pf_have) pf_t = pf_item.t0;
-                }
-            };
-            auto prefetch_next = [&]() {
-                if (!pf_have) return;
-                const int pb = pf_item.bj / a.n_q;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) tma_prefetch_l2_3d(&map_lat, 256 * rank + 64 * i, pf_t * kKeys, pb);
-                tma_prefetch_l2_3d(&map_rope, 512 + 32 * rank, pf_t * kKeys, pb);
-                if (++pf_t == pf_item.t1) {
-                    pf_have = pf_iter.next(pf_item);
-                    if (pf_have) pf_t = pf_item.t0;
-                }
-            };
-            // the prefetch starts once the ring has cycled: the first stages' loads
-            // are not made to share the start-up burst with it
-            for (int i = 0; i < kStages + kPrefetchTiles; ++i) prefetch_skip_next();
             uint32_t it = 0;
             bool ok = true;
             while (ok && iter.next(item)) {
                 const int b = item.bj / a.n_q;
                 for (int t = item.t0; t < item.t1; ++t, ++it) {
-                    if (it >= kStages) prefetch_next();
                     const int s = it % kStages;
                     if (it >= kStages && !mbar_wait(&empty[s], ((it / kStages) - 1) & 1, abort)) {
                         ok = false;

@@ -59,14 +59,15 @@ combine_kernel(const int32_t* __restrict__ cum, int BJ, int pairs, const __nv_bf
     auto empty = [&](int p) { return start(p) == (p + 1 < pairs ? start(p + 1) : T); };
     // pieces in batches of kBatch: every load of a batch (log-sum-exps and partial
     // rows) is issued before any is used, so a batch costs one memory round trip
-    constexpr int kBatch = 4;
+    // (two pieces per batch keep the registers low enough for ~1.5 waves)
+    constexpr int kBatch = 2;
     float acc[16];
     for (int i = 0; i < 16; ++i) acc[i] = 0.f;
     float wsum = 0.f;
     float M = -INFINITY;
     int p0 = pf;
     while (p0 <= pl) {
-        int slots[kBatch] = {0, 0, 0, 0};
+        int slots[kBatch] = {};
         int np = 0;
         for (; p0 <= pl && np < kBatch; ++p0) {
             if (p0 == pf || !empty(p0)) {
