@@ -123,9 +123,15 @@ MLA_API int mla_rope(const mla_dims* dims, int64_t n_rows, void* x, int64_t row_
  * rounded once to dims->dtype.
  *   x          (device) [batch*n_new][hidden]; token i of sequence b is row b*n_new+i.
  *   W_dkv      (device) [hidden][d_c + d_rope].
- *   rms_gamma  must be NULL (latent RMSNorm is not implemented: MLA_ERR_UNSUPPORTED).
- *   positions  (device) int32[batch*n_new]: slot of each new token.  A position
- *              outside [0, capacity) sets MLA_ERR_POS and that row is not written.
+ *   rms_gamma  (device) float[d_c] or NULL.  Non-NULL: the latent alone is
+ *              RMS-normalised before it is stored, latent = gamma * y[0:d_c] /
+ *              sqrt(mean(y[0:d_c]^2) + 1e-6) ("Understanding MLA", Phase A step
+ *              A2; the pages give no epsilon, 1e-6 is the usual choice); the rope
+ *              key is not normalised.  On the bf16 path y[0:d_c] is rounded to
+ *              bf16 once before the normalisation and once after it.
+ *   positions  (device) int32[batch*n_new]: slot of each new token, distinct
+ *              within a sequence.  A position outside [0, capacity) sets
+ *              MLA_ERR_POS and that row is not written.
  *   cache      (device) [batch][capacity][d_c + d_rope]; only the addressed slots
  *              are written, every other byte is left untouched.
  *   status     (device) int32 status word. */

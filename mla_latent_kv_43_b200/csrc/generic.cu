@@ -319,6 +319,57 @@ int generic_append(const AppendCall& c, int* launches) {
     return c.d.dtype == MLA_FP32 ? append_t<float>(c, launches) : append_t<__nv_bfloat16>(c, launches);
 }
 
+namespace {
+
+// RMSNorm of the latent of each appended row, in place ("Understanding MLA",
+// Phase A step A2): row[0:d_c] = gamma * row / sqrt(mean(row^2) + 1e-6), the
+// rope columns untouched.  One block per new token; rows whose position is
+// outside the cache were not written (the append kernel set MLA_ERR_POS).
+template <typename T>
+__global__ void rms_rows_kernel(int d_c, int D, int n_new, const int32_t* __restrict__ positions,
+                                const float* __restrict__ gamma, T* cache, int64_t capacity) {
+    __shared__ float part[32];
+    const int m = blockIdx.x;
+    const int64_t pos = positions[m];
+    if (pos < 0 || pos >= capacity) return;
+    T* row = cache + ((int64_t)(m / n_new) * capacity + pos) * D;
+    float ss = 0.f;
+    for (int i = threadIdx.x; i < d_c; i += blockDim.x) {
+        const float v = to_f32(row[i]);
+        ss = fmaf(v, v, ss);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float v = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (threadIdx.x == 0) part[0] = v;
+    }
+    __syncthreads();
+    const float inv = 1.f / sqrtf(part[0] / (float)d_c + 1e-6f);
+    for (int i = threadIdx.x; i < d_c; i += blockDim.x) row[i] = from_f32<T>(gamma[i] * to_f32(row[i]) * inv);
+}
+
+}  // namespace
+
+int rms_norm_rows(const AppendCall& c, int* launches) {
+    const int M = c.batch * c.n_new, D = c.d.d_c + c.d.d_rope;
+    if (M == 0) return MLA_OK;
+    prof_begin(c.stream, "rms_norm_rows");
+    if (c.d.dtype == MLA_FP32)
+        rms_rows_kernel<float><<<M, 128, 0, c.stream>>>(c.d.d_c, D, c.n_new, c.positions, c.rms_gamma,
+                                                        (float*)c.cache, c.capacity);
+    else
+        rms_rows_kernel<__nv_bfloat16><<<M, 128, 0, c.stream>>>(c.d.d_c, D, c.n_new, c.positions, c.rms_gamma,
+                                                                (__nv_bfloat16*)c.cache, c.capacity);
+    prof_end(c.stream);
+    if (launches) ++*launches;
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
               const int32_t* positions, cudaStream_t stream) {
     const int64_t total = n_rows * (d.d_rope / 2);

@@ -25,6 +25,7 @@ struct AppendCall {
     mla_dims d;
     int batch, n_new, hidden;
     const void *x, *W_dkv;
+    const float* rms_gamma;   // [d_c] or nullptr
     const int32_t* positions;
     void* cache;
     int64_t capacity;
@@ -50,6 +51,8 @@ int generic_append(const AppendCall& c, int* launches);
 int sm100_append(const AppendCall& c, int* launches);
 int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
               const int32_t* positions, cudaStream_t stream);
+// RMSNorm of the latent of every appended row (after either append kernel).
+int rms_norm_rows(const AppendCall& c, int* launches);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

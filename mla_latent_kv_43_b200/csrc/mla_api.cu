@@ -85,10 +85,9 @@ int mla_append(const mla_dims* dims, int32_t batch, int32_t n_new, int32_t hidde
     int rc = validate_dims(dims);
     if (rc) return rc;
     if (batch < 0 || n_new < 0 || hidden <= 0 || capacity <= 0) return MLA_ERR_ARG;
-    if (rms_gamma) return MLA_ERR_UNSUPPORTED;
     if (batch == 0 || n_new == 0) return MLA_OK;
     if (!x || !W_dkv || !positions || !cache || !status) return MLA_ERR_ARG;
-    mla::AppendCall c{*dims, batch, n_new, hidden, x, W_dkv, positions, cache, capacity, status,
+    mla::AppendCall c{*dims, batch, n_new, hidden, x, W_dkv, rms_gamma, positions, cache, capacity, status,
                       (cudaStream_t)stream};
     int launches = 0;
     if (mla::sm100_append_supported(*dims, hidden)) {
@@ -97,6 +96,7 @@ int mla_append(const mla_dims* dims, int32_t batch, int32_t n_new, int32_t hidde
     } else {
         rc = mla::generic_append(c, &launches);
     }
+    if (rc == MLA_OK && rms_gamma) rc = mla::rms_norm_rows(c, &launches);
     g_last_launches = launches;
     return rc;
 }

@@ -21,7 +21,8 @@ What it computes, and where each step is stated:
 * The append step: one projection x W_DKV to d_c + d_R values, split into
   the latent and the rope key, rope key rotated at the token's position
   (Phase A, step A1; "Multi-head latent attention" on aicassindra,
-  "End-to-end flow").
+  "End-to-end flow"); optionally the latent alone RMS-normalised first
+  (Phase A, step A2; epsilon 1e-6, which the pages do not give).
 * An absorbed variant, used only to check the regrouping
   Q_nope . (W_K c) = (Q_nope W_K) . c ("Understanding MLA", section 4).
 
@@ -185,15 +186,31 @@ def decode_absorbed(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, n_q: int
 # ---------------------------------------------------------------------------
 # Append ("Understanding MLA", Phase A step A1, Phase B step B2)
 # ---------------------------------------------------------------------------
-def append_rows(x, W_dkv, positions, d_c: int, base: float = 10000.0) -> np.ndarray:
+RMS_EPS = 1e-6   # not given by the pages: the usual RMSNorm epsilon (a reading)
+
+
+def rms_norm(c, gamma, eps: float = RMS_EPS) -> np.ndarray:
+    """RMSNorm of each row: gamma * c / sqrt(mean(c^2) + eps), one shared RMS
+    over the whole row ("Understanding MLA", Phase A step A2)."""
+    c = _f64(c)
+    rms = np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + eps)
+    return _f64(gamma) * c / rms
+
+
+def append_rows(x, W_dkv, positions, d_c: int, base: float = 10000.0, rms_gamma=None,
+                eps: float = RMS_EPS) -> np.ndarray:
     """Cache rows for new tokens: [latent (d_c) || rotated rope key (d_R)].
 
     x [M][hidden], W_dkv [hidden][d_c + d_R], positions [M].  One projection
     to d_c + d_R values, split into the latent (first d_c) and the rope key
-    (last d_R); only the rope key is rotated, at the token's position.
+    (last d_R); only the rope key is rotated, at the token's position.  With
+    ``rms_gamma`` [d_c] the latent alone is RMS-normalised before it is cached
+    and the rope key is left as it is ("Understanding MLA", Phase A step A2).
     """
     y = _f64(x) @ _f64(W_dkv)                                   # [M][d_c + d_R]
     rows = y.copy()
+    if rms_gamma is not None:
+        rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)
     rows[:, d_c:] = rope(y[:, d_c:], np.asarray(positions), base)
     return rows
 

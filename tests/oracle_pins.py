@@ -272,6 +272,44 @@ def pin_append_brute_force(O):
             _close(rows[m, d_c + 2 * i + 1], a * math.sin(ang) + b * math.cos(ang), rtol=1e-12, atol=1e-13)
 
 
+def pin_append_rms_norm(O):
+    """RMSNorm of the latent at append ("Understanding MLA", Phase A step A2):
+    with gamma = 1 the cached latent has root-mean-square 1 (up to eps), it is
+    unchanged when x is scaled (the norm divides the scale out), gamma scales it
+    linearly, the rope key is exactly the un-normalised one, and explicit loops
+    on a tiny input give the same values."""
+    rng = np.random.default_rng(31)
+    M, hidden, d_c, d_r = 4, 7, 6, 4
+    x = rng.standard_normal((M, hidden))
+    W = rng.standard_normal((hidden, d_c + d_r))
+    pos = np.array([0, 3, 17, 4096])
+    ones = np.ones(d_c)
+    rows = O.append_rows(x, W, pos, d_c, rms_gamma=ones, eps=0.0)
+    _close(np.sqrt(np.mean(rows[:, :d_c] ** 2, axis=1)), np.ones(M), rtol=1e-13)
+    _close(O.append_rows(7.5 * x, W, pos, d_c, rms_gamma=ones, eps=0.0)[:, :d_c], rows[:, :d_c], rtol=1e-13)
+    g = rng.uniform(0.5, 2.0, d_c)
+    _close(O.append_rows(x, W, pos, d_c, rms_gamma=g, eps=0.0)[:, :d_c], rows[:, :d_c] * g, rtol=1e-13)
+    plain = O.append_rows(x, W, pos, d_c)
+    assert np.array_equal(rows[:, d_c:], plain[:, d_c:])
+    eps = 1e-6
+    rows = O.append_rows(x, W, pos, d_c, rms_gamma=g, eps=eps)
+    for m in range(M):
+        y = [sum(x[m, k] * W[k, n] for k in range(hidden)) for n in range(d_c)]
+        ms = sum(v * v for v in y) / d_c
+        _close(rows[m, :d_c], [g[n] * y[n] / math.sqrt(ms + eps) for n in range(d_c)], rtol=1e-13)
+
+
+def pin_rms_norm_does_not_commute_with_up_projection(O):
+    """The page's remark that W RMSNorm(c) != RMSNorm(W c): the norm has to be
+    applied to the cached latent itself, before any head's up-projection."""
+    rng = np.random.default_rng(32)
+    c = rng.standard_normal((3, 8))
+    W = rng.standard_normal((8, 5))
+    a = O.rms_norm(c, np.ones(8)) @ W
+    b = O.rms_norm(c @ W, np.ones(5))
+    assert np.max(np.abs(a - b)) > 1e-3
+
+
 def pin_cache_arithmetic(O):
     """Per-token storage figures printed on the pages."""
     g = json.load(open(os.path.join(GOLDEN, "cache_arithmetic.json")))

@@ -109,7 +109,9 @@ def test_append_argument_checks():
                                   k.get("x", FAKE), k.get("W", FAKE), k.get("gamma", None),
                                   k.get("pos", FAKE), k.get("cache", FAKE), k.get("cap", 10),
                                   k.get("status", FAKE), None)
-    assert ok(gamma=FAKE) == B.CODES["MLA_ERR_UNSUPPORTED"]
+    # a gamma is accepted (latent RMSNorm); argument errors are still reported
+    # before anything is launched
+    assert ok(gamma=FAKE, cache=None) == B.CODES["MLA_ERR_ARG"]
     assert ok(cache=None) == B.CODES["MLA_ERR_ARG"]
     assert ok(pos=None) == B.CODES["MLA_ERR_ARG"]
     assert ok(status=None) == B.CODES["MLA_ERR_ARG"]

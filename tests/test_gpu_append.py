@@ -22,7 +22,7 @@ CASES = {"fp32_small": ("fp32", SMALL, 24), "bf16_small": ("bf16", SMALL, 40),
          "bf16_v3": ("bf16", V3, 7168)}
 
 
-def run_append(case, positions, batch, n_new, capacity, seed=0):
+def run_append(case, positions, batch, n_new, capacity, seed=0, gamma=None):
     dtype, g, hidden = CASES[case]
     tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
     rng = np.random.default_rng(seed)
@@ -36,7 +36,8 @@ def run_append(case, positions, batch, n_new, capacity, seed=0):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     dims = B.make_dims(dtype=dtype, **g)
     pos = torch.tensor(positions, dtype=torch.int32)
-    B.mla_append(dims, x.cuda(), W.cuda(), pos.cuda(), cache, status, batch=batch, n_new=n_new)
+    g = None if gamma is None else torch.as_tensor(gamma, dtype=torch.float32).cuda()
+    B.mla_append(dims, x.cuda(), W.cuda(), pos.cuda(), cache, status, batch=batch, n_new=n_new, rms_gamma=g)
     code = B.mla_get_status(status)
     return dims, x, W, pos, before, cache, code
 
@@ -101,3 +102,31 @@ def test_tensor_core_append_shapes(hidden, tokens):
     rows = O.append_rows(x, W, positions, dims.d_c, dims.rope_base)
     got = np.stack([cache[r, p].double().cpu().numpy() for r, p in enumerate(positions)])
     assert rel_err(got, rows) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_append_rms_norm_of_the_latent(case):
+    """rms_gamma: the latent alone is RMS-normalised before it is cached
+    ("Understanding MLA", Phase A step A2); the rope key is bit-identical to the
+    un-normalised append; other slots keep the sentinel; a position outside the
+    cache still sets MLA_ERR_POS and leaves its slot alone."""
+    batch, n_new, cap = 3, 2, 12
+    positions = [5, 6, 0, 1, 10, cap]                   # the last one is outside
+    dtype, g, hidden = CASES[case]
+    gamma = np.random.default_rng(5).uniform(0.5, 2.0, g["d_c"]).astype(np.float32)
+    dims, x, W, pos, before, cache, code = run_append(case, positions, batch, n_new, cap, seed=4, gamma=gamma)
+    _, _, _, _, _, plain, _ = run_append(case, positions, batch, n_new, cap, seed=4)
+    assert code == B.CODES["MLA_ERR_POS"]
+    d_c = dims.d_c
+    rows = O.append_rows(x, W, positions, d_c, dims.rope_base, rms_gamma=gamma)
+    valid = [(r, p) for r, p in enumerate(positions) if p < cap]
+    got = np.stack([cache[r // n_new, p].double().cpu().numpy() for r, p in valid])
+    ref = np.stack([rows[r] for r, _ in valid])
+    tol = TOL["fp32"] if case.startswith("fp32") else TOL["bf16"]
+    assert rel_err(got[:, :d_c], ref[:, :d_c]) <= tol
+    for r, p in valid:
+        assert torch.equal(cache[r // n_new, p, d_c:], plain[r // n_new, p, d_c:])
+    mask = torch.ones(batch, cap, dtype=torch.bool)
+    for r, p in valid:
+        mask[r // n_new, p] = False
+    assert torch.equal(cache[mask], before[mask])

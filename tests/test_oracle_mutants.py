@@ -37,6 +37,13 @@ MUTANTS = [
     ("append split taken from the wrong end", "y = _f64(x) @ _f64(W_dkv)", "y = np.roll(_f64(x) @ _f64(W_dkv), 3, axis=1)"),
     ("appended row written one slot late", "c[b, pos[b, i]] = r[:d_c]", "c[b, pos[b, i] - 1] = r[:d_c]"),
     ("mha cache count without the value", "return heads * (qk_dim + v_dim)", "return heads * qk_dim"),
+    ("rms over the sum instead of the mean", "np.mean(c * c, axis=-1, keepdims=True)",
+     "np.sum(c * c, axis=-1, keepdims=True)"),
+    ("rms norm applied to the rope key too", "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)",
+     "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)\n        rows[:, d_c:] = y[:, d_c:] / np.sqrt(np.mean(y[:, d_c:] ** 2, axis=-1, keepdims=True) + eps)\n        y = rows"),
+    ("rms norm without gamma", "return _f64(gamma) * c / rms", "return c / rms"),
+    ("rms epsilon outside the square root", "np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + eps)",
+     "np.sqrt(np.mean(c * c, axis=-1, keepdims=True)) + eps"),
 ]
 
 
