@@ -75,6 +75,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
     int32_t run = incl - sum;
     for (int w = 0; w < warp; ++w) run += part[w];
     if (tid == 0) a.cum[0] = 0;
+    const int32_t run_lo = run;                 // cum[lo]
     for (int bj = lo; bj < hi; ++bj) {
         const int b = bj / a.n_q, j = bj % a.n_q;
         const int64_t len = a.seq_lens[b];
@@ -82,19 +83,31 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
             run += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
         a.cum[bj + 1] = run;
     }
-    // first query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
-    // the first bj with cum[bj + 1] > p T / pairs (the attention kernel reads it
-    // instead of searching the prefix itself)
-    __syncthreads();
-    const int T = a.cum[a.BJ];
-    for (int p = tid; p < a.pairs; p += kThreads) {
+    // First query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
+    // the first bj with cum[bj + 1] > floor(p T / pairs).  The thread whose prefix
+    // range [cum[lo], cum[hi]) holds that start answers from its own values: those
+    // are the clusters p with ceil(cum[lo] pairs / T) <= p < ceil(cum[hi] pairs / T).
+    int32_t T = 0;
+    for (int w = 0; w < kThreads / 32; ++w) T += part[w];
+    if (T == 0) {
+        for (int p = tid; p < a.pairs; p += kThreads) a.first_bj[p] = a.BJ;
+        return;
+    }
+    const int p0 = (int)(((int64_t)run_lo * a.pairs + T - 1) / T);
+    const int p1 = min(a.pairs, (int)(((int64_t)run * a.pairs + T - 1) / T));
+    for (int p = p0; p < p1; ++p) {
         const int s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        int lo = 0, hi = a.BJ;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (a.cum[mid + 1] > s0) hi = mid; else lo = mid + 1;
+        int32_t c = run_lo;
+        for (int bj = lo; bj < hi; ++bj) {
+            const int b = bj / a.n_q, j = bj % a.n_q;
+            const int64_t len = a.seq_lens[b];
+            if (len_ok(len, a.n_q, a.capacity, a.max_len))
+                c += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
+            if (c > s0) {
+                a.first_bj[p] = bj;
+                break;
+            }
         }
-        a.first_bj[p] = lo;
     }
 }
 
