@@ -167,14 +167,26 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
+def oracle_decode(O, w, host, batches, heads=None, k_rot=None):
+    """The oracle's decode of the workload for the given sequences: over every
+    visible key, or over the selected keys of a top-k workload (whose cache,
+    rotated once outside the timing, is ``k_rot``)."""
+    if w.top_k:
+        return O.decode_sparse(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"], host["c_kv"], k_rot,
+                               host["seq_lens"], host["sel"].numpy(), host["n_sel"].numpy(), w.n_q,
+                               w.softmax_scale, w.rope_base, batches=batches, heads=heads)
+    return O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=batches, heads=heads)
+
+
 def cpu_sample(w, host, budget_s: float):
     """Time the fp64 oracle on whole sequences (all heads) until the budget is
     spent; returns (query-tokens/s, description, threads)."""
     from oracle import mla_oracle as O
+    k_rot = O.rope_cache(host["k_rope"], host["seq_lens"], w.rope_base) if w.top_k else None
     t0 = time.perf_counter()
     done = 0
     for b in range(w.batch):
-        O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=[b])
+        oracle_decode(O, w, host, [b], k_rot=k_rot)
         done += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -192,9 +204,9 @@ def run_reference(a, rank, world):
     w = gen.WORKLOADS[a.workload]
     host = gen.generate(w)
     heads = list(range(0, w.heads, max(1, w.heads // 16)))[:16]
+    k_rot = O.rope_cache(host["k_rope"], host["seq_lens"], w.rope_base) if w.top_k else None
     def one(k):
-        O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=[k % w.batch],
-                      heads=heads)
+        oracle_decode(O, w, host, [k % w.batch], heads=heads, k_rot=k_rot)
     for k in range(a.warmup):
         one(k)
     t0 = time.perf_counter()
@@ -290,6 +302,10 @@ def run_ours(a, rank, world, local):
     if prob.has_append:
         h_x = host["x"].pin_memory()
         h2d += h_x.numel() * h_x.element_size()
+    if prob.sparse:                       # the selection arrives with the queries
+        h_sel = host["sel"].pin_memory()
+        h_nsel = host["n_sel"].pin_memory()
+        h2d += (h_sel.numel() + h_nsel.numel()) * 4
     d2h = h_out.numel() * h_out.element_size()
     e2e_ms = 0.0
     barrier(world)
@@ -302,6 +318,9 @@ def run_ours(a, rank, world, local):
         prob.seq_lens.copy_(h_len, non_blocking=True)
         if prob.has_append:
             prob.x.copy_(h_x, non_blocking=True)
+        if prob.sparse:
+            prob.sel.copy_(h_sel, non_blocking=True)
+            prob.n_sel.copy_(h_nsel, non_blocking=True)
         prob.step()
         h_out.copy_(prob.out, non_blocking=True)
         e.record(stream)

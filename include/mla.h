@@ -54,7 +54,8 @@ enum mla_status {
     MLA_ERR_CUDA = 5,         /* a CUDA launch or API call failed */
     MLA_ERR_LEN = 6,          /* device: len_b < n_q, len_b > capacity or len_b > max_len */
     MLA_ERR_POS = 7,          /* device: an append position outside [0, capacity) */
-    MLA_ERR_TIMEOUT = 8       /* device: a bounded wait inside a kernel expired */
+    MLA_ERR_TIMEOUT = 8,      /* device: a bounded wait inside a kernel expired */
+    MLA_ERR_INDEX = 9         /* device: a selected cache slot outside the query's visible keys */
 };
 
 /* Model geometry.  The per-head query/key width is qk_nope + d_rope and the
@@ -166,6 +167,30 @@ MLA_API int mla_append(const mla_dims* dims, int32_t batch, int32_t n_new, int32
 MLA_API int mla_decode(const mla_dims* dims, int32_t batch, int32_t n_q,
                const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
                const void* cache, int64_t capacity, const int32_t* seq_lens, int64_t max_len,
+               void* out, void* workspace, size_t workspace_bytes, int32_t splits,
+               int32_t* status, void* stream);
+
+/* Absorbed MLA decode over a selected subset of each query's cached keys
+ * ("Multi-Head Latent Attention", section 4: a selector picks a top-k subset of
+ * the cached latents for every query -- k = 2048 in DeepSeek-V3.2 -- and MLA
+ * runs unchanged on that subset; the selector itself is not part of this
+ * library).  Arguments as mla_decode, plus
+ *   sel      (device) int32[batch][n_q][max_sel]: the cache slots query (b, j)
+ *            attends, distinct, each in [0, p] for the query's position p;
+ *            entries past n_sel are ignored.  Their order does not matter.
+ *   n_sel    (device) int32[batch][n_q]: how many leading entries of sel are
+ *            used, 1 <= n_sel <= min(max_sel, p + 1); any other count sets
+ *            MLA_ERR_LEN and that query's outputs are zero.
+ *   max_sel  (host) row length of sel, 1 <= max_sel <= max_len.
+ * A slot outside [0, p] sets MLA_ERR_INDEX and the call's outputs are then
+ * unspecified (finite).  Implemented on the tensor-core path (bf16 with the
+ * DeepSeek-V3 head geometry); other dims return MLA_ERR_UNSUPPORTED.  The
+ * workspace is mla_decode_workspace_bytes(dims, batch, n_q, max_sel, splits)
+ * bytes; batch * capacity must fit in 31 bits. */
+MLA_API int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q,
+               const void* q_nope, const void* q_rope, const void* W_uk, const void* W_uv,
+               const void* cache, int64_t capacity, const int32_t* seq_lens, int64_t max_len,
+               const int32_t* sel, const int32_t* n_sel, int32_t max_sel,
                void* out, void* workspace, size_t workspace_bytes, int32_t splits,
                int32_t* status, void* stream);
 

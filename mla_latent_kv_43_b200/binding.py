@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmla.so")
 MLA_BF16, MLA_FP32 = 0, 1
 STATUS = {0: "MLA_OK", 1: "MLA_ERR_ARG", 2: "MLA_ERR_ALIGN", 3: "MLA_ERR_WORKSPACE",
           4: "MLA_ERR_UNSUPPORTED", 5: "MLA_ERR_CUDA", 6: "MLA_ERR_LEN", 7: "MLA_ERR_POS",
-          8: "MLA_ERR_TIMEOUT"}
+          8: "MLA_ERR_TIMEOUT", 9: "MLA_ERR_INDEX"}
 CODES = {v: k for k, v in STATUS.items()}
 
 
@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.mla_append.restype = ctypes.c_int
         L.mla_decode.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, SZ, I32, P, P]
         L.mla_decode.restype = ctypes.c_int
+        L.mla_decode_sparse.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, I32, P, P, SZ, I32, P, P]
+        L.mla_decode_sparse.restype = ctypes.c_int
         L.mla_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.mla_get_status.restype = ctypes.c_int
         L.mla_status_string.argtypes = [ctypes.c_int]
@@ -149,6 +151,19 @@ def mla_decode(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: 
                             _ptr(W_uv), _ptr(cache), cache.shape[1], _ptr(seq_lens), max_len,
                             _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
                             splits, _ptr(status), _stream(stream)), "mla_decode")
+
+
+def mla_decode_sparse(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor,
+                      W_uv: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor, max_len: int,
+                      sel: torch.Tensor, n_sel: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor,
+                      status: torch.Tensor, splits: int = 0, stream=None):
+    """Decode over the selected cache slots sel[b][j][:n_sel[b][j]] of each query."""
+    batch, n_q = q_nope.shape[0], q_nope.shape[1]
+    _check(lib().mla_decode_sparse(ctypes.byref(dims), batch, n_q, _ptr(q_nope), _ptr(q_rope), _ptr(W_uk),
+                                   _ptr(W_uv), _ptr(cache), cache.shape[1], _ptr(seq_lens), max_len,
+                                   _ptr(sel), _ptr(n_sel), sel.shape[-1], _ptr(out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), splits, _ptr(status),
+                                   _stream(stream)), "mla_decode_sparse")
 
 
 def mla_decode_noalloc(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor,

@@ -19,6 +19,10 @@ struct DecodeCall {
     mla_ws_layout L;
     int32_t* status;
     cudaStream_t stream;
+    // sparse decode (mla_decode_sparse): selected slots, counts, row length
+    const int32_t* sel = nullptr;
+    const int32_t* n_sel = nullptr;
+    int max_sel = 0;
 };
 
 struct AppendCall {

@@ -130,6 +130,40 @@ int mla_decode(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_n
     return rc;
 }
 
+int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_nope,
+                      const void* q_rope, const void* W_uk, const void* W_uv, const void* cache,
+                      int64_t capacity, const int32_t* seq_lens, int64_t max_len, const int32_t* sel,
+                      const int32_t* n_sel, int32_t max_sel, void* out, void* workspace,
+                      size_t workspace_bytes, int32_t splits, int32_t* status, void* stream) {
+    g_last_launches = 0;
+    int rc = validate_dims(dims);
+    if (rc) return rc;
+    if (batch < 0 || n_q < 0 || splits < 0 || capacity <= 0) return MLA_ERR_ARG;
+    if (batch == 0 || n_q == 0) return MLA_OK;
+    if (max_len < n_q || max_len > capacity || max_sel < 1 || max_sel > max_len) return MLA_ERR_ARG;
+    if (!q_nope || !q_rope || !W_uk || !W_uv || !cache || !seq_lens || !sel || !n_sel || !out || !workspace ||
+        !status)
+        return MLA_ERR_ARG;
+    if (!use_sm100_decode(*dims)) return MLA_ERR_UNSUPPORTED;
+    if ((int64_t)batch * capacity >= ((int64_t)1 << 31)) return MLA_ERR_UNSUPPORTED;
+    mla_ws_layout L;
+    if ((rc = layout_for(dims, batch, n_q, max_sel, splits, &L))) return rc;
+    if (workspace_bytes < L.total) return MLA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_ALIGN;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache) ||
+        !aligned16(out))
+        return MLA_ERR_ALIGN;
+    mla::DecodeCall c{*dims, batch, n_q, q_nope, q_rope, W_uk, W_uv, cache, capacity, seq_lens,
+                      max_len, out, static_cast<char*>(workspace), L, status, (cudaStream_t)stream};
+    c.sel = sel;
+    c.n_sel = n_sel;
+    c.max_sel = max_sel;
+    int launches = 0;
+    rc = mla::sm100_decode(c, &launches);
+    g_last_launches = launches;
+    return rc;
+}
+
 int mla_get_status(int32_t* status, void* stream, int32_t* host_status) {
     if (!status || !host_status) return MLA_ERR_ARG;
     cudaStream_t s = (cudaStream_t)stream;
@@ -151,6 +185,7 @@ const char* mla_status_string(int code) {
         case MLA_ERR_LEN: return "MLA_ERR_LEN";
         case MLA_ERR_POS: return "MLA_ERR_POS";
         case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+        case MLA_ERR_INDEX: return "MLA_ERR_INDEX";
         default: return "MLA_ERR_UNKNOWN";
     }
 }

@@ -80,22 +80,30 @@ struct AttnArgs {
     __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
     float* part_lse;              // [2 * pairs][128], log2 domain
     int32_t* status;
+    // sparse decode: the selected slots of each query token and their count
+    const int32_t* sel;           // [BJ][max_sel]
+    const int32_t* n_sel;         // [BJ] (nullptr: dense decode over keys 0..p)
+    int max_sel;
+    int64_t capacity;
 };
 
 struct Item {
-    int bj, t0, t1, n_vis, slot;  // slot < 0: finished here
+    int bj, t0, t1, n_vis, slot;  // slot < 0: finished here; n_vis: keys this token attends
+    int p;                        // the query's position
 };
 
 // Pieces of the concatenated tile range [s0, s1) of one cluster, in order.
 struct ItemIter {
     const int32_t* cum;
     const int32_t* lens;
+    const int32_t* n_sel;
     int BJ, n_q, bj, s0, s1, pair;
     __device__ void init(const AttnArgs& a, int p) {
         cum = a.cum;
         BJ = a.BJ;
         n_q = a.n_q;
         lens = a.seq_lens;
+        n_sel = a.n_sel;
         pair = p;
         const int T = cum[BJ];
         s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
@@ -114,7 +122,8 @@ struct ItemIter {
             it.t0 = lo - c0;
             it.t1 = hi - c0;
             const int b = cur / n_q, j = cur % n_q;
-            it.n_vis = (int)(query_pos(lens[b], n_q, j) + 1);
+            it.p = (int)query_pos(lens[b], n_q, j);
+            it.n_vis = n_sel ? n_sel[cur] : it.p + 1;
             it.slot = (c0 >= s0 && c1 <= s1) ? -1 : (c0 < s0 ? 2 * pair : 2 * pair + 1);
             return true;
         }
@@ -149,6 +158,9 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// kSparse: the key tiles are gathered rows (tile::gather4 from 2-D maps over
+// [batch * capacity][576]); otherwise 64 consecutive keys (3-D maps).
+template <bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
               AttnArgs a) {
@@ -245,10 +257,38 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     uint8_t* st = smem + s * kStageBytes;
                     mbar_expect_tx(&full[s], kStageBytes);
                     const int key0 = t * kKeys;
+                    if constexpr (kSparse) {
+                        // the tile's 64 selected slots (padded with the first one past the
+                        // count; those rows are masked and zeroed before the latent GEMM)
+                        const int32_t* srow = a.sel + (int64_t)item.bj * a.max_sel + key0;
+                        const int n = min(kKeys, item.n_vis - key0);
+                        const int32_t rowbase = b * (int32_t)a.capacity;
+                        int32_t rows[kKeys];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        tma_load_3d(st + i * kLatBox, &map_lat, &full[s], 256 * rank + 64 * i, key0, b);
-                    tma_load_3d(st + 4 * kLatBox, &map_rope, &full[s], 512 + 32 * rank, key0, b);
+                        for (int i = 0; i < kKeys; ++i) rows[i] = srow[i < n ? i : 0];
+                        bool bad = false;
+#pragma unroll
+                        for (int i = 0; i < kKeys; ++i) {
+                            const bool ok_i = rows[i] >= 0 && rows[i] <= item.p;
+                            bad |= !ok_i;
+                            rows[i] = rowbase + (ok_i ? rows[i] : 0);
+                        }
+                        if (bad) set_status(a.status, MLA_ERR_INDEX);
+#pragma unroll
+                        for (int g4 = 0; g4 < kKeys / 4; ++g4) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                tma_gather4(st + i * kLatBox + g4 * 512, &map_lat, &full[s], 256 * rank + 64 * i,
+                                            rows[4 * g4], rows[4 * g4 + 1], rows[4 * g4 + 2], rows[4 * g4 + 3]);
+                            tma_gather4(st + 4 * kLatBox + g4 * 256, &map_rope, &full[s], 512 + 32 * rank, rows[4 * g4],
+                                        rows[4 * g4 + 1], rows[4 * g4 + 2], rows[4 * g4 + 3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            tma_load_3d(st + i * kLatBox, &map_lat, &full[s], 256 * rank + 64 * i, key0, b);
+                        tma_load_3d(st + 4 * kLatBox, &map_rope, &full[s], 512 + 32 * rank, key0, b);
+                    }
                 }
             }
             if (!ok) fail();
@@ -673,12 +713,22 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
                   __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches) {
+    const bool sparse = c.n_sel != nullptr;
     CUtensorMap ml, mr;
-    const uint64_t dims[3] = {576, (uint64_t)c.capacity, (uint64_t)c.batch};
-    const uint64_t str[2] = {576 * 2, (uint64_t)c.capacity * 576 * 2};
-    const uint32_t box_l[3] = {64, 64, 1}, box_r[3] = {32, 64, 1};
-    if (!make_map(&ml, c.cache, 3, dims, str, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-    if (!make_map(&mr, c.cache, 3, dims, str, box_r, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+    if (sparse) {
+        // 2-D view [batch * capacity][576], boxes one row high for tile::gather4
+        const uint64_t dims[2] = {576, (uint64_t)c.capacity * (uint64_t)c.batch};
+        const uint64_t str[1] = {576 * 2};
+        const uint32_t box_l[2] = {64, 1}, box_r[2] = {32, 1};
+        if (!make_map(&ml, c.cache, 2, dims, str, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mr, c.cache, 2, dims, str, box_r, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+    } else {
+        const uint64_t dims[3] = {576, (uint64_t)c.capacity, (uint64_t)c.batch};
+        const uint64_t str[2] = {576 * 2, (uint64_t)c.capacity * 576 * 2};
+        const uint32_t box_l[3] = {64, 64, 1}, box_r[3] = {32, 64, 1};
+        if (!make_map(&ml, c.cache, 3, dims, str, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mr, c.cache, 3, dims, str, box_r, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+    }
     AttnArgs a{};
     a.q_lat = q_lat;
     a.cum = cum;
@@ -692,11 +742,16 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
     a.part_o = part_o;
     a.part_lse = part_lse;
     a.status = c.status;
+    a.sel = c.sel;
+    a.n_sel = c.n_sel;
+    a.max_sel = c.max_sel;
+    a.capacity = c.capacity;
     const size_t smem = kSmemBytes + 1024;
-    if (cudaFuncSetAttribute(attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    auto kernel = sparse ? attend_kernel<true> : attend_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(c.stream, "sm100_attend");
-    const cudaError_t e = launch_pdl(attend_kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, ml, mr, a);
+    const cudaError_t e = launch_pdl(kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, ml, mr, a);
     prof_end(c.stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;

@@ -172,8 +172,10 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
 
 int sm100_decode(const DecodeCall& c, int* launches) {
     // The tile ranges of the clusters are p * T / P in 32-bit arithmetic on the
-    // device (T = total key tiles <= B * n_q * ceil(max_len / 64)).
-    if ((int64_t)c.batch * c.n_q * ((c.max_len + 63) / 64) * c.L.splits >= ((int64_t)1 << 31))
+    // device (T = total key tiles <= B * n_q * ceil(max_len / 64), or
+    // ceil(max_sel / 64) per query for the sparse decode).
+    const int64_t keys_bound = c.n_sel ? c.max_sel : c.max_len;
+    if ((int64_t)c.batch * c.n_q * ((keys_bound + 63) / 64) * c.L.splits >= ((int64_t)1 << 31))
         return MLA_ERR_UNSUPPORTED;
     auto* q_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.q_lat);
     auto* o_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.o_lat);

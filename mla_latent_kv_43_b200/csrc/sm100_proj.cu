@@ -40,10 +40,33 @@ struct ProjArgs {
     int32_t* cum;            // [BJ + 1] key tiles prefix of each query token
     int32_t* first_bj;       // [pairs] first query token of each attention cluster's tile range
     int pairs;
+    const int32_t* n_sel;    // sparse decode: selected keys per query token (nullptr: dense)
+    int max_sel;
     // upproj
     __nv_bfloat16* out;
     int32_t* status;
 };
+
+// Key tiles query token bj attends: its visible keys 0..p, or its selected
+// keys in the sparse decode; 0 (and *bad) when its length or count is invalid.
+__device__ __forceinline__ int32_t tiles_of(const ProjArgs& a, int bj, bool* bad) {
+    const int b = bj / a.n_q, j = bj % a.n_q;
+    const int64_t len = a.seq_lens[b];
+    if (!len_ok(len, a.n_q, a.capacity, a.max_len)) {
+        *bad = true;
+        return 0;
+    }
+    const int64_t p = query_pos(len, a.n_q, j);
+    if (a.n_sel) {
+        const int32_t n = a.n_sel[bj];
+        if (n < 1 || n > a.max_sel || (int64_t)n > p + 1) {
+            *bad = true;
+            return 0;
+        }
+        return (n + kKeysPerTile - 1) / kKeysPerTile;
+    }
+    return (int32_t)((p + kKeysPerTile) / kKeysPerTile);
+}
 
 __device__ void plan_tiles(const ProjArgs& a, int tid) {
     // Tiles of 64 keys each query token attends; 0 for an invalid length.
@@ -52,14 +75,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
     const int lo = min(a.BJ, tid * per), hi = min(a.BJ, lo + per);
     int32_t sum = 0;
     bool bad = false;
-    for (int bj = lo; bj < hi; ++bj) {
-        const int b = bj / a.n_q, j = bj % a.n_q;
-        const int64_t len = a.seq_lens[b];
-        if (len_ok(len, a.n_q, a.capacity, a.max_len))
-            sum += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
-        else
-            bad = true;
-    }
+    for (int bj = lo; bj < hi; ++bj) sum += tiles_of(a, bj, &bad);
     if (bad) set_status(a.status, MLA_ERR_LEN);
     // exclusive prefix of the per-thread sums: shuffle scan in each warp, then
     // the four warp totals
@@ -76,11 +92,9 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
     for (int w = 0; w < warp; ++w) run += part[w];
     if (tid == 0) a.cum[0] = 0;
     const int32_t run_lo = run;                 // cum[lo]
+    bool ignored = false;
     for (int bj = lo; bj < hi; ++bj) {
-        const int b = bj / a.n_q, j = bj % a.n_q;
-        const int64_t len = a.seq_lens[b];
-        if (len_ok(len, a.n_q, a.capacity, a.max_len))
-            run += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
+        run += tiles_of(a, bj, &ignored);
         a.cum[bj + 1] = run;
     }
     // First query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
@@ -99,10 +113,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
         const int s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
         int32_t c = run_lo;
         for (int bj = lo; bj < hi; ++bj) {
-            const int b = bj / a.n_q, j = bj % a.n_q;
-            const int64_t len = a.seq_lens[b];
-            if (len_ok(len, a.n_q, a.capacity, a.max_len))
-                c += (int32_t)((query_pos(len, a.n_q, j) + kKeysPerTile) / kKeysPerTile);
+            c += tiles_of(a, bj, &ignored);
             if (c > s0) {
                 a.first_bj[p] = bj;
                 break;
@@ -351,6 +362,7 @@ int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs&
 // absorb + q-RoPE + plan.  q_nope [BJ][H][128], W_uk [H][512][128], q_rope [BJ][H][64]
 int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32_t* first_bj, int pairs,
                   int* launches) {
+    // (sparse decode: c.n_sel / c.max_sel give the tile counts)
     const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 128);
     CUtensorMap A, B;
     {
@@ -377,6 +389,8 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
     a.cum = cum;
     a.first_bj = first_bj;
     a.pairs = pairs;
+    a.n_sel = c.n_sel;
+    a.max_sel = c.max_sel;
     a.status = c.status;
     const dim3 grid(H, 4, (BJ + N - 1) / N);
     return launch(absorb_kernel, A, B, a, grid, 2 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches,

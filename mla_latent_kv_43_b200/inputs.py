@@ -53,6 +53,7 @@ class Workload:
     latent_rms_norm: bool = False
     hidden: int = 0
     n_new: int = 0
+    top_k: int = 0                  # > 0: each query attends a selected subset of its keys
     rope_base: float = 10000.0
     seed: int = 0
 
@@ -96,6 +97,12 @@ WORKLOADS: Dict[str, Workload] = {
         name="v3_b32_append2", dtype="bf16", batch=32, n_q=2,
         lens=(4098,) * 32, capacity=4098, latent_rms_norm=True, hidden=7168,
         n_new=2, seed=4, **V3),
+    # sparse decode over a top-k selection of the cached keys ("Multi-Head
+    # Latent Attention", section 4: k = 2048 per query); the selection is a
+    # seeded uniform subset of the visible keys, standing in for an indexer
+    "v3_b32_topk2048": Workload(
+        name="v3_b32_topk2048", dtype="bf16", batch=32, n_q=1, lens=(8192,) * 32,
+        capacity=8192, latent_rms_norm=True, top_k=2048, seed=5, **V3),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
@@ -127,7 +134,9 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
     rotated), c_kv [B][cap][d_c], k_rope [B][cap][d_rope] (not yet rotated),
     W_uk [H][d_c][qk_nope], W_uv [H][d_c][v_dim], seq_lens int32 [B]; with
     n_new > 0 also x [B*n_new][hidden], W_dkv [hidden][d_c+d_rope],
-    positions int32 [B*n_new] and old_lens int32 [B].
+    positions int32 [B*n_new] and old_lens int32 [B]; with top_k > 0 also
+    sel int32 [B][n_q][top_k] (distinct visible slots, unused tail entries 0)
+    and n_sel int32 [B][n_q] = min(top_k, p + 1).
     """
     rng = np.random.default_rng(w.seed)
     if w.lens is None:
@@ -159,12 +168,23 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
         pos = (old[:, None] + np.arange(w.n_new, dtype=np.int32)[None, :]).reshape(-1)
         out["positions"] = torch.from_numpy(pos.astype(np.int32))
         out["old_lens"] = torch.from_numpy(old.astype(np.int32))
+    if w.top_k:
+        sel = np.zeros((w.batch, w.n_q, w.top_k), dtype=np.int32)
+        n_sel = np.zeros((w.batch, w.n_q), dtype=np.int32)
+        for b in range(w.batch):
+            for j in range(w.n_q):
+                p = int(lens[b]) - w.n_q + j
+                n = min(w.top_k, p + 1)
+                sel[b, j, :n] = rng.choice(p + 1, size=n, replace=False)
+                n_sel[b, j] = n
+        out["sel"] = torch.from_numpy(sel)
+        out["n_sel"] = torch.from_numpy(n_sel)
     return out
 
 
 def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6,
          v_dim=5, n_q=1, lens=(5, 9), capacity=None, seed=0, latent_rms_norm=False,
-         hidden=0, n_new=0) -> Workload:
+         hidden=0, n_new=0, top_k=0) -> Workload:
     """A small custom workload for pins and edge cases (batch = len(lens))."""
     cap = capacity if capacity is not None else max(lens)
     if batch is None:
@@ -172,4 +192,4 @@ def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6
     return Workload(name="custom", dtype=dtype, batch=batch, heads=heads, d_c=d_c,
                     d_rope=d_rope, qk_nope=qk_nope, v_dim=v_dim, n_q=n_q,
                     lens=tuple(lens), capacity=cap, latent_rms_norm=latent_rms_norm,
-                    hidden=hidden, n_new=n_new, seed=seed)
+                    hidden=hidden, n_new=n_new, top_k=top_k, seed=seed)

@@ -50,6 +50,10 @@ def step_work(w, lens: Sequence[int]) -> Dict[str, float]:
     visible = sum(sum(L - w.n_q + j + 1 for j in range(w.n_q)) for L in keys_per_seq)
     r = {}
     r["cache_bytes"] = sum(keys_per_seq) * D * es
+    if w.top_k:
+        # sparse decode: each query reads only its selected rows (min(k, p + 1) of them)
+        visible = sum(sum(min(w.top_k, L - w.n_q + j + 1) for j in range(w.n_q)) for L in keys_per_seq)
+        r["cache_bytes"] = visible * D * es
     r["weight_bytes"] = H * w.d_c * (w.qk_nope + w.v_dim) * es
     r["q_bytes"] = qt * H * (w.qk_nope + w.d_rope) * es
     r["out_bytes"] = qt * H * w.v_dim * es
@@ -79,7 +83,10 @@ def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_ele
     qt = w.batch * w.n_q
     H = w.heads
     if "attend" in kernel or "core" in kernel:
-        return sum(int(L) for L in lens) * D * es + qt * H * D * q_lat_elem + qt * H * w.d_c * o_lat_elem
+        keys = sum(int(L) for L in lens)
+        if w.top_k:
+            keys = sum(sum(min(w.top_k, int(L) - w.n_q + j + 1) for j in range(w.n_q)) for L in lens)
+        return keys * D * es + qt * H * D * q_lat_elem + qt * H * w.d_c * o_lat_elem
     if "absorb" in kernel:
         return H * w.d_c * w.qk_nope * es + qt * H * (w.qk_nope + w.d_rope) * es + qt * H * D * q_lat_elem
     if "upproj" in kernel:

@@ -5,7 +5,8 @@ the library takes: the cache as [B][capacity][d_c + d_rope] with its rope
 keys rotated at their slot positions by ``mla_rope`` (what the append step
 would have stored), the weights, per-sequence lengths, and caller-owned
 output, workspace and status buffers.  ``step()`` runs one decode step
-(append of the new tokens when the workload has them, then attention).
+(append of the new tokens when the workload has them, then attention: over
+every visible key, or over the selected ones for a top-k workload).
 """
 from __future__ import annotations
 
@@ -44,7 +45,12 @@ class DeviceProblem:
         del slot_pos
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.out = torch.empty(w.batch, w.n_q, w.heads, w.v_dim, dtype=w.torch_dtype, device=dev)
-        self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, self.max_len, splits)
+        self.sparse = w.top_k > 0
+        if self.sparse:
+            self.sel = to(host["sel"])
+            self.n_sel = to(host["n_sel"])
+        ws_len = w.top_k if self.sparse else self.max_len    # the tile bound of the plan
+        self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, ws_len, splits)
         self.workspace = torch.empty(max(self.layout["total"], 256), dtype=torch.uint8, device=dev)
         self.has_append = w.n_new > 0
         if self.has_append:
@@ -58,6 +64,11 @@ class DeviceProblem:
                      batch=self.w.batch, n_new=self.w.n_new, stream=self.stream)
 
     def decode(self):
+        if self.sparse:
+            B.mla_decode_sparse(self.dims, self.q_nope, self.q_rope, self.W_uk, self.W_uv, self.cache,
+                                self.seq_lens, self.max_len, self.sel, self.n_sel, self.out, self.workspace,
+                                self.status, splits=self.splits, stream=self.stream)
+            return
         B.mla_decode(self.dims, self.q_nope, self.q_rope, self.W_uk, self.W_uv, self.cache,
                      self.seq_lens, self.max_len, self.out, self.workspace, self.status,
                      splits=self.splits, stream=self.stream)

@@ -23,6 +23,9 @@ What it computes, and where each step is stated:
   (Phase A, step A1; "Multi-head latent attention" on aicassindra,
   "End-to-end flow"); optionally the latent alone RMS-normalised first
   (Phase A, step A2; epsilon 1e-6, which the pages do not give).
+* Decode over a selected subset of each query's cached keys (the top-k
+  selection of "Multi-Head Latent Attention", section 4; the selector itself
+  is not part of this oracle).
 * An absorbed variant, used only to check the regrouping
   Q_nope . (W_K c) = (Q_nope W_K) . c ("Understanding MLA", section 4).
 
@@ -130,6 +133,40 @@ def decode_naive(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, n_q: int,
                     weights[(b, j, h)] = w
     if return_weights:
         return out, weights
+    return out
+
+
+def decode_sparse(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, sel, n_sel, n_q: int,
+                  scale: float, base: float = 10000.0, *, batches=None, heads=None):
+    """Decode restricted to a selected subset of each query's cached keys.
+
+    "Multi-Head Latent Attention", section 4: a selector picks a top-k subset
+    of the cached latents per query and MLA runs unchanged on that subset.
+    sel [B][n_q][max_sel] holds distinct cache slots (each <= the query's
+    position p), n_sel [B][n_q] how many leading entries are used.  Per head:
+    the same naive K = c W_K, V = c W_V, RoPE and softmax as decode_naive, over
+    the selected rows only, in the order given.
+    """
+    q_nope, q_rope = _f64(q_nope), _f64(q_rope)
+    W_uk, W_uv = _f64(W_uk), _f64(W_uv)
+    lens = [int(v) for v in np.asarray(lens).tolist()]
+    sel, n_sel = np.asarray(sel), np.asarray(n_sel)
+    B, _, H, _ = q_nope.shape
+    batches = range(B) if batches is None else batches
+    heads = range(H) if heads is None else heads
+    out = np.zeros((B, n_q, H, W_uv.shape[-1]), dtype=np.float64)
+    for b in batches:
+        L = lens[b]
+        for j in range(n_q):
+            p = L - n_q + j
+            rows = sel[b, j, : int(n_sel[b, j])]
+            c = _f64(c_kv[b, rows])                             # [k][d_c]
+            k_r = _f64(k_rope_rot[b, rows])                     # [k][d_R]
+            for h in heads:
+                q = np.concatenate([q_nope[b, j, h], rope(q_rope[b, j, h], p, base)])
+                K = np.concatenate([c @ W_uk[h], k_r], axis=1)
+                w = softmax((K @ q) * scale)
+                out[b, j, h] = w @ (c @ W_uv[h])
     return out
 
 

@@ -27,6 +27,11 @@ def rel_err(got, ref) -> float:
 
 
 def oracle_out(w, host, batches=None, heads=None):
+    if "sel" in host:                       # decode over the selected keys
+        k_rot = O.rope_cache(host["k_rope"], host["seq_lens"], w.rope_base)
+        return O.decode_sparse(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"], host["c_kv"], k_rot,
+                               host["seq_lens"], host["sel"].numpy(), host["n_sel"].numpy(), w.n_q,
+                               w.softmax_scale, w.rope_base, batches=batches, heads=heads)
     return O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base,
                          batches=batches, heads=heads)
 

@@ -310,6 +310,66 @@ def pin_rms_norm_does_not_commute_with_up_projection(O):
     assert np.max(np.abs(a - b)) > 1e-3
 
 
+def pin_sparse_decode(O):
+    """Decode over selected keys: selecting every visible key gives the dense
+    decode, the order of the selected keys does not matter, a single selected
+    key returns its value c_k W_V exactly, and explicit loops over a tiny
+    selection agree."""
+    n_q, lens = 2, (9, 13)
+    w, inp = _tiny_inputs(seed=41, lens=lens, n_q=n_q)
+    k_rot = O.rope_cache(inp["k_rope"], inp["seq_lens"])
+    args = (inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"], k_rot, inp["seq_lens"])
+    B, kmax = len(lens), max(lens)
+    sel = np.zeros((B, n_q, kmax), dtype=np.int64)
+    n_sel = np.zeros((B, n_q), dtype=np.int64)
+    for b, L in enumerate(lens):
+        for j in range(n_q):
+            p = L - n_q + j
+            sel[b, j, : p + 1] = np.arange(p + 1)
+            n_sel[b, j] = p + 1
+    dense = O.decode_naive(*args, n_q, w.softmax_scale)
+    _close(O.decode_sparse(*args, sel, n_sel, n_q, w.softmax_scale), dense, rtol=1e-12)
+    rng = np.random.default_rng(42)
+    shuffled = sel.copy()
+    for b in range(B):
+        for j in range(n_q):
+            shuffled[b, j, : n_sel[b, j]] = rng.permutation(sel[b, j, : n_sel[b, j]])
+    _close(O.decode_sparse(*args, shuffled, n_sel, n_q, w.softmax_scale), dense, rtol=1e-12)
+    one = np.zeros_like(sel)
+    one[:, :, 0] = 2
+    got = O.decode_sparse(*args, one, np.ones_like(n_sel), n_q, w.softmax_scale)
+    c, W_uv = np.asarray(inp["c_kv"], np.float64), np.asarray(inp["W_uv"], np.float64)
+    for b in range(B):
+        for h in range(w.heads):
+            assert np.array_equal(got[b, :, h], np.stack([c[b, 2] @ W_uv[h]] * n_q))
+    # explicit loops: sequence 1, query 1 (position 12), keys {12, 3, 7}
+    sub = np.zeros_like(sel)
+    sub[1, 1, :3] = [12, 3, 7]
+    ns = np.zeros_like(n_sel)
+    ns[:, :] = 1
+    ns[1, 1] = 3
+    got = O.decode_sparse(*args, sub, ns, n_q, w.softmax_scale)
+    W_uk = np.asarray(inp["W_uk"], np.float64)
+    qn, qr = np.asarray(inp["q_nope"], np.float64), np.asarray(inp["q_rope"], np.float64)
+    for h in range(w.heads):
+        qrot = [0.0] * w.d_rope
+        for i in range(w.d_rope // 2):
+            ang = 12 * 10000.0 ** (-2 * i / w.d_rope)
+            a, bb = qr[1, 1, h, 2 * i], qr[1, 1, h, 2 * i + 1]
+            qrot[2 * i], qrot[2 * i + 1] = a * math.cos(ang) - bb * math.sin(ang), a * math.sin(ang) + bb * math.cos(ang)
+        scores = []
+        for n in (12, 3, 7):
+            kn = [sum(c[1, n, i] * W_uk[h][i][t] for i in range(w.d_c)) for t in range(w.qk_nope)]
+            s_ = sum(qn[1, 1, h, t] * kn[t] for t in range(w.qk_nope)) + sum(qrot[t] * k_rot[1, n, t] for t in range(w.d_rope))
+            scores.append(s_ * w.softmax_scale)
+        mx = max(scores)
+        e = [math.exp(v - mx) for v in scores]
+        wts = [v / sum(e) for v in e]
+        ref = [sum(wts[k] * sum(c[1, n, i] * W_uv[h][i][v] for i in range(w.d_c)) for k, n in enumerate((12, 3, 7)))
+               for v in range(w.v_dim)]
+        _close(got[1, 1, h], ref, rtol=1e-11)
+
+
 def pin_cache_arithmetic(O):
     """Per-token storage figures printed on the pages."""
     g = json.load(open(os.path.join(GOLDEN, "cache_arithmetic.json")))

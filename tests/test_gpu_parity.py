@@ -1,4 +1,5 @@
-"""CUDA path against the fp64 oracle on the five workloads (same seeded
+"""CUDA path against the fp64 oracle on the five workloads and the top-k
+sparse workload (same seeded
 inputs; full outputs where the oracle is quick, sampled (batch, head)
 outputs at full size, in the launch configuration the benchmark times)."""
 import os
@@ -22,6 +23,7 @@ CASES = [
     ("v3_b64_ragged", [0, 9, 17, 33, 48, 63], [0, 5, 77, 127]),
     ("v3_b4_ctx131072", [0, 3], [0, 64, 127]),
     ("v3_b32_append2", [0, 13, 31], [0, 33, 100]),
+    ("v3_b32_topk2048", [0, 17, 31], [0, 64, 127]),
 ]
 
 

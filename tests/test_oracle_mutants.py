@@ -42,6 +42,11 @@ MUTANTS = [
     ("rms norm applied to the rope key too", "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)",
      "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)\n        rows[:, d_c:] = y[:, d_c:] / np.sqrt(np.mean(y[:, d_c:] ** 2, axis=-1, keepdims=True) + eps)\n        y = rows"),
     ("rms norm without gamma", "return _f64(gamma) * c / rms", "return c / rms"),
+    ("sparse selection ignores the count", "rows = sel[b, j, : int(n_sel[b, j])]", "rows = sel[b, j]"),
+    ("sparse rows taken one slot late", "c = _f64(c_kv[b, rows])                             # [k][d_c]",
+     "c = _f64(c_kv[b, rows + 1])                         # [k][d_c]"),
+    ("sparse query rotated at the wrong position", "q = np.concatenate([q_nope[b, j, h], rope(q_rope[b, j, h], p, base)])",
+     "q = np.concatenate([q_nope[b, j, h], rope(q_rope[b, j, h], p + 1, base)])"),
     ("rms epsilon outside the square root", "np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + eps)",
      "np.sqrt(np.mean(c * c, axis=-1, keepdims=True)) + eps"),
 ]
