@@ -134,3 +134,24 @@ def test_status_strings():
         assert B.mla_status_string(code) == name
     assert B.mla_status_string(99) == "MLA_ERR_UNKNOWN"
     assert B.lib().mla_get_status(None, None, None) == B.CODES["MLA_ERR_ARG"]
+
+
+def test_sparse_decode_argument_checks():
+    """mla_decode_sparse reports argument errors before anything is launched."""
+    L = B.lib()
+
+    def sparse(dims, max_sel=16, max_len=100, sel=FAKE, n_sel=FAKE, ws_bytes=None, capacity=100):
+        d = ctypes.byref(dims)
+        if ws_bytes is None:
+            ws_bytes = L.mla_decode_workspace_bytes(d, 2, 1, max(1, min(max_sel, max_len)), 0)
+        return L.mla_decode_sparse(d, 2, 1, FAKE, FAKE, FAKE, FAKE, FAKE, capacity, FAKE, max_len, sel, n_sel,
+                                   max_sel, FAKE, FAKE, ws_bytes, 0, FAKE, None)
+
+    assert sparse(v3(), sel=None) == B.CODES["MLA_ERR_ARG"]
+    assert sparse(v3(), n_sel=None) == B.CODES["MLA_ERR_ARG"]
+    assert sparse(v3(), max_sel=0) == B.CODES["MLA_ERR_ARG"]
+    assert sparse(v3(), max_sel=101) == B.CODES["MLA_ERR_ARG"]            # > max_len
+    assert sparse(v3(), ws_bytes=0) == B.CODES["MLA_ERR_WORKSPACE"]
+    assert sparse(v3(dtype="fp32")) == B.CODES["MLA_ERR_UNSUPPORTED"]     # tensor-core path only
+    assert sparse(v3(), capacity=1 << 30, max_len=100) == B.CODES["MLA_ERR_UNSUPPORTED"]   # batch*capacity > 2^31
+    assert B.CODES["MLA_ERR_INDEX"] == 9 and B.STATUS[9] == "MLA_ERR_INDEX"
