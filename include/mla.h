@@ -194,6 +194,16 @@ MLA_API int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q,
                void* out, void* workspace, size_t workspace_bytes, int32_t splits,
                int32_t* status, void* stream);
 
+/* Failure-path self-test.  Every kernel of the library waits on its
+ * barriers through one bounded wait that gives up after a time limit,
+ * records MLA_ERR_TIMEOUT in the status word and lets the kernel leave
+ * normally (no trap, no fault).  This call runs that wait in one CTA on a
+ * barrier that nothing ever arrives on, with the limit limit_ns (0 < limit_ns
+ * <= 10 s): afterwards the status word holds MLA_ERR_TIMEOUT and the context
+ * remains usable.  It has no counterpart on the pages; it exists for tests.
+ *   status  (device) int32 status word. */
+MLA_API int mla_selftest_wait_timeout(int32_t* status, int64_t limit_ns, void* stream);
+
 /* Size of the fixed scratch area behind mla_decode_noalloc. */
 #define MLA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

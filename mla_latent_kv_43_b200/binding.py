@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.restype = ctypes.c_int
         L.mla_decode_sparse.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, I32, P, P, SZ, I32, P, P]
         L.mla_decode_sparse.restype = ctypes.c_int
+        L.mla_selftest_wait_timeout.argtypes = [P, I64, P]
+        L.mla_selftest_wait_timeout.restype = ctypes.c_int
         L.mla_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.mla_get_status.restype = ctypes.c_int
         L.mla_status_string.argtypes = [ctypes.c_int]
@@ -164,6 +166,11 @@ def mla_decode_sparse(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor,
                                    _ptr(sel), _ptr(n_sel), sel.shape[-1], _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), splits, _ptr(status),
                                    _stream(stream)), "mla_decode_sparse")
+
+
+def mla_selftest_wait_timeout(status: torch.Tensor, limit_ns: int, stream=None):
+    """Run the library's bounded wait on a barrier nothing arrives on."""
+    _check(lib().mla_selftest_wait_timeout(_ptr(status), limit_ns, _stream(stream)), "mla_selftest_wait_timeout")
 
 
 def mla_decode_noalloc(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor,

@@ -120,14 +120,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 // Wait for the phase with parity `parity` to complete.  Returns false when
 // the time limit passed or *abort became non-zero.
 template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (abort && *abort) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) return false;
+            if (globaltimer() - t0 > limit_ns) return false;
         }
     }
 }
