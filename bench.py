@@ -48,6 +48,7 @@ FLUSH_BYTES = 512 << 20
 KERNEL_SOURCES = {  # kernel name prefix -> source file whose hash keys committed ncu traffic
     "sm100_attend": "mla_latent_kv_43_b200/csrc/sm100_attend.cu",
     "generic_attend": "mla_latent_kv_43_b200/csrc/generic.cu",
+    "sm100_oproj": "mla_latent_kv_43_b200/csrc/sm100_append.cu",
 }
 
 
@@ -172,10 +173,19 @@ def oracle_decode(O, w, host, batches, heads=None, k_rot=None):
     visible key, or over the selected keys of a top-k workload (whose cache,
     rotated once outside the timing, is ``k_rot``)."""
     if w.top_k:
-        return O.decode_sparse(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"], host["c_kv"], k_rot,
-                               host["seq_lens"], host["sel"].numpy(), host["n_sel"].numpy(), w.n_q,
-                               w.softmax_scale, w.rope_base, batches=batches, heads=heads)
-    return O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=batches, heads=heads)
+        out = O.decode_sparse(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"], host["c_kv"], k_rot,
+                              host["seq_lens"], host["sel"].numpy(), host["n_sel"].numpy(), w.n_q,
+                              w.softmax_scale, w.rope_base, batches=batches, heads=heads)
+    else:
+        out = O.decode_step(host, w.n_q, w.d_c, w.softmax_scale, w.rope_base, batches=batches, heads=heads)
+    if w.hidden_out:
+        # project the chosen sequences' outputs of the chosen heads (the other
+        # heads' outputs are zero there): their share of y = out W_O
+        bs = list(range(w.batch)) if batches is None else list(batches)
+        hs = list(range(w.heads)) if heads is None else list(heads)
+        W = host["W_O"].reshape(w.heads, w.v_dim, w.hidden_out)[hs].reshape(len(hs) * w.v_dim, w.hidden_out)
+        out = O.output_projection(out[bs][:, :, hs].reshape(len(bs) * w.n_q, len(hs), w.v_dim), W)
+    return out
 
 
 def cpu_sample(w, host, budget_s: float):
@@ -234,6 +244,7 @@ def workload_config(w, host, world):
             "n_q": w.n_q, "heads": w.heads, "d_c": w.d_c, "d_rope": w.d_rope, "qk_nope": w.qk_nope,
             "v_dim": w.v_dim, "seq_len_mean": sum(lens) / len(lens), "seq_len_min": min(lens),
             "seq_len_max": max(lens), "capacity": w.capacity, "n_new": w.n_new, "hidden": w.hidden,
+            "top_k": w.top_k, "hidden_out": w.hidden_out,
             "l2": "flushed before every timed step (512 MiB write, outside the timed events)",
             "parallelism": f"dp{world} (independent sequence shards)"}
 
@@ -297,7 +308,7 @@ def run_ours(a, rank, world, local):
     h_qn = host["q_nope"].pin_memory()
     h_qr = host["q_rope"].pin_memory()
     h_len = host["seq_lens"].pin_memory()
-    h_out = torch.empty(prob.out.shape, dtype=prob.out.dtype).pin_memory()
+    h_out = torch.empty(prob.result.shape, dtype=prob.result.dtype).pin_memory()
     h2d = h_qn.numel() * h_qn.element_size() + h_qr.numel() * h_qr.element_size() + h_len.numel() * 4
     if prob.has_append:
         h_x = host["x"].pin_memory()
@@ -322,7 +333,7 @@ def run_ours(a, rank, world, local):
             prob.sel.copy_(h_sel, non_blocking=True)
             prob.n_sel.copy_(h_nsel, non_blocking=True)
         prob.step()
-        h_out.copy_(prob.out, non_blocking=True)
+        h_out.copy_(prob.result, non_blocking=True)
         e.record(stream)
         e.synchronize()
         e2e_ms += s.elapsed_time(e)
@@ -354,8 +365,11 @@ def run_ours(a, rank, world, local):
             "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(kname),
             "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": avg_s * 1e6,
             "peak_source": peaks["source"]}
-    kernels = {n: {"launches": c, "avg_us": t / c * 1e3, "share": t / sum(v[1] for v in prof.values())}
-               for n, (c, t) in sorted(prof.items())}
+    kernels = {}
+    for n, (c, t) in sorted(prof.items()):
+        kb = RF.kernel_bytes(n, w_rank, lens, q_el, q_el)
+        kernels[n] = {"launches": c, "avg_us": t / c * 1e3, "share": t / sum(v[1] for v in prof.values()),
+                      "hbm_frac": (kb / (t / c * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kb else None}
     t_hbm = work["bytes"] / (peaks["hbm_gbs"] * 1e9)
     t_tc = work["flops"] / (peaks["bf16_tflops"] * 1e12)
     line = {

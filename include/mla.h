@@ -194,6 +194,24 @@ MLA_API int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q,
                void* out, void* workspace, size_t workspace_bytes, int32_t splits,
                int32_t* status, void* stream);
 
+/* The output projection ("Understanding MLA", Phase D step D2): the per-head
+ * outputs of a decode step, concatenated head after head, projected to the
+ * hidden width: y[t] = [out[t][0] || out[t][1] || ... || out[t][H-1]] W_O.
+ *   tokens  number of query tokens (batch * n_q of the decode).
+ *   hidden  output width; a multiple of 8 for the tensor-core path.
+ *   out     (device) [tokens][heads][v_dim] (mla_decode's output), dims->dtype.
+ *   W_O     (device) [heads * v_dim][hidden], dims->dtype.
+ *   y       (device) [tokens][hidden], dims->dtype; float accumulation, one rounding.
+ *   status  (device) int32 status word.
+ * bf16 runs a tcgen05 GEMM with K split over clusters of eight CTAs; fp32
+ * (or a width that is not a multiple of 8) runs on CUDA cores.
+ * Errors: MLA_ERR_ARG (tokens < 0, hidden <= 0, a null pointer when tokens > 0),
+ * MLA_ERR_ALIGN (a bf16 tensor-core operand not 16-byte aligned),
+ * MLA_ERR_UNSUPPORTED (more than 65535 * 256 tokens on the tensor-core path);
+ * tokens == 0 returns MLA_OK and touches nothing. */
+MLA_API int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t hidden, const void* out,
+               const void* W_O, void* y, int32_t* status, void* stream);
+
 /* Failure-path self-test.  Every kernel of the library waits on its
  * barriers through one bounded wait that gives up after a time limit,
  * records MLA_ERR_TIMEOUT in the status word and lets the kernel leave

@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.restype = ctypes.c_int
         L.mla_decode_sparse.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, I32, P, P, SZ, I32, P, P]
         L.mla_decode_sparse.restype = ctypes.c_int
+        L.mla_output_projection.argtypes = [D, I32, I32, P, P, P, P, P]
+        L.mla_output_projection.restype = ctypes.c_int
         L.mla_selftest_wait_timeout.argtypes = [P, I64, P]
         L.mla_selftest_wait_timeout.restype = ctypes.c_int
         L.mla_get_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
@@ -166,6 +168,14 @@ def mla_decode_sparse(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor,
                                    _ptr(sel), _ptr(n_sel), sel.shape[-1], _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), splits, _ptr(status),
                                    _stream(stream)), "mla_decode_sparse")
+
+
+def mla_output_projection(dims: MlaDims, out: torch.Tensor, W_O: torch.Tensor, y: torch.Tensor,
+                          status: torch.Tensor, stream=None):
+    """y [tokens][hidden] = heads of out [..][H][v_dim] concatenated, times W_O."""
+    tokens = out.numel() // (dims.heads * dims.v_dim)
+    _check(lib().mla_output_projection(ctypes.byref(dims), tokens, y.shape[-1], _ptr(out), _ptr(W_O), _ptr(y),
+                                       _ptr(status), _stream(stream)), "mla_output_projection")
 
 
 def mla_selftest_wait_timeout(status: torch.Tensor, limit_ns: int, stream=None):

@@ -355,6 +355,39 @@ __global__ void rms_rows_kernel(int d_c, int D, int n_new, const int32_t* __rest
 
 }  // namespace
 
+namespace {
+
+// y[t][n] = sum_k x[t][k] W[k][n]: one thread per output element, float
+// accumulation (the CUDA-core output projection).
+template <typename T>
+__global__ void gemm_xw_kernel(const T* __restrict__ x, const T* __restrict__ W, int M, int K, int n_out,
+                               T* __restrict__ y) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= n_out) return;
+    for (int t = blockIdx.y; t < M; t += gridDim.y) {
+        float acc = 0.f;
+        for (int k = 0; k < K; ++k)
+            acc = fmaf(to_f32(x[(int64_t)t * K + k]), to_f32(W[(int64_t)k * n_out + n]), acc);
+        y[(int64_t)t * n_out + n] = from_f32<T>(acc);
+    }
+}
+
+}  // namespace
+
+int generic_gemm_xw(mla_dtype dtype, const void* x, const void* W, int M, int K, int n_out, void* y,
+                    cudaStream_t stream, int* launches) {
+    const dim3 grid((n_out + 127) / 128, M < 65535 ? M : 65535);
+    prof_begin(stream, "generic_oproj");
+    if (dtype == MLA_FP32)
+        gemm_xw_kernel<float><<<grid, 128, 0, stream>>>((const float*)x, (const float*)W, M, K, n_out, (float*)y);
+    else
+        gemm_xw_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)W, M,
+                                                                K, n_out, (__nv_bfloat16*)y);
+    prof_end(stream);
+    if (launches) ++*launches;
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int rms_norm_rows(const AppendCall& c, int* launches) {
     const int M = c.batch * c.n_new, D = c.d.d_c + c.d.d_rope;
     if (M == 0) return MLA_OK;

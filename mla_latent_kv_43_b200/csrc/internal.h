@@ -1,5 +1,6 @@
 // Internal interface between the C ABI (mla_api.cu) and the kernel files.
 #pragma once
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -55,6 +56,13 @@ int generic_append(const AppendCall& c, int* launches);
 int sm100_append(const AppendCall& c, int* launches);
 int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
               const int32_t* positions, cudaStream_t stream);
+// The output projection y = x W (x [M][K], W [K][n_out]): tcgen05 (bf16) and CUDA-core versions.
+namespace sm100 {
+int gemm_xw_launch(const void* x, const void* W, int M, int K, int n_out, __nv_bfloat16* y, int32_t* status,
+                   cudaStream_t stream, const char* name, int* launches);
+}
+int generic_gemm_xw(mla_dtype dtype, const void* x, const void* W, int M, int K, int n_out, void* y,
+                    cudaStream_t stream, int* launches);
 // RMSNorm of the latent of every appended row (after either append kernel).
 int rms_norm_rows(const AppendCall& c, int* launches);
 

@@ -164,6 +164,27 @@ int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q, const vo
     return rc;
 }
 
+int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t hidden, const void* out, const void* W_O,
+                          void* y, int32_t* status, void* stream) {
+    g_last_launches = 0;
+    int rc = validate_dims(dims);
+    if (rc) return rc;
+    if (tokens < 0 || hidden <= 0) return MLA_ERR_ARG;
+    if (tokens == 0) return MLA_OK;
+    if (!out || !W_O || !y || !status) return MLA_ERR_ARG;
+    const int K = dims->heads * dims->v_dim;
+    int launches = 0;
+    if (dims->dtype == MLA_BF16 && hidden % 8 == 0 && K % 8 == 0) {
+        if (!aligned16(out) || !aligned16(W_O) || !aligned16(y)) return MLA_ERR_ALIGN;
+        rc = mla::sm100::gemm_xw_launch(out, W_O, tokens, K, hidden, (__nv_bfloat16*)y, status, (cudaStream_t)stream,
+                                        "sm100_oproj", &launches);
+    } else {
+        rc = mla::generic_gemm_xw((mla_dtype)dims->dtype, out, W_O, tokens, K, hidden, y, (cudaStream_t)stream, &launches);
+    }
+    g_last_launches = launches;
+    return rc;
+}
+
 int mla_get_status(int32_t* status, void* stream, int32_t* host_status) {
     if (!status || !host_status) return MLA_ERR_ARG;
     cudaStream_t s = (cudaStream_t)stream;

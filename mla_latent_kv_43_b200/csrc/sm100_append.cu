@@ -1,4 +1,4 @@
-// Cache append on tcgen05 tensor cores.
+// Cache append (and the output projection's plain product) on tcgen05 tensor cores.
 //
 // For the new tokens m (x [M][hidden], M = batch * n_new) at their slots
 // pos_m ("Understanding MLA (Multi-head Latent Attention)", Phase A step A1
@@ -17,6 +17,12 @@
 // barrier CTA r sums feature rows [16r, 16r + 16) of the tile over the eight
 // partials through distributed shared memory, rotates the rope pairs and
 // stores bf16 cache entries.
+//
+// The output projection ("Understanding MLA", Phase D step D2: the heads'
+// outputs flattened and projected to the hidden width) is the same product
+// y = x W with x = the decode output [tokens][heads * v_dim] and W = W_O
+// [heads * v_dim][hidden]; the same kernel stores y rows instead of cache
+// entries.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -38,6 +44,8 @@ constexpr int kFeatures = 576;
 
 struct AppendArgs {
     int M, n_new, kblocks, N;            // tokens, tokens per sequence, k blocks of 64, token tile
+    int n_out;                           // output width: 576 for the append, the hidden width for W_O
+    __nv_bfloat16* y;                    // plain product [M][n_out] (the output projection)
     const int32_t* positions;
     __nv_bfloat16* cache;
     int64_t capacity;
@@ -49,6 +57,9 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
     return n <= 32 ? 32u : (n <= 64 ? 64u : (n <= 128 ? 128u : 256u));
 }
 
+// kAppend: rotate the rope features and store cache entries at the tokens'
+// slots; otherwise store the plain product y = x W (the output projection).
+template <bool kAppend>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads, 1)
 append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapX, AppendArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -169,11 +180,15 @@ append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ 
             v0[0] += u0.x; v0[1] += u0.y; v0[2] += u0.z; v0[3] += u0.w;
             v1[0] += u1.x; v1[1] += u1.y; v1[2] += u1.z; v1[3] += u1.w;
         }
-        if (n >= kFeatures) continue;                  // zero fill past the 576 features
+        if (n >= a.n_out) continue;                    // zero fill past the last feature
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int m = nt * N + m4 + i;
             if (m >= a.M) break;
+            if constexpr (!kAppend) {
+                *reinterpret_cast<uint32_t*>(a.y + (int64_t)m * a.n_out + n) = pack_bf16(v0[i], v1[i]);
+                continue;
+            }
             const int64_t pos = a.positions[m];
             if (pos < 0 || pos >= a.capacity) {
                 set_status(a.status, MLA_ERR_POS);
@@ -208,6 +223,7 @@ int append_launch(const AppendCall& c, int* launches) {
     }
     AppendArgs a{};
     a.M = M;
+    a.n_out = kFeatures;
     a.n_new = c.n_new;
     a.kblocks = (c.hidden + 63) / 64;
     a.N = N;
@@ -219,12 +235,53 @@ int append_launch(const AppendCall& c, int* launches) {
     const int stage_bytes = 2 * kBoxA + N * 128;
     const int part_bytes = 128 * (N * 4 + 16);
     const size_t smem = (size_t)(kStages * stage_bytes > part_bytes ? kStages * stage_bytes : part_bytes) + 1024;
-    if (cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(append_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid((kFeatures + 127) / 128 * kSplit, (M + N - 1) / N);
     prof_begin(c.stream, "sm100_append");
-    const cudaError_t e = launch_plain(append_kernel, grid, dim3(kThreads), smem, c.stream, mw, mx, a);
+    const cudaError_t e = launch_plain(append_kernel<true>, grid, dim3(kThreads), smem, c.stream, mw, mx, a);
     prof_end(c.stream);
+    if (launches) ++*launches;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// y [M][n_out] = x [M][K] W [K][n_out], bf16 in and out, fp32 accumulation:
+// the same split-K cluster kernel without the cache epilogue.
+int gemm_xw_launch(const void* x, const void* W, int M, int K, int n_out, __nv_bfloat16* y, int32_t* status,
+                   cudaStream_t stream, const char* name, int* launches) {
+    int N = (M + 15) / 16 * 16;
+    if (N > kMaxN) N = kMaxN;
+    if ((M + N - 1) / N > 65535) return MLA_ERR_UNSUPPORTED;    // token tiles on grid.y
+    CUtensorMap mw, mx;
+    {
+        const uint64_t dims[2] = {(uint64_t)n_out, (uint64_t)K}, str[1] = {(uint64_t)n_out * 2};
+        const uint32_t box[2] = {64, 64};
+        if (!make_map(&mw, W, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M}, str[1] = {(uint64_t)K * 2};
+        const uint32_t box[2] = {64, (uint32_t)N};
+        if (!make_map(&mx, x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    AppendArgs a{};
+    a.M = M;
+    a.n_out = n_out;
+    a.y = y;
+    a.n_new = 1;
+    a.kblocks = (K + 63) / 64;
+    a.N = N;
+    a.status = status;
+    const int stage_bytes = 2 * kBoxA + N * 128;
+    const int part_bytes = 128 * (N * 4 + 16);
+    const size_t smem = (size_t)(kStages * stage_bytes > part_bytes ? kStages * stage_bytes : part_bytes) + 1024;
+    if (cudaFuncSetAttribute(append_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid((n_out + 127) / 128 * kSplit, (M + N - 1) / N);
+    prof_begin(stream, name);
+    const cudaError_t e = launch_plain(append_kernel<false>, grid, dim3(kThreads), smem, stream, mw, mx, a);
+    prof_end(stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
 }

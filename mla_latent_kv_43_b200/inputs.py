@@ -54,6 +54,7 @@ class Workload:
     hidden: int = 0
     n_new: int = 0
     top_k: int = 0                  # > 0: each query attends a selected subset of its keys
+    hidden_out: int = 0             # > 0: the step ends with the output projection to this width
     rope_base: float = 10000.0
     seed: int = 0
 
@@ -103,6 +104,13 @@ WORKLOADS: Dict[str, Workload] = {
     "v3_b32_topk2048": Workload(
         name="v3_b32_topk2048", dtype="bf16", batch=32, n_q=1, lens=(8192,) * 32,
         capacity=8192, latent_rms_norm=True, top_k=2048, seed=5, **V3),
+    # the batched decode followed by the output projection W_O to the model
+    # width 7168 ("Understanding MLA", Phase D step D2); same draws as
+    # v3_b64_ragged plus W_O
+    "v3_b64_ragged_oproj": Workload(
+        name="v3_b64_ragged_oproj", dtype="bf16", batch=64, n_q=1, lens=None,
+        lens_range=(1024, 4096), capacity=4096, latent_rms_norm=True, seed=2,
+        hidden_out=7168, **V3),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
@@ -136,7 +144,8 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
     n_new > 0 also x [B*n_new][hidden], W_dkv [hidden][d_c+d_rope],
     positions int32 [B*n_new] and old_lens int32 [B]; with top_k > 0 also
     sel int32 [B][n_q][top_k] (distinct visible slots, unused tail entries 0)
-    and n_sel int32 [B][n_q] = min(top_k, p + 1).
+    and n_sel int32 [B][n_q] = min(top_k, p + 1); with hidden_out > 0 also
+    W_O [H*v_dim][hidden_out] (drawn last, so the other draws do not change).
     """
     rng = np.random.default_rng(w.seed)
     if w.lens is None:
@@ -179,12 +188,15 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
                 n_sel[b, j] = n
         out["sel"] = torch.from_numpy(sel)
         out["n_sel"] = torch.from_numpy(n_sel)
+    if w.hidden_out:
+        K = w.heads * w.v_dim
+        out["W_O"] = _cast(_normal(rng, (K, w.hidden_out), 1.0 / math.sqrt(K)), dt)
     return out
 
 
 def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6,
          v_dim=5, n_q=1, lens=(5, 9), capacity=None, seed=0, latent_rms_norm=False,
-         hidden=0, n_new=0, top_k=0) -> Workload:
+         hidden=0, n_new=0, top_k=0, hidden_out=0) -> Workload:
     """A small custom workload for pins and edge cases (batch = len(lens))."""
     cap = capacity if capacity is not None else max(lens)
     if batch is None:
@@ -192,4 +204,4 @@ def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6
     return Workload(name="custom", dtype=dtype, batch=batch, heads=heads, d_c=d_c,
                     d_rope=d_rope, qk_nope=qk_nope, v_dim=v_dim, n_q=n_q,
                     lens=tuple(lens), capacity=cap, latent_rms_norm=latent_rms_norm,
-                    hidden=hidden, n_new=n_new, top_k=top_k, seed=seed)
+                    hidden=hidden, n_new=n_new, top_k=top_k, hidden_out=hidden_out, seed=seed)

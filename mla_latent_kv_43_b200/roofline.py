@@ -12,7 +12,9 @@ results are implementation traffic and are not counted.  FLOPs are 2 per
 multiply-add of the absorbed form: per visible key and query token,
 H * (d_c + d_rope) for the score and H * d_c for the weighted latent sum;
 per query token, H * qk_nope * d_c for the absorption and H * d_c * v_dim
-for the value up-projection; 2 * hidden * (d_c + d_rope) per appended token.
+for the value up-projection; 2 * hidden * (d_c + d_rope) per appended token;
+2 * H * v_dim * hidden_out per query token for the output projection, which
+reads W_O once and the head outputs once more and writes y.
 """
 from __future__ import annotations
 
@@ -65,8 +67,15 @@ def step_work(w, lens: Sequence[int]) -> Dict[str, float]:
         m = B * w.n_new
         r["append_bytes"] = (w.hidden * D + m * w.hidden + m * D) * es
         r["append_flops"] = 2 * m * w.hidden * D
-    r["bytes"] = r["cache_bytes"] + r["weight_bytes"] + r["q_bytes"] + r["out_bytes"] + r["append_bytes"]
-    r["flops"] = r["core_flops"] + r["proj_flops"] + r["append_flops"]
+    r["oproj_bytes"] = 0
+    r["oproj_flops"] = 0
+    if w.hidden_out:
+        K = H * w.v_dim
+        r["oproj_bytes"] = (K * w.hidden_out + qt * K + qt * w.hidden_out) * es
+        r["oproj_flops"] = 2 * qt * K * w.hidden_out
+    r["bytes"] = (r["cache_bytes"] + r["weight_bytes"] + r["q_bytes"] + r["out_bytes"] + r["append_bytes"]
+                  + r["oproj_bytes"])
+    r["flops"] = r["core_flops"] + r["proj_flops"] + r["append_flops"] + r["oproj_flops"]
     r["query_tokens"] = qt
     return r
 
@@ -94,4 +103,7 @@ def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_ele
     if "append" in kernel:
         m = w.batch * w.n_new
         return (w.hidden * D + m * w.hidden + m * D) * es
+    if "oproj" in kernel:
+        K = H * w.v_dim
+        return (K * w.hidden_out + qt * K + qt * w.hidden_out) * es
     return 0.0

@@ -6,7 +6,8 @@ keys rotated at their slot positions by ``mla_rope`` (what the append step
 would have stored), the weights, per-sequence lengths, and caller-owned
 output, workspace and status buffers.  ``step()`` runs one decode step
 (append of the new tokens when the workload has them, then attention: over
-every visible key, or over the selected ones for a top-k workload).
+every visible key, or over the selected ones for a top-k workload), then,
+when the workload has a W_O, the output projection into ``y``.
 """
 from __future__ import annotations
 
@@ -52,6 +53,10 @@ class DeviceProblem:
         ws_len = w.top_k if self.sparse else self.max_len    # the tile bound of the plan
         self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, ws_len, splits)
         self.workspace = torch.empty(max(self.layout["total"], 256), dtype=torch.uint8, device=dev)
+        self.has_oproj = w.hidden_out > 0
+        if self.has_oproj:
+            self.W_O = to(host["W_O"])
+            self.y = torch.empty(w.batch * w.n_q, w.hidden_out, dtype=w.torch_dtype, device=dev)
         self.has_append = w.n_new > 0
         if self.has_append:
             self.x = to(host["x"])
@@ -73,6 +78,9 @@ class DeviceProblem:
                      self.seq_lens, self.max_len, self.out, self.workspace, self.status,
                      splits=self.splits, stream=self.stream)
 
+    def project(self):
+        B.mla_output_projection(self.dims, self.out, self.W_O, self.y, self.status, stream=self.stream)
+
     def step(self) -> int:
         """One decode step; returns the number of kernels it enqueued."""
         n = 0
@@ -80,7 +88,16 @@ class DeviceProblem:
             self.append()
             n += B.mla_last_launch_count()
         self.decode()
-        return n + B.mla_last_launch_count()
+        n += B.mla_last_launch_count()
+        if self.has_oproj:
+            self.project()
+            n += B.mla_last_launch_count()
+        return n
+
+    @property
+    def result(self) -> torch.Tensor:
+        """What the step hands back: y after the output projection, else the head outputs."""
+        return self.y if self.has_oproj else self.out
 
     def get_status(self) -> int:
         return B.mla_get_status(self.status, stream=self.stream)

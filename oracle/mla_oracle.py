@@ -17,7 +17,9 @@ What it computes, and where each step is stated:
 * Concatenation Q = [Q_nope || Q_rope], K = [K_nope || K_rope] and
   softmax(Q K^T / sqrt(qk_nope + d_R)) V (Phase D, steps D1-D2;
   "Multi-Head Latent Attention", section 3, the sketch's last two lines).
-  The output stops at the per-head value vector (no output projection).
+  decode_* stop at the per-head value vector; output_projection concatenates
+  the heads and projects to the hidden width ("Understanding MLA", Phase D
+  step D2).
 * The append step: one projection x W_DKV to d_c + d_R values, split into
   the latent and the rope key, rope key rotated at the token's position
   (Phase A, step A1; "Multi-head latent attention" on aicassindra,
@@ -218,6 +220,20 @@ def decode_absorbed(q_nope, q_rope, W_uk, W_uv, c_kv, k_rope_rot, lens, n_q: int
     if return_intermediates:
         return out, inter
     return out
+
+
+# ---------------------------------------------------------------------------
+# Output projection ("Understanding MLA", Phase D step D2)
+# ---------------------------------------------------------------------------
+def output_projection(out, W_O) -> np.ndarray:
+    """The per-head outputs concatenated head after head and projected to the
+    hidden width: y[t] = [out[t][0] || out[t][1] || ...] W_O.
+
+    out [T][H][v_dim], W_O [H * v_dim][hidden]; returns y [T][hidden].
+    """
+    out = _f64(out)
+    T, H, v = out.shape
+    return out.reshape(T, H * v) @ _f64(W_O)
 
 
 # ---------------------------------------------------------------------------

@@ -370,6 +370,33 @@ def pin_sparse_decode(O):
         _close(got[1, 1, h], ref, rtol=1e-11)
 
 
+def pin_output_projection(O):
+    """Heads concatenated head-major then projected: the same as summing each
+    head's block product, as torch's float64 linear map of the flattened
+    heads, and as the absorbed form sum_h o_lat[h] (W_V[h] W_O[h-block]) (the
+    value up-projection folded into the output projection, aicassindra
+    "Multi-head latent attention", "End-to-end flow")."""
+    rng = np.random.default_rng(51)
+    T, H, v, hidden = 3, 4, 5, 7
+    out = rng.standard_normal((T, H, v))
+    W_O = rng.standard_normal((H * v, hidden))
+    y = O.output_projection(out, W_O)
+    _close(y, sum(out[:, h] @ W_O[h * v:(h + 1) * v] for h in range(H)), rtol=1e-12)
+    ref = torch.nn.functional.linear(torch.from_numpy(out.reshape(T, H * v)), torch.from_numpy(W_O.T.copy()))
+    _close(y, ref.numpy(), rtol=1e-12)
+    # absorbed: through the decode's latent outputs
+    w, inp = _tiny_inputs(seed=52, lens=(6, 9), v_dim=v, heads=H)
+    k_rot = O.rope_cache(inp["k_rope"], inp["seq_lens"])
+    W_O = rng.standard_normal((H * v, hidden))
+    outs, inter = O.decode_absorbed(inp["q_nope"], inp["q_rope"], inp["W_uk"], inp["W_uv"], inp["c_kv"], k_rot,
+                                    inp["seq_lens"], 1, w.softmax_scale, return_intermediates=True)
+    W_uv = np.asarray(inp["W_uv"], np.float64)
+    for b in range(2):
+        y_b = O.output_projection(outs[b], W_O)[0]
+        folded = sum(inter[(b, 0, h)][1] @ (W_uv[h] @ W_O[h * v:(h + 1) * v]) for h in range(H))
+        _close(y_b, folded, rtol=1e-11)
+
+
 def pin_cache_arithmetic(O):
     """Per-token storage figures printed on the pages."""
     g = json.load(open(os.path.join(GOLDEN, "cache_arithmetic.json")))

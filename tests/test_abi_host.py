@@ -155,3 +155,17 @@ def test_sparse_decode_argument_checks():
     assert sparse(v3(dtype="fp32")) == B.CODES["MLA_ERR_UNSUPPORTED"]     # tensor-core path only
     assert sparse(v3(), capacity=1 << 30, max_len=100) == B.CODES["MLA_ERR_UNSUPPORTED"]   # batch*capacity > 2^31
     assert B.CODES["MLA_ERR_INDEX"] == 9 and B.STATUS[9] == "MLA_ERR_INDEX"
+
+
+def test_output_projection_argument_checks():
+    """mla_output_projection rejects bad sizes and pointers before any launch;
+    zero tokens is a no-op that touches nothing."""
+    L = B.lib()
+    d = ctypes.byref(v3())
+    P = FAKE
+    assert L.mla_output_projection(d, -1, 7168, P, P, P, P, None) == B.CODES["MLA_ERR_ARG"]
+    assert L.mla_output_projection(d, 4, 0, P, P, P, P, None) == B.CODES["MLA_ERR_ARG"]
+    assert L.mla_output_projection(d, 0, 7168, None, None, None, None, None) == B.CODES["MLA_OK"]
+    assert L.mla_output_projection(d, 4, 7168, None, P, P, P, None) == B.CODES["MLA_ERR_ARG"]
+    assert L.mla_output_projection(d, 4, 7168, P, P, P, None, None) == B.CODES["MLA_ERR_ARG"]
+    assert L.mla_output_projection(d, 4, 7168, P + 2, P, P, P, None) == B.CODES["MLA_ERR_ALIGN"]

@@ -1,0 +1,53 @@
+"""Host logic of the bench and the input generator (no GPU).
+
+* W_O is drawn after every other input, so a workload with the output
+  projection has the same queries, cache and weights as the one without;
+* the reference arm's head sample projects a subset of the heads: the
+  projections of disjoint head subsets add up to the projection of all heads;
+* the roofline counts the output projection's bytes: W_O once, the head
+  outputs once, y once."""
+import os
+import sys
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from mla_latent_kv_43_b200 import inputs as gen  # noqa: E402
+from mla_latent_kv_43_b200 import roofline as RF  # noqa: E402
+from oracle import mla_oracle as O  # noqa: E402
+
+
+def test_w_o_draw_leaves_the_other_inputs_unchanged():
+    w = gen.tiny("fp32", lens=(9, 13), n_q=2, seed=3)
+    a, b = gen.generate(w), gen.generate(w.with_(hidden_out=11))
+    assert set(b) - set(a) == {"W_O"} and b["W_O"].shape == (w.heads * w.v_dim, 11)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_head_subset_projections_add_up():
+    w = gen.tiny("fp32", lens=(9, 13), n_q=2, seed=4, heads=4, hidden_out=6)
+    host = gen.generate(w)
+    full = bench.oracle_decode(O, w, host, [0, 1])
+    halves = bench.oracle_decode(O, w, host, [0, 1], heads=[0, 2]) + \
+        bench.oracle_decode(O, w, host, [0, 1], heads=[1, 3])
+    assert full.shape == (w.batch * w.n_q, 6)
+    np.testing.assert_allclose(halves, full, rtol=1e-12, atol=1e-12)
+    # and the full projection is the decode output times W_O
+    dec = O.decode_step(host, w.n_q, w.d_c, w.softmax_scale).reshape(w.batch * w.n_q, -1)
+    np.testing.assert_allclose(full, dec @ host["W_O"].double().numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_roofline_counts_the_output_projection():
+    w = gen.WORKLOADS["v3_b64_ragged_oproj"]
+    lens = [2048] * w.batch
+    K = w.heads * w.v_dim
+    expect = (K * w.hidden_out + 64 * K + 64 * w.hidden_out) * 2
+    assert RF.kernel_bytes("sm100_oproj", w, lens, 2, 2) == expect
+    base = RF.step_work(gen.WORKLOADS["v3_b64_ragged"], lens)
+    got = RF.step_work(w, lens)
+    assert got["bytes"] - base["bytes"] == expect
+    assert got["flops"] - base["flops"] == 2 * 64 * K * w.hidden_out

@@ -42,6 +42,10 @@ MUTANTS = [
     ("rms norm applied to the rope key too", "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)",
      "rows[:, :d_c] = rms_norm(y[:, :d_c], rms_gamma, eps)\n        rows[:, d_c:] = y[:, d_c:] / np.sqrt(np.mean(y[:, d_c:] ** 2, axis=-1, keepdims=True) + eps)\n        y = rows"),
     ("rms norm without gamma", "return _f64(gamma) * c / rms", "return c / rms"),
+    ("output heads concatenated value-major", "return out.reshape(T, H * v) @ _f64(W_O)",
+     "return out.transpose(0, 2, 1).reshape(T, H * v) @ _f64(W_O)"),
+    ("output projection with the weight transposed per block", "return out.reshape(T, H * v) @ _f64(W_O)",
+     "return out.reshape(T, H * v) @ _f64(W_O)[::-1]"),
     ("sparse selection ignores the count", "rows = sel[b, j, : int(n_sel[b, j])]", "rows = sel[b, j]"),
     ("sparse rows taken one slot late", "c = _f64(c_kv[b, rows])                             # [k][d_c]",
      "c = _f64(c_kv[b, rows + 1])                         # [k][d_c]"),
