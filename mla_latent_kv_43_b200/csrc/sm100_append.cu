@@ -36,7 +36,7 @@ namespace sm100 {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kSplit = 8;                // CTAs per cluster, splitting K
+constexpr int kSplitMax = 8;             // CTAs per cluster splitting K (the append's split)
 constexpr int kStages = 4;
 constexpr int kBoxA = 8192;              // 64 k rows x 64 features x 2 B
 constexpr int kMaxN = 256;               // tokens per launch tile
@@ -59,7 +59,8 @@ __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
 
 // kAppend: rotate the rope features and store cache entries at the tokens'
 // slots; otherwise store the plain product y = x W (the output projection).
-template <bool kAppend>
+// kSplit CTAs of a cluster share one 128-feature tile, each over 1/kSplit of K.
+template <bool kAppend, int kSplit>
 __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kThreads, 1)
 append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapX, AppendArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -158,15 +159,18 @@ append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ 
     tc_fence_before();
     cluster_sync();          // every partial of the cluster is in place
 
-    // CTA `rank` finishes feature rows [16 rank, 16 rank + 16) of the tile: thread
-    // (pair p, token group g) sums rows 2p, 2p + 1 for tokens 4g .. 4g + 3.
-    const int p = t >> 4, g = t & 15;
-    const int row = 16 * (int)rank + 2 * p;
+    // CTA `rank` finishes feature rows [R rank, R rank + R) of the tile, R = 128 /
+    // kSplit: thread (pair p, token group g) sums rows 2p, 2p + 1 for tokens
+    // 4g .. 4g + 3 (+ multiples of 4 * kGroups).
+    constexpr int kRows = 128 / kSplit, kGroups = kThreads / (kRows / 2);
+    static_assert(kRows % 2 == 0 && kThreads % (kRows / 2) == 0, "feature rows per CTA");
+    const int p = t / kGroups, g = t % kGroups;
+    const int row = kRows * (int)rank + 2 * p;
     const int n = 128 * mt + row;
     uint32_t peer_part[kSplit];
 #pragma unroll
     for (int c = 0; c < kSplit; ++c) peer_part[c] = map_peer(part, (uint32_t)c);
-    for (int m4 = 4 * g; m4 < N; m4 += 64) {
+    for (int m4 = 4 * g; m4 < N; m4 += 4 * kGroups) {
         float v0[4] = {0.f, 0.f, 0.f, 0.f}, v1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < kSplit; ++c) {
@@ -235,12 +239,13 @@ int append_launch(const AppendCall& c, int* launches) {
     const int stage_bytes = 2 * kBoxA + N * 128;
     const int part_bytes = 128 * (N * 4 + 16);
     const size_t smem = (size_t)(kStages * stage_bytes > part_bytes ? kStages * stage_bytes : part_bytes) + 1024;
-    if (cudaFuncSetAttribute(append_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(append_kernel<true, kSplitMax>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
-    const dim3 grid((kFeatures + 127) / 128 * kSplit, (M + N - 1) / N);
+    const dim3 grid((kFeatures + 127) / 128 * kSplitMax, (M + N - 1) / N);
     prof_begin(c.stream, "sm100_append");
-    const cudaError_t e = launch_plain(append_kernel<true>, grid, dim3(kThreads), smem, c.stream, mw, mx, a);
+    const cudaError_t e =
+        launch_plain(append_kernel<true, kSplitMax>, grid, dim3(kThreads), smem, c.stream, mw, mx, a);
     prof_end(c.stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
@@ -275,12 +280,18 @@ int gemm_xw_launch(const void* x, const void* W, int M, int K, int n_out, __nv_b
     const int stage_bytes = 2 * kBoxA + N * 128;
     const int part_bytes = 128 * (N * 4 + 16);
     const size_t smem = (size_t)(kStages * stage_bytes > part_bytes ? kStages * stage_bytes : part_bytes) + 1024;
-    if (cudaFuncSetAttribute(append_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+    // the widest split whose grid still runs in one wave (two CTAs per SM when
+    // their shared memory fits: a 448-CTA grid at 7168 columns took 1.5 waves)
+    const int tiles = (n_out + 127) / 128 * ((M + N - 1) / N);
+    const int per_sm = smem <= 112 * 1024 ? 2 : 1;
+    int split = kSplitMax;
+    while (split > 2 && tiles * split > per_sm * sm_count()) split /= 2;
+    auto kern = split == 8 ? append_kernel<false, 8> : split == 4 ? append_kernel<false, 4> : append_kernel<false, 2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
-    const dim3 grid((n_out + 127) / 128 * kSplit, (M + N - 1) / N);
+    const dim3 grid((n_out + 127) / 128 * split, (M + N - 1) / N);
     prof_begin(stream, name);
-    const cudaError_t e = launch_plain(append_kernel<false>, grid, dim3(kThreads), smem, stream, mw, mx, a);
+    const cudaError_t e = launch_plain(kern, grid, dim3(kThreads), smem, stream, mw, mx, a);
     prof_end(stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
