@@ -212,6 +212,25 @@ MLA_API int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q,
 MLA_API int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t hidden, const void* out,
                const void* W_O, void* y, int32_t* status, void* stream);
 
+/* Prefill: the same attention as mla_decode (same inputs, same outputs, the
+ * queries' own entries already in the cache) evaluated in the materialised
+ * factorisation, for many query tokens per sequence: each cached latent of the
+ * first max_len rows of a sequence is expanded once into per-head keys c W_uk[h]
+ * and values c W_uv[h], then ordinary causal attention runs per head over the
+ * 192-wide key [c W_uk[h] || k_rope] and the 128-wide value ("Understanding MLA",
+ * sections "Reference code vs serving engines" and 6; "Multi-Head Latent
+ * Attention", section 3).  The materialised rows live in the workspace.
+ * Arguments as for mla_decode; workspace >= mla_prefill_workspace_bytes(),
+ * 256-byte aligned.  bf16 with d_c 512, d_rope 64, qk_nope 128, v_dim 128 and
+ * any head count; other dims return MLA_ERR_UNSUPPORTED, as do sizes whose
+ * batch * n_q, batch * max_len or batch * capacity reach 2^31.  A sequence with
+ * a bad length sets MLA_ERR_LEN and gets zero outputs. */
+MLA_API size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len);
+MLA_API int mla_prefill(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_nope, const void* q_rope,
+                        const void* W_uk, const void* W_uv, const void* cache, int64_t capacity,
+                        const int32_t* seq_lens, int64_t max_len, void* out, void* workspace,
+                        size_t workspace_bytes, int32_t* status, void* stream);
+
 /* Failure-path self-test.  Every kernel of the library waits on its
  * barriers through one bounded wait that gives up after a time limit,
  * records MLA_ERR_TIMEOUT in the status word and lets the kernel leave

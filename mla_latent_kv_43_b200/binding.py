@@ -66,6 +66,10 @@ def lib() -> ctypes.CDLL:
         L.mla_decode.restype = ctypes.c_int
         L.mla_decode_sparse.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, I32, P, P, SZ, I32, P, P]
         L.mla_decode_sparse.restype = ctypes.c_int
+        L.mla_prefill_workspace_bytes.argtypes = [D, I32, I32, I64]
+        L.mla_prefill_workspace_bytes.restype = ctypes.c_size_t
+        L.mla_prefill.argtypes = [D, I32, I32, P, P, P, P, P, I64, P, I64, P, P, ctypes.c_size_t, P, P]
+        L.mla_prefill.restype = ctypes.c_int
         L.mla_output_projection.argtypes = [D, I32, I32, P, P, P, P, P]
         L.mla_output_projection.restype = ctypes.c_int
         L.mla_selftest_wait_timeout.argtypes = [P, I64, P]
@@ -168,6 +172,21 @@ def mla_decode_sparse(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor,
                                    _ptr(sel), _ptr(n_sel), sel.shape[-1], _ptr(out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), splits, _ptr(status),
                                    _stream(stream)), "mla_decode_sparse")
+
+
+def mla_prefill_workspace_bytes(dims: MlaDims, batch: int, n_q: int, max_len: int) -> int:
+    return lib().mla_prefill_workspace_bytes(ctypes.byref(dims), batch, n_q, max_len)
+
+
+def mla_prefill(dims: MlaDims, q_nope: torch.Tensor, q_rope: torch.Tensor, W_uk: torch.Tensor,
+                W_uv: torch.Tensor, cache: torch.Tensor, seq_lens: torch.Tensor, max_len: int,
+                out: torch.Tensor, workspace: torch.Tensor, status: torch.Tensor, stream=None):
+    """The decode's attention in the materialised factorisation (many query tokens)."""
+    batch, n_q = q_nope.shape[0], q_nope.shape[1]
+    _check(lib().mla_prefill(ctypes.byref(dims), batch, n_q, _ptr(q_nope), _ptr(q_rope), _ptr(W_uk), _ptr(W_uv),
+                             _ptr(cache), cache.shape[1], _ptr(seq_lens), max_len, _ptr(out), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)),
+           "mla_prefill")
 
 
 def mla_output_projection(dims: MlaDims, out: torch.Tensor, W_O: torch.Tensor, y: torch.Tensor,

@@ -164,6 +164,46 @@ int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q, const vo
     return rc;
 }
 
+static bool prefill_dims_ok(const mla_dims* d) {
+    return d->dtype == MLA_BF16 && d->d_c == 512 && d->d_rope == 64 && d->qk_nope == 128 && d->v_dim == 128;
+}
+
+size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len) {
+    if (validate_dims(dims) || batch < 0 || n_q < 0 || max_len < 0) return 0;
+    mla::sm100::PrefillLayout L;
+    mla::sm100::prefill_layout(*dims, batch, n_q, max_len, &L);
+    return (size_t)L.total;
+}
+
+int mla_prefill(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_nope, const void* q_rope,
+                const void* W_uk, const void* W_uv, const void* cache, int64_t capacity, const int32_t* seq_lens,
+                int64_t max_len, void* out, void* workspace, size_t workspace_bytes, int32_t* status,
+                void* stream) {
+    g_last_launches = 0;
+    int rc = validate_dims(dims);
+    if (rc) return rc;
+    if (batch < 0 || n_q < 0 || capacity <= 0) return MLA_ERR_ARG;
+    if (batch == 0 || n_q == 0) return MLA_OK;
+    if (max_len < n_q || max_len > capacity) return MLA_ERR_ARG;
+    if (!q_nope || !q_rope || !W_uk || !W_uv || !cache || !seq_lens || !out || !workspace || !status)
+        return MLA_ERR_ARG;
+    if (!prefill_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
+    const int64_t lim = (int64_t)1 << 31;
+    if ((int64_t)batch * n_q >= lim || (int64_t)batch * max_len >= lim || (int64_t)batch * capacity >= lim)
+        return MLA_ERR_UNSUPPORTED;
+    if (workspace_bytes < mla_prefill_workspace_bytes(dims, batch, n_q, max_len)) return MLA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_ALIGN;
+    if (!aligned16(q_nope) || !aligned16(q_rope) || !aligned16(W_uk) || !aligned16(W_uv) || !aligned16(cache) ||
+        !aligned16(out))
+        return MLA_ERR_ALIGN;
+    mla::sm100::PrefillCall c{*dims, batch, n_q, q_nope, q_rope, W_uk, W_uv, cache, capacity, seq_lens,
+                              max_len, out, static_cast<char*>(workspace), status, (cudaStream_t)stream};
+    int launches = 0;
+    rc = mla::sm100::prefill_launch(c, &launches);
+    g_last_launches = launches;
+    return rc;
+}
+
 int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t hidden, const void* out, const void* W_O,
                           void* y, int32_t* status, void* stream) {
     g_last_launches = 0;

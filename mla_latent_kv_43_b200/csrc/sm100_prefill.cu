@@ -1,0 +1,474 @@
+// Prefill (materialised) MLA attention on tcgen05 tensor cores.
+//
+// With many query tokens per sequence the absorbed form stops paying: its
+// score and weighted sum run over the 576-wide latent for every (query, key)
+// pair, 2 H (576 + 512) flops, while expanding each cached latent once into
+// the per-head keys and values costs 2 * 512 * 256 H flops per key and the
+// attention itself then runs in the 192/128-wide head space, 2 H (192 + 128)
+// flops per pair.  This is the training / reference factorisation of
+// "Understanding MLA (Multi-head Latent Attention)" (sections "Reference code
+// vs serving engines" and 6, "Training vs decode"), written out in
+// "Multi-Head Latent Attention", section 3 (reference implementation):
+// k_content = c W_UK, v = c W_UV, the shared rotated rope key broadcast to
+// every head, ordinary scaled dot-product attention over the concatenated
+// 192 dims, scale 1/sqrt(192).
+//
+// Steps of one call (same inputs and outputs as the absorbed decode):
+//   1. q_rot[t][h] = RoPE(q_rope[t][h], p(t))                       (CUDA cores)
+//   2. Kn = c W_uk, V = c W_uv for rows t < max_len of each sequence,
+//      rows at or past the sequence's length zeroed                  (tcgen05 GEMM)
+//   3. causal flash attention per (128-query tile, head, sequence)   (this file)
+//
+// Attention kernel.  One CTA: 128 queries (the TMEM lanes / M of both GEMMs)
+// of one head.  Per 64-key tile: S = [q_nope || q_rot] [Kn || k_rope]^T
+// (M 128, N 64, K 192) into one of two TMEM score buffers; the softmax warps
+// (one thread per query row) mask keys past the row's position, keep a
+// base-2 running maximum that moves only when it grows by more than 2^8
+// (O and the row sum are rescaled then), write P as bf16 into one of two
+// shared-memory tiles; O += P V (M 128, N 128, K 64) with V read MN-major.
+// Roles (192 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax.
+// TMEM: O [0,128), S double buffer [128,256).
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "profile.h"
+#include "sm100_host.h"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace sm100 {
+
+namespace {
+
+constexpr int kQ = 128;                            // queries per CTA
+constexpr int kKeys = 64;                          // keys per tile
+constexpr int kStages = 3;
+constexpr int kBox = 8192;                         // 64 rows x 128 B
+constexpr int kQBox = 16384;                       // 128 rows x 128 B
+constexpr int kOffStage = 3 * kQBox;               // Q: q_nope[0:64], q_nope[64:128], q_rot
+constexpr int kStageBytes = 5 * kBox;              // Kn[0:64], Kn[64:128], k_rope, V[0:64], V[64:128]
+constexpr int kOffP = kOffStage + kStages * kStageBytes;
+constexpr int kSmemBytes = kOffP + 2 * kQBox;      // two P tiles (128 queries x 64 keys, bf16)
+constexpr int kThreads = 192;
+constexpr uint32_t kColO = 0, kColS = 128, kTmemCols = 256;
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+struct PrefillArgs {
+    const int32_t* seq_lens;
+    int B, n_q, H, q_tiles;
+    int64_t capacity, max_len;
+    float scale_log2;                              // softmax scale * log2(e)
+    __nv_bfloat16* out;                            // [B][n_q][H][128]
+    int32_t* status;
+};
+
+struct RopeTurns {
+    uint64_t turn[32];
+};
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// q_rot[t][h][0:64] = RoPE(q_rope[t][h], p(t)): one thread per (token, head).
+__global__ void __launch_bounds__(128) prefill_qrope_kernel(const __nv_bfloat16* __restrict__ q_rope,
+                                                            const int32_t* __restrict__ seq_lens, int BJ, int n_q,
+                                                            int H, RopeTurns rt, __nv_bfloat16* __restrict__ q_rot) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)BJ * H) return;
+    const int t = (int)(i / H);
+    const int b = t / n_q, j = t % n_q;
+    const int64_t p = query_pos(seq_lens[b], n_q, j);
+    const uint4* src = reinterpret_cast<const uint4*>(q_rope + i * 64);
+    uint4* dst = reinterpret_cast<uint4*>(q_rot + i * 64);
+    uint4 v[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] = src[c];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
+            float y0, y1;
+            rope_pair_turn(x.x, x.y, p, rt.turn[4 * c + k], &y0, &y1);
+            w[k] = pack_bf16(y0, y1);
+        }
+        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_constant__ CUtensorMap map_qr,
+                      const __grid_constant__ CUtensorMap map_kn, const __grid_constant__ CUtensorMap map_kr,
+                      const __grid_constant__ CUtensorMap map_v, PrefillArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // o_done[g & 1] completes when O GEMM g is done; it also frees P tile g & 1
+    // and (through kv_empty) stage g % 3.  Every waiter sees each completion of
+    // a barrier in order, so a parity names exactly one completion.
+    __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2], o_done[2],
+        drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // longest query tiles first: block L takes tile q_tiles - 1 - L / (H B)
+    const int per = a.H * a.B;
+    const int qt = a.q_tiles - 1 - (int)(blockIdx.x / per);
+    const int hb = (int)(blockIdx.x % per);
+    const int h = hb % a.H, b = hb / a.H;
+    const int q0 = qt * kQ;
+    const int64_t len = a.seq_lens[b];
+    const bool seq_ok = len_ok(len, a.n_q, a.capacity, a.max_len);
+    // keys 0 .. p of the tile's last query are visible to some query of the tile
+    const int j_last = min(q0 + kQ, a.n_q) - 1;
+    const int n_tiles = seq_ok ? (int)((len - a.n_q + j_last) / kKeys) + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_free[i], 4);      // the four softmax warps have read the score tile
+            mbar_init(&p_full[i], 4);      // ... have written their P rows
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(&drain, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    const uint32_t sbase = smem_u32(smem);
+    volatile int* abort = &abort_flag;
+    auto fail = [&]() {
+        *abort = 1;
+        set_status(a.status, MLA_ERR_TIMEOUT);
+    };
+    // lane 0 waits (bounded), the warp follows its outcome
+    auto wait_w = [&](uint64_t* bar, uint32_t parity) -> bool {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (n_tiles > 0 && elect_one()) {
+            tma_prefetch(&map_kn);
+            tma_prefetch(&map_v);
+            const int qrow = b * a.n_q + q0;
+            mbar_expect_tx(&q_full, 3 * kQBox);
+            tma_load_3d(smem, &map_qn, &q_full, 0, h, qrow);
+            tma_load_3d(smem + kQBox, &map_qn, &q_full, 64, h, qrow);
+            tma_load_3d(smem + 2 * kQBox, &map_qr, &q_full, 0, h, qrow);
+            const int krow = b * (int)a.max_len, crow = b * (int)a.capacity;
+            int i = 0;
+            for (; i < n_tiles; ++i) {
+                const int s = i % kStages;
+                if (i >= kStages && !mbar_wait(&kv_empty[s], ((i / kStages) - 1) & 1, abort)) {
+                    fail();
+                    break;
+                }
+                uint8_t* st = smem + kOffStage + s * kStageBytes;
+                const int t0 = i * kKeys;
+                // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
+                // tensor they are zero filled
+                mbar_expect_tx(&kv_full[s], kStageBytes);
+                tma_load_3d(st, &map_kn, &kv_full[s], 0, h, krow + t0);
+                tma_load_3d(st + kBox, &map_kn, &kv_full[s], 64, h, krow + t0);
+                tma_load_2d(st + 2 * kBox, &map_kr, &kv_full[s], 512, crow + t0);
+                tma_load_3d(st + 3 * kBox, &map_v, &kv_full[s], 0, h, krow + t0);
+                tma_load_3d(st + 4 * kBox, &map_v, &kv_full[s], 64, h, krow + t0);
+            }
+            // no copy of this CTA may still be in flight when it exits
+            mbar_wait(&q_full, 0, nullptr);
+            for (int k = i > kStages ? i - kStages : 0; k < i; ++k)
+                mbar_wait(&kv_full[k % kStages], (k / kStages) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // S(i) is issued before O(i - 1), so the softmax of tile i overlaps the
+        // value GEMM of tile i - 1.
+        if (n_tiles > 0) {
+            constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
+            constexpr uint32_t idO = idesc_bf16(128, 128, false, true);
+            const uint64_t dQ = sdesc(sbase, 16, 1024, kSwizzle128);                          // K-major
+            const uint64_t dK = sdesc(sbase + kOffStage, 16, 1024, kSwizzle128);              // K-major
+            const uint64_t dV = sdesc(sbase + kOffStage + 3 * kBox, kBox, 1024, kSwizzle128);  // MN-major
+            const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);                  // K-major
+            auto issue_o = [&](int g) -> bool {
+                const int pb = g & 1, s = g % kStages;
+                if (!wait_w(&p_full[pb], (g >> 1) & 1)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ss_w(tmem + kColO, sdesc_add(dP, pb * kQBox + ks * 32),
+                             sdesc_add(dV, s * kStageBytes + ks * 2048), idO, (g | ks) ? 1u : 0u);
+                mma_commit_w(&kv_empty[s]);
+                mma_commit_w(&o_done[pb]);
+                return true;
+            };
+            bool ok = wait_w(&q_full, 0);
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                const int s = i % kStages, sb = i & 1;
+                ok = wait_w(&kv_full[s], (i / kStages) & 1) && (i < 2 || wait_w(&s_free[sb], ((i >> 1) - 1) & 1));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t dS = tmem + kColS + 64 * sb;
+#pragma unroll
+                for (int kb = 0; kb < 3; ++kb)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss_w(dS, sdesc_add(dQ, kb * kQBox + ks * 32),
+                                 sdesc_add(dK, s * kStageBytes + kb * kBox + ks * 32), idS, (kb | ks) ? 1u : 0u);
+                mma_commit_w(&s_full[sb]);
+                if (i >= 1) ok = issue_o(i - 1);
+            }
+            if (ok) ok = issue_o(n_tiles - 1);
+            if (!ok && lane == 0) fail();
+            mma_commit_w(&drain);
+            if (lane == 0) mbar_wait(&drain, 0, nullptr);
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int q = warp & 3;                      // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;                 // query row of the tile
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const int j = q0 + r;
+        const bool row_ok = j < a.n_q;
+        const int64_t p = (seq_ok && row_ok) ? query_pos(len, a.n_q, j) : -1;
+        uint4* orow = reinterpret_cast<uint4*>(a.out + (((int64_t)b * a.n_q + j) * a.H + h) * 128);
+        if (!seq_ok) {
+            if (row_ok)
+#pragma unroll
+                for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (r == 0) set_status(a.status, MLA_ERR_LEN);
+        } else {
+            float m_used = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int sb = i & 1;
+                if (!(ok = wait_w(&s_full[sb], (i >> 1) & 1))) break;
+                tc_fence_after();
+                float x[64];
+                {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, rr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(rr[k]);
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, rr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) x[32 + k] = __uint_as_float(rr[k]);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[sb]);
+                // causal mask (selects, so whatever lies past the sequence never leaks in)
+                const int64_t key0 = (int64_t)i * kKeys;
+                if (key0 + kKeys - 1 > p) {
+#pragma unroll
+                    for (int n = 0; n < 64; ++n) x[n] = key0 + n <= p ? x[n] : -INFINITY;
+                }
+                float mx8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mx8[k] = fmaxf(fmaxf(fmaxf(x[k], x[k + 8]), fmaxf(x[k + 16], x[k + 24])),
+                                   fmaxf(fmaxf(x[k + 32], x[k + 40]), fmaxf(x[k + 48], x[k + 56])));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
+                const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
+                // the maximum moves only when it grew by more than 2^8 (-inf + 8 is -inf)
+                const float m = mx > m_used + kRescaleThreshold ? mx : m_used;
+                // P tile sb is free once O GEMM i - 2 is done
+                if (i >= 2 && !(ok = wait_w(&o_done[sb], ((i - 2) >> 1) & 1))) break;
+                // O holds tiles 0 .. i - 1 relative to m_used: rescale it when m moved.
+                // TMEM accesses are warp-collective, so lanes that need none multiply by 1.
+                const bool need = m_used != -INFINITY && m > m_used;
+                if (__any_sync(0xffffffffu, need)) {
+                    if (!(ok = wait_w(&o_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
+                    tc_fence_after();
+                    const float alpha = need ? ex2(m_used - m) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t rr[16];
+                        const uint32_t ta = tmem + lane_off + kColO + 16 * c;
+                        tmem_ld16(ta, rr);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) rr[k] = __float_as_uint(__uint_as_float(rr[k]) * alpha);
+                        tmem_st16(ta, rr);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+                if (need) l *= ex2(m_used - m);
+                m_used = m;
+                const bool live = m_used != -INFINITY;      // a row with no visible key yet (or none at all)
+                const uint32_t prow = sbase + kOffP + sb * kQBox + r * 128;
+                float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t pw[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float p0 = live ? ex2(fmaf(x[8 * c + 2 * k], a.scale_log2, -m_used)) : 0.f;
+                        const float p1 = live ? ex2(fmaf(x[8 * c + 2 * k + 1], a.scale_log2, -m_used)) : 0.f;
+                        ps4[k] += p0 + p1;
+                        pw[k] = pack_bf16(p0, p1);
+                    }
+                    st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                }
+                l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[sb]);
+            }
+            // every O GEMM is done once the last one is
+            if (ok) ok = wait_w(&o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+            if (!ok) {
+                if (lane == 0) fail();
+            } else {
+                tc_fence_after();
+                const float inv = (row_ok && l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem + lane_off + kColO + 32 * c, rr);
+                    tmem_wait_ld();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        w[k] = pack_bf16(__uint_as_float(rr[2 * k]) * inv, __uint_as_float(rr[2 * k + 1]) * inv);
+                    if (row_ok)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            orow[4 * c + k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+void prefill_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, PrefillLayout* L) {
+    auto up = [](int64_t v) { return (v + 255) / 256 * 256; };
+    L->q_rot = 0;
+    L->kn = up((int64_t)batch * n_q * d.heads * 64 * 2);
+    L->v = L->kn + up((int64_t)batch * max_len * d.heads * 128 * 2);
+    L->total = L->v + up((int64_t)batch * max_len * d.heads * 128 * 2);
+}
+
+int prefill_launch(const PrefillCall& c, int* launches) {
+    const int B = c.batch, H = c.d.heads, n_q = c.n_q;
+    const int BJ = B * n_q;
+    PrefillLayout L;
+    prefill_layout(c.d, B, n_q, c.max_len, &L);
+    __nv_bfloat16* q_rot = reinterpret_cast<__nv_bfloat16*>(c.ws + L.q_rot);
+    __nv_bfloat16* kn = reinterpret_cast<__nv_bfloat16*>(c.ws + L.kn);
+    __nv_bfloat16* v = reinterpret_cast<__nv_bfloat16*>(c.ws + L.v);
+
+    // 1. query rope
+    RopeTurns rt;
+    rope_turn_table(c.d.rope_base, 64, rt.turn);
+    {
+        const int64_t n = (int64_t)BJ * H;
+        prof_begin(c.stream, "sm100_prefill_qrope");
+        prefill_qrope_kernel<<<(unsigned)((n + 127) / 128), 128, 0, c.stream>>>(
+            (const __nv_bfloat16*)c.q_rope, c.seq_lens, BJ, n_q, H, rt, q_rot);
+        prof_end(c.stream);
+        ++*launches;
+        if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+    // 2. per-head keys and values from the latent rows
+    for (int which = 0; which < 2; ++which) {
+        GemmXW g{};
+        g.x = c.cache;
+        g.W = which == 0 ? c.W_uk : c.W_uv;
+        g.K = 512;
+        g.n_out = H * 128;
+        g.y = which == 0 ? kn : v;
+        g.w_heads = H;
+        g.batches = B;
+        g.x_len = (int)c.max_len;
+        g.x_row_elems = 576;
+        g.x_batch_rows = c.capacity;
+        g.seq_lens = c.seq_lens;
+        const int rc = gemm_xw_launch(g, c.status, c.stream, which == 0 ? "sm100_prefill_kn" : "sm100_prefill_v",
+                                      launches);
+        if (rc != MLA_OK) return rc;
+    }
+    // 3. causal attention
+    CUtensorMap mqn, mqr, mkn, mkr, mv;
+    {
+        const uint64_t dims[3] = {128, (uint64_t)H, (uint64_t)BJ}, str[2] = {256, (uint64_t)H * 256};
+        const uint32_t box[3] = {64, 1, (uint32_t)kQ};
+        if (!make_map(&mqn, c.q_nope, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[3] = {64, (uint64_t)H, (uint64_t)BJ}, str[2] = {128, (uint64_t)H * 128};
+        const uint32_t box[3] = {64, 1, (uint32_t)kQ};
+        if (!make_map(&mqr, q_rot, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[3] = {128, (uint64_t)H, (uint64_t)B * c.max_len}, str[2] = {256, (uint64_t)H * 256};
+        const uint32_t box[3] = {64, 1, (uint32_t)kKeys};
+        if (!make_map(&mkn, kn, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mv, v, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[2] = {576, (uint64_t)B * c.capacity}, str[1] = {576 * 2};
+        const uint32_t box[2] = {64, (uint32_t)kKeys};
+        if (!make_map(&mkr, c.cache, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    PrefillArgs a{};
+    a.seq_lens = c.seq_lens;
+    a.B = B;
+    a.n_q = n_q;
+    a.H = H;
+    a.q_tiles = (n_q + kQ - 1) / kQ;
+    a.capacity = c.capacity;
+    a.max_len = c.max_len;
+    a.scale_log2 = c.d.softmax_scale * 1.4426950408889634f;
+    a.out = (__nv_bfloat16*)c.out;
+    a.status = c.status;
+    const size_t smem = kSmemBytes + 1024;
+    if (cudaFuncSetAttribute(prefill_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MLA_ERR_CUDA;
+    const int64_t blocks = (int64_t)a.q_tiles * H * B;
+    prof_begin(c.stream, "sm100_prefill_attend");
+    const cudaError_t e = launch_plain(prefill_attend_kernel, dim3((unsigned)blocks), dim3(kThreads), smem, c.stream,
+                                       mqn, mqr, mkn, mkr, mv, a);
+    prof_end(c.stream);
+    ++*launches;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace sm100
+}  // namespace mla

@@ -55,6 +55,7 @@ class Workload:
     n_new: int = 0
     top_k: int = 0                  # > 0: each query attends a selected subset of its keys
     hidden_out: int = 0             # > 0: the step ends with the output projection to this width
+    prefill: bool = False           # True: the materialised factorisation (mla_prefill)
     rope_base: float = 10000.0
     seed: int = 0
 
@@ -111,6 +112,12 @@ WORKLOADS: Dict[str, Workload] = {
         name="v3_b64_ragged_oproj", dtype="bf16", batch=64, n_q=1, lens=None,
         lens_range=(1024, 4096), capacity=4096, latent_rms_norm=True, seed=2,
         hidden_out=7168, **V3),
+    # prefill of a 4096-token prompt (every cached token is a query, causal)
+    # in the materialised factorisation ("Understanding MLA", section 6:
+    # training / prefill expands the latent and runs ordinary attention)
+    "v3_b1_prefill4096": Workload(
+        name="v3_b1_prefill4096", dtype="bf16", batch=1, n_q=4096, lens=(4096,),
+        capacity=4096, latent_rms_norm=True, prefill=True, seed=6, **V3),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
@@ -196,7 +203,7 @@ def generate(w: Workload) -> Dict[str, torch.Tensor]:
 
 def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6,
          v_dim=5, n_q=1, lens=(5, 9), capacity=None, seed=0, latent_rms_norm=False,
-         hidden=0, n_new=0, top_k=0, hidden_out=0) -> Workload:
+         hidden=0, n_new=0, top_k=0, hidden_out=0, prefill=False) -> Workload:
     """A small custom workload for pins and edge cases (batch = len(lens))."""
     cap = capacity if capacity is not None else max(lens)
     if batch is None:
@@ -204,4 +211,5 @@ def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6
     return Workload(name="custom", dtype=dtype, batch=batch, heads=heads, d_c=d_c,
                     d_rope=d_rope, qk_nope=qk_nope, v_dim=v_dim, n_q=n_q,
                     lens=tuple(lens), capacity=cap, latent_rms_norm=latent_rms_norm,
-                    hidden=hidden, n_new=n_new, top_k=top_k, hidden_out=hidden_out, seed=seed)
+                    hidden=hidden, n_new=n_new, top_k=top_k, hidden_out=hidden_out, prefill=prefill,
+                    seed=seed)

@@ -15,6 +15,12 @@ per query token, H * qk_nope * d_c for the absorption and H * d_c * v_dim
 for the value up-projection; 2 * hidden * (d_c + d_rope) per appended token;
 2 * H * v_dim * hidden_out per query token for the output projection, which
 reads W_O once and the head outputs once more and writes y.
+
+A prefill workload (the materialised factorisation) counts its own FLOPs:
+2 * H * (qk_nope + d_rope + v_dim) per visible (query, key) pair for the
+attention and 2 * d_c * H * (qk_nope + v_dim) per cached key for expanding
+the latent into per-head keys and values; its bytes are the same inputs and
+outputs (the expanded keys and values are implementation traffic).
 """
 from __future__ import annotations
 
@@ -61,6 +67,9 @@ def step_work(w, lens: Sequence[int]) -> Dict[str, float]:
     r["out_bytes"] = qt * H * w.v_dim * es
     r["core_flops"] = visible * 2 * H * (D + w.d_c)
     r["proj_flops"] = qt * 2 * H * w.d_c * (w.qk_nope + w.v_dim)
+    if w.prefill:
+        r["core_flops"] = visible * 2 * H * (w.qk_nope + w.d_rope + w.v_dim)
+        r["proj_flops"] = sum(keys_per_seq) * 2 * w.d_c * H * (w.qk_nope + w.v_dim)
     r["append_bytes"] = 0
     r["append_flops"] = 0
     if w.n_new:
@@ -91,6 +100,8 @@ def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_ele
     D = w.d_c + w.d_rope
     qt = w.batch * w.n_q
     H = w.heads
+    if "prefill" in kernel:
+        return 0.0                     # tensor-bound: see kernel_flops
     if "attend" in kernel or "core" in kernel:
         keys = sum(int(L) for L in lens)
         if w.top_k:
@@ -106,4 +117,24 @@ def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_ele
     if "oproj" in kernel:
         K = H * w.v_dim
         return (K * w.hidden_out + qt * K + qt * w.hidden_out) * es
+    return 0.0
+
+
+def visible_pairs(w, lens: Sequence[int]) -> int:
+    """(query, key) pairs of a causal step: query j of a sequence of L keys sees
+    keys 0 .. L - n_q + j."""
+    n = w.n_q
+    return sum(n * (int(L) - n + 1) + n * (n - 1) // 2 for L in lens)
+
+
+def kernel_flops(kernel: str, w, lens: Sequence[int]) -> float:
+    """Algorithmic FLOPs of one launch of a tensor-bound kernel (the prefill's
+    attention and latent expansion); 0 for the HBM-bound kernels."""
+    H = w.heads
+    if "prefill_attend" in kernel:
+        return 2.0 * H * (w.qk_nope + w.d_rope + w.v_dim) * visible_pairs(w, lens)
+    if "prefill_kn" in kernel:
+        return 2.0 * sum(int(L) for L in lens) * w.d_c * H * w.qk_nope
+    if "prefill_v" in kernel:
+        return 2.0 * sum(int(L) for L in lens) * w.d_c * H * w.v_dim
     return 0.0

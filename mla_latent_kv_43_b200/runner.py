@@ -6,7 +6,8 @@ keys rotated at their slot positions by ``mla_rope`` (what the append step
 would have stored), the weights, per-sequence lengths, and caller-owned
 output, workspace and status buffers.  ``step()`` runs one decode step
 (append of the new tokens when the workload has them, then attention: over
-every visible key, or over the selected ones for a top-k workload), then,
+every visible key, or over the selected ones for a top-k workload; in the
+materialised factorisation for a prefill workload), then,
 when the workload has a W_O, the output projection into ``y``.
 """
 from __future__ import annotations
@@ -50,8 +51,12 @@ class DeviceProblem:
         if self.sparse:
             self.sel = to(host["sel"])
             self.n_sel = to(host["n_sel"])
+        self.prefill = w.prefill
         ws_len = w.top_k if self.sparse else self.max_len    # the tile bound of the plan
-        self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, ws_len, splits)
+        if self.prefill:
+            self.layout = {"total": B.mla_prefill_workspace_bytes(self.dims, w.batch, w.n_q, self.max_len)}
+        else:
+            self.layout = B.mla_decode_workspace_layout(self.dims, w.batch, w.n_q, ws_len, splits)
         self.workspace = torch.empty(max(self.layout["total"], 256), dtype=torch.uint8, device=dev)
         self.has_oproj = w.hidden_out > 0
         if self.has_oproj:
@@ -69,6 +74,10 @@ class DeviceProblem:
                      batch=self.w.batch, n_new=self.w.n_new, stream=self.stream)
 
     def decode(self):
+        if self.prefill:
+            B.mla_prefill(self.dims, self.q_nope, self.q_rope, self.W_uk, self.W_uv, self.cache, self.seq_lens,
+                          self.max_len, self.out, self.workspace, self.status, stream=self.stream)
+            return
         if self.sparse:
             B.mla_decode_sparse(self.dims, self.q_nope, self.q_rope, self.W_uk, self.W_uv, self.cache,
                                 self.seq_lens, self.max_len, self.sel, self.n_sel, self.out, self.workspace,

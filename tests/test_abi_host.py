@@ -169,3 +169,29 @@ def test_output_projection_argument_checks():
     assert L.mla_output_projection(d, 4, 7168, None, P, P, P, None) == B.CODES["MLA_ERR_ARG"]
     assert L.mla_output_projection(d, 4, 7168, P, P, P, None, None) == B.CODES["MLA_ERR_ARG"]
     assert L.mla_output_projection(d, 4, 7168, P + 2, P, P, P, None) == B.CODES["MLA_ERR_ALIGN"]
+
+
+def test_prefill_argument_checks():
+    """mla_prefill reports argument errors before anything is launched."""
+    L = B.lib()
+
+    def pre(dims, batch=2, n_q=4, capacity=100, max_len=100, ws_bytes=None, ptr=FAKE, out=FAKE):
+        d = ctypes.byref(dims)
+        if ws_bytes is None:
+            ws_bytes = L.mla_prefill_workspace_bytes(d, batch, n_q, max_len)
+        return L.mla_prefill(d, batch, n_q, ptr, FAKE, FAKE, FAKE, FAKE, capacity, FAKE, max_len, out, FAKE,
+                             ws_bytes, FAKE, None)
+
+    assert pre(v3(), batch=0) == B.CODES["MLA_OK"]
+    assert pre(v3(), n_q=0) == B.CODES["MLA_OK"]
+    assert pre(v3(), max_len=3) == B.CODES["MLA_ERR_ARG"]           # < n_q
+    assert pre(v3(), max_len=101) == B.CODES["MLA_ERR_ARG"]         # > capacity
+    assert pre(v3(), ptr=None) == B.CODES["MLA_ERR_ARG"]
+    assert pre(v3(dtype="fp32")) == B.CODES["MLA_ERR_UNSUPPORTED"]
+    assert pre(v3(), ws_bytes=0) == B.CODES["MLA_ERR_WORKSPACE"]
+    assert pre(v3(), out=FAKE + 2) == B.CODES["MLA_ERR_ALIGN"]
+    assert pre(v3(), capacity=1 << 30, max_len=100) == B.CODES["MLA_ERR_UNSUPPORTED"]   # batch * capacity
+    # the workspace covers the rotated queries and the expanded keys and values
+    d = ctypes.byref(v3())
+    need = L.mla_prefill_workspace_bytes(d, 2, 4, 100)
+    assert need >= 2 * 4 * 128 * 64 * 2 + 2 * (2 * 100 * 128 * 128 * 2)
