@@ -60,21 +60,6 @@ int rope_rows(const mla_dims& d, int64_t n_rows, void* x, int64_t row_stride,
 namespace sm100 {
 int gemm_xw_launch(const void* x, const void* W, int M, int K, int n_out, __nv_bfloat16* y, int32_t* status,
                    cudaStream_t stream, const char* name, int* launches);
-// The general form: W optionally per head ([w_heads][K][128], n_out = 128 w_heads);
-// x optionally per sequence (batches > 0: x rows t < x_len of sequence b at
-// x + (b * x_batch_rows + t) * x_row_elems; y row b * x_len + t, zero where
-// t >= seq_lens[b]); otherwise x is [M][K] and y is [M][n_out].
-struct GemmXW {
-    const void* x;
-    const void* W;
-    int M, K, n_out;
-    __nv_bfloat16* y;
-    int w_heads;
-    int batches, x_len;
-    int64_t x_row_elems, x_batch_rows;
-    const int32_t* seq_lens;
-};
-int gemm_xw_launch(const GemmXW& g, int32_t* status, cudaStream_t stream, const char* name, int* launches);
 
 // Prefill: the materialised form (per-head keys and values, then causal attention).
 struct PrefillCall {

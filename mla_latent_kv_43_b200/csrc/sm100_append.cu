@@ -46,12 +46,6 @@ struct AppendArgs {
     int M, n_new, kblocks, N;            // tokens, tokens per sequence, k blocks of 64, token tile
     int n_out;                           // output width: 576 for the append, the hidden width for W_O
     __nv_bfloat16* y;                    // plain product [M][n_out] (the output projection)
-    // per-head weights: W is [n_out / 128][K][128] (one 128-column tile per head, 3-D map)
-    int w_heads;
-    // per-sequence token rows: x is [batches][x_len rows][K] (3-D map, x_tiles token tiles per
-    // sequence); output row b * x_len + t, zero where t >= seq_lens[b]
-    int x_len, x_tiles;
-    const int32_t* seq_lens;
     const int32_t* positions;
     __nv_bfloat16* cache;
     int64_t capacity;
@@ -110,17 +104,9 @@ append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ 
                 if (i >= kStages && !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, nullptr)) break;
                 uint8_t* st = smem + s * stage_bytes;
                 mbar_expect_tx(&full[s], stage_bytes);
-                if (a.w_heads) {
-                    tma_load_3d(st, &mapW, &full[s], 0, kb * 64, mt);
-                    tma_load_3d(st + kBoxA, &mapW, &full[s], 64, kb * 64, mt);
-                } else {
-                    tma_load_2d(st, &mapW, &full[s], 128 * mt, kb * 64);
-                    tma_load_2d(st + kBoxA, &mapW, &full[s], 128 * mt + 64, kb * 64);
-                }
-                if (a.x_len)
-                    tma_load_3d(st + 2 * kBoxA, &mapX, &full[s], kb * 64, (nt % a.x_tiles) * N, nt / a.x_tiles);
-                else
-                    tma_load_2d(st + 2 * kBoxA, &mapX, &full[s], kb * 64, nt * N);
+                tma_load_2d(st, &mapW, &full[s], 128 * mt, kb * 64);
+                tma_load_2d(st + kBoxA, &mapW, &full[s], 128 * mt + 64, kb * 64);
+                tma_load_2d(st + 2 * kBoxA, &mapX, &full[s], kb * 64, nt * N);
             }
         }
         __syncwarp();
@@ -201,20 +187,12 @@ append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ 
         if (n >= a.n_out) continue;                    // zero fill past the last feature
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            int m = nt * N + m4 + i;
+            const int m = nt * N + m4 + i;
+            if (m >= a.M) break;
             if constexpr (!kAppend) {
-                if (a.x_len) {
-                    const int bq = nt / a.x_tiles, t = (nt % a.x_tiles) * N + m4 + i;
-                    if (t >= a.x_len) break;
-                    m = bq * a.x_len + t;
-                    if (t >= a.seq_lens[bq]) v0[i] = v1[i] = 0.f;   // past the sequence: zero rows
-                } else if (m >= a.M) {
-                    break;
-                }
                 *reinterpret_cast<uint32_t*>(a.y + (int64_t)m * a.n_out + n) = pack_bf16(v0[i], v1[i]);
                 continue;
             }
-            if (m >= a.M) break;
             const int64_t pos = a.positions[m];
             if (pos < 0 || pos >= a.capacity) {
                 set_status(a.status, MLA_ERR_POS);
@@ -277,74 +255,41 @@ int append_launch(const AppendCall& c, int* launches) {
 // the same split-K cluster kernel without the cache epilogue.
 int gemm_xw_launch(const void* x, const void* W, int M, int K, int n_out, __nv_bfloat16* y, int32_t* status,
                    cudaStream_t stream, const char* name, int* launches) {
-    GemmXW g{};
-    g.x = x;
-    g.W = W;
-    g.M = M;
-    g.K = K;
-    g.n_out = n_out;
-    g.y = y;
-    return gemm_xw_launch(g, status, stream, name, launches);
-}
-
-int gemm_xw_launch(const GemmXW& g, int32_t* status, cudaStream_t stream, const char* name, int* launches) {
-    const int M = g.batches ? g.x_len : g.M, K = g.K, n_out = g.n_out;
     int N = (M + 15) / 16 * 16;
     if (N > kMaxN) N = kMaxN;
-    const int x_tiles = (M + N - 1) / N;
-    const int64_t token_tiles = (int64_t)x_tiles * (g.batches ? g.batches : 1);
-    if (token_tiles > 65535) return MLA_ERR_UNSUPPORTED;    // token tiles on grid.y
-    if (g.w_heads && n_out != 128 * g.w_heads) return MLA_ERR_ARG;
+    if ((M + N - 1) / N > 65535) return MLA_ERR_UNSUPPORTED;    // token tiles on grid.y
     CUtensorMap mw, mx;
-    if (g.w_heads) {
-        const uint64_t dims[3] = {128, (uint64_t)K, (uint64_t)g.w_heads}, str[2] = {256, (uint64_t)K * 256};
-        const uint32_t box[3] = {64, 64, 1};
-        if (!make_map(&mw, g.W, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-    } else {
+    {
         const uint64_t dims[2] = {(uint64_t)n_out, (uint64_t)K}, str[1] = {(uint64_t)n_out * 2};
         const uint32_t box[2] = {64, 64};
-        if (!make_map(&mw, g.W, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mw, W, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
-    if (g.batches) {
-        const uint64_t dims[3] = {(uint64_t)K, (uint64_t)g.x_len, (uint64_t)g.batches},
-                       str[2] = {(uint64_t)g.x_row_elems * 2, (uint64_t)g.x_batch_rows * g.x_row_elems * 2};
-        const uint32_t box[3] = {64, (uint32_t)N, 1};
-        if (!make_map(&mx, g.x, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-    } else {
+    {
         const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M}, str[1] = {(uint64_t)K * 2};
         const uint32_t box[2] = {64, (uint32_t)N};
-        if (!make_map(&mx, g.x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mx, x, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     AppendArgs a{};
     a.M = M;
     a.n_out = n_out;
-    a.y = g.y;
+    a.y = y;
     a.n_new = 1;
     a.kblocks = (K + 63) / 64;
     a.N = N;
     a.status = status;
-    a.w_heads = g.w_heads;
-    if (g.batches) {
-        a.x_len = g.x_len;
-        a.x_tiles = x_tiles;
-        a.seq_lens = g.seq_lens;
-    }
     const int stage_bytes = 2 * kBoxA + N * 128;
     const int part_bytes = 128 * (N * 4 + 16);
     const size_t smem = (size_t)(kStages * stage_bytes > part_bytes ? kStages * stage_bytes : part_bytes) + 1024;
     // the widest split whose grid still runs in one wave (two CTAs per SM when
     // their shared memory fits: a 448-CTA grid at 7168 columns took 1.5 waves)
-    const int64_t tiles = (int64_t)(n_out + 127) / 128 * token_tiles;
+    const int tiles = (n_out + 127) / 128 * ((M + N - 1) / N);
     const int per_sm = smem <= 112 * 1024 ? 2 : 1;
     int split = kSplitMax;
-    while (split > 1 && tiles * split > per_sm * sm_count()) split /= 2;
-    auto kern = split == 8   ? append_kernel<false, 8>
-                : split == 4 ? append_kernel<false, 4>
-                : split == 2 ? append_kernel<false, 2>
-                             : append_kernel<false, 1>;
+    while (split > 2 && tiles * split > per_sm * sm_count()) split /= 2;
+    auto kern = split == 8 ? append_kernel<false, 8> : split == 4 ? append_kernel<false, 4> : append_kernel<false, 2>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
-    const dim3 grid((n_out + 127) / 128 * split, (unsigned)token_tiles);
+    const dim3 grid((n_out + 127) / 128 * split, (M + N - 1) / N);
     prof_begin(stream, name);
     const cudaError_t e = launch_plain(kern, grid, dim3(kThreads), smem, stream, mw, mx, a);
     prof_end(stream);

@@ -16,7 +16,7 @@
 // Steps of one call (same inputs and outputs as the absorbed decode):
 //   1. q_rot[t][h] = RoPE(q_rope[t][h], p(t))                       (CUDA cores)
 //   2. Kn = c W_uk, V = c W_uv for rows t < max_len of each sequence,
-//      rows at or past the sequence's length zeroed                  (tcgen05 GEMM)
+//      rows at or past the sequence's length zeroed                  (expand_kernel)
 //   3. causal flash attention per (128-query tile, head, sequence)   (this file)
 //
 // Attention kernel.  One CTA: 128 queries (the TMEM lanes / M of both GEMMs)
@@ -104,6 +104,121 @@ __global__ void __launch_bounds__(128) prefill_qrope_kernel(const __nv_bfloat16*
         }
         dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
     }
+}
+
+// Expansion of the cached latents into per-head keys and values: one CTA per
+// (128 cache rows of a sequence, head h) computes [Kn | V][t][h] = c[t]
+// [W_uk[h] | W_uv[h]] as one GEMM with M = 128 rows, N = 256 (the head's
+// 128 key and 128 value columns), K = 512 in eight 64-wide blocks through a
+// two-stage ring.  Two CTAs share an SM (96 KB each, 256 TMEM columns each),
+// so one's epilogue overlaps the other's MMAs.
+constexpr int kExThreads = 128;
+constexpr int kExStages = 2;
+constexpr int kExStageBytes = kQBox + 4 * kBox;    // c rows [128][64], W_uk[h] 64 x 128, W_uv[h] 64 x 128
+constexpr int kExSmem = kExStages * kExStageBytes;
+
+struct ExpandArgs {
+    const int32_t* seq_lens;
+    int H, max_len, row_tiles;                     // row tiles of 128 per sequence
+    __nv_bfloat16 *kn, *v;                         // [B * max_len][H][128]
+    int32_t* status;
+};
+
+__global__ void __launch_bounds__(kExThreads, 2)
+expand_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_wk,
+              const __grid_constant__ CUtensorMap map_wv, ExpandArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[kExStages], empty[kExStages], done;
+    __shared__ uint32_t tmem_base;
+    __shared__ int flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int b = blockIdx.x / a.row_tiles, t0 = (blockIdx.x % a.row_tiles) * 128;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kExStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(&done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base;
+    constexpr int kBlocks = 8;                     // K = 512
+    if (warp == 0) {
+        if (elect_one()) {
+            for (int kb = 0; kb < kBlocks; ++kb) {
+                const int s = kb % kExStages;
+                if (kb >= kExStages && !mbar_wait(&empty[s], ((kb / kExStages) - 1) & 1, nullptr)) break;
+                uint8_t* st = smem + s * kExStageBytes;
+                mbar_expect_tx(&full[s], kExStageBytes);
+                tma_load_3d(st, &map_c, &full[s], kb * 64, t0, b);
+                tma_load_3d(st + kQBox, &map_wk, &full[s], 0, kb * 64, h);
+                tma_load_3d(st + kQBox + kBox, &map_wk, &full[s], 64, kb * 64, h);
+                tma_load_3d(st + kQBox + 2 * kBox, &map_wv, &full[s], 0, kb * 64, h);
+                tma_load_3d(st + kQBox + 3 * kBox, &map_wv, &full[s], 64, kb * 64, h);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        constexpr uint32_t idesc = idesc_bf16(128, 256, false, true);
+        const uint32_t sb0 = smem_u32(smem);
+        const uint64_t da = sdesc(sb0, 16, 1024, kSwizzle128);                 // c rows, K-major
+        const uint64_t db = sdesc(sb0 + kQBox, kBox, 1024, kSwizzle128);       // weights, MN-major
+        bool ok = true;
+        for (int kb = 0; kb < kBlocks && ok; ++kb) {
+            const int s = kb % kExStages;
+            int r = 0;
+            if (lane == 0) r = mbar_wait(&full[s], (kb / kExStages) & 1, nullptr) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_ss_w(tmem, sdesc_add(da, s * kExStageBytes + ks * 32),
+                         sdesc_add(db, s * kExStageBytes + ks * 2048), idesc, (kb | ks) ? 1u : 0u);
+            mma_commit_w(&empty[s]);
+        }
+        mma_commit_w(&done);
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        flag = mbar_wait(&done, 0, nullptr) ? 1 : 0;
+        if (!flag) set_status(a.status, MLA_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    tc_fence_after();
+    // row t0 + r of sequence b: 256 columns leave TMEM in eight 32-column chunks
+    const int r = warp * 32 + lane, t = t0 + r;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const bool row_ok = t < a.max_len;
+    const bool zero = !flag || t >= a.seq_lens[b];
+    const int64_t orow = ((int64_t)b * a.max_len + t) * a.H + h;
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_off + 32 * c, rr);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            w[k] = zero ? 0u : pack_bf16(__uint_as_float(rr[2 * k]), __uint_as_float(rr[2 * k + 1]));
+        if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>((c < 4 ? a.kn : a.v) + orow * 128 + 32 * (c & 3));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tmem, 256);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -406,22 +521,41 @@ int prefill_launch(const PrefillCall& c, int* launches) {
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
     // 2. per-head keys and values from the latent rows
-    for (int which = 0; which < 2; ++which) {
-        GemmXW g{};
-        g.x = c.cache;
-        g.W = which == 0 ? c.W_uk : c.W_uv;
-        g.K = 512;
-        g.n_out = H * 128;
-        g.y = which == 0 ? kn : v;
-        g.w_heads = H;
-        g.batches = B;
-        g.x_len = (int)c.max_len;
-        g.x_row_elems = 576;
-        g.x_batch_rows = c.capacity;
-        g.seq_lens = c.seq_lens;
-        const int rc = gemm_xw_launch(g, c.status, c.stream, which == 0 ? "sm100_prefill_kn" : "sm100_prefill_v",
-                                      launches);
-        if (rc != MLA_OK) return rc;
+    {
+        CUtensorMap mc, mwk, mwv;
+        {
+            const uint64_t dims[3] = {512, (uint64_t)c.max_len, (uint64_t)B},
+                           str[2] = {576 * 2, (uint64_t)c.capacity * 576 * 2};
+            const uint32_t box[3] = {64, 128, 1};
+            if (!make_map(&mc, c.cache, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        }
+        {
+            const uint64_t dims[3] = {128, 512, (uint64_t)H}, str[2] = {256, 512 * 256};
+            const uint32_t box[3] = {64, 64, 1};
+            if (!make_map(&mwk, c.W_uk, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+            if (!make_map(&mwv, c.W_uv, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        }
+        ExpandArgs e{};
+        e.seq_lens = c.seq_lens;
+        e.H = H;
+        e.max_len = (int)c.max_len;
+        e.row_tiles = (int)((c.max_len + 127) / 128);
+        e.kn = kn;
+        e.v = v;
+        e.status = c.status;
+        const size_t smem = kExSmem + 1024;
+        if (cudaFuncSetAttribute(expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return MLA_ERR_CUDA;
+        const int64_t gx = (int64_t)B * e.row_tiles;
+        if (gx >= ((int64_t)1 << 31) || H > 65535) return MLA_ERR_UNSUPPORTED;
+        prof_begin(c.stream, "sm100_prefill_expand");
+        const cudaError_t err =
+            launch_plain(expand_kernel, dim3((unsigned)gx, (unsigned)H), dim3(kExThreads), smem, c.stream, mc, mwk,
+                         mwv, e);
+        prof_end(c.stream);
+        ++*launches;
+        if (err != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
     // 3. causal attention
     CUtensorMap mqn, mqr, mkn, mkr, mv;

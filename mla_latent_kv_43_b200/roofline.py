@@ -133,8 +133,6 @@ def kernel_flops(kernel: str, w, lens: Sequence[int]) -> float:
     H = w.heads
     if "prefill_attend" in kernel:
         return 2.0 * H * (w.qk_nope + w.d_rope + w.v_dim) * visible_pairs(w, lens)
-    if "prefill_kn" in kernel:
-        return 2.0 * sum(int(L) for L in lens) * w.d_c * H * w.qk_nope
-    if "prefill_v" in kernel:
-        return 2.0 * sum(int(L) for L in lens) * w.d_c * H * w.v_dim
+    if "prefill_expand" in kernel:
+        return 2.0 * sum(int(L) for L in lens) * w.d_c * H * (w.qk_nope + w.v_dim)
     return 0.0

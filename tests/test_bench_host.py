@@ -51,3 +51,18 @@ def test_roofline_counts_the_output_projection():
     got = RF.step_work(w, lens)
     assert got["bytes"] - base["bytes"] == expect
     assert got["flops"] - base["flops"] == 2 * 64 * K * w.hidden_out
+
+
+def test_prefill_flop_counts():
+    """Causal pairs in closed form equal the count by brute force; the
+    prefill's kernels count the materialised factorisation's FLOPs."""
+    w = gen.tiny("bf16", lens=(7, 12, 30), n_q=5, prefill=True, heads=3, d_c=8, d_rope=4, qk_nope=6, v_dim=5)
+    lens = [7, 12, 30]
+    brute = sum(1 for L in lens for j in range(w.n_q) for k in range(L) if k <= L - w.n_q + j)
+    assert RF.visible_pairs(w, lens) == brute
+    assert RF.kernel_flops("sm100_prefill_attend", w, lens) == 2 * 3 * (6 + 4 + 5) * brute
+    assert RF.kernel_flops("sm100_prefill_expand", w, lens) == 2 * sum(lens) * 8 * 3 * (6 + 5)
+    assert RF.kernel_bytes("sm100_prefill_attend", w, lens, 2, 2) == 0.0
+    step = RF.step_work(w, lens)
+    assert step["flops"] == RF.kernel_flops("sm100_prefill_attend", w, lens) + \
+        RF.kernel_flops("sm100_prefill_expand", w, lens)
