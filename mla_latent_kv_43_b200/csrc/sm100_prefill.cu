@@ -26,6 +26,11 @@
 // base-2 running maximum that moves only when it grows by more than 2^8
 // (O and the row sum are rescaled then), write P as bf16 into one of two
 // shared-memory tiles; O += P V (M 128, N 128, K 64) with V read MN-major.
+// Keys and values have rings of their own: a key tile is released when its
+// score GEMM completes, a value tile when its value GEMM does, so the loads
+// run several tiles ahead of the softmax.  The grid runs head by head (the
+// query tiles of one head, longest first, then the next head), so the CTAs
+// in flight share a few heads' keys and values in L2.
 // Roles (192 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax.
 // TMEM: O [0,128), S double buffer [128,256).
 #include <cuda_bf16.h>
@@ -44,12 +49,14 @@ namespace {
 
 constexpr int kQ = 128;                            // queries per CTA
 constexpr int kKeys = 64;                          // keys per tile
-constexpr int kStages = 3;
+constexpr int kKStages = 3, kVStages = 4;
 constexpr int kBox = 8192;                         // 64 rows x 128 B
 constexpr int kQBox = 16384;                       // 128 rows x 128 B
-constexpr int kOffStage = 3 * kQBox;               // Q: q_nope[0:64], q_nope[64:128], q_rot
-constexpr int kStageBytes = 5 * kBox;              // Kn[0:64], Kn[64:128], k_rope, V[0:64], V[64:128]
-constexpr int kOffP = kOffStage + kStages * kStageBytes;
+constexpr int kOffK = 3 * kQBox;                   // Q: q_nope[0:64], q_nope[64:128], q_rot
+constexpr int kKBytes = 3 * kBox;                  // key tile: Kn[0:64], Kn[64:128], k_rope
+constexpr int kVBytes = 2 * kBox;                  // value tile: V[0:64], V[64:128]
+constexpr int kOffV = kOffK + kKStages * kKBytes;
+constexpr int kOffP = kOffV + kVStages * kVBytes;
 constexpr int kSmemBytes = kOffP + 2 * kQBox;      // two P tiles (128 queries x 64 keys, bf16)
 constexpr int kThreads = 192;
 constexpr uint32_t kColO = 0, kColS = 128, kTmemCols = 256;
@@ -227,20 +234,20 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                       const __grid_constant__ CUtensorMap map_v, PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // o_done[g & 1] completes when O GEMM g is done; it also frees P tile g & 1
-    // and (through kv_empty) stage g % 3.  Every waiter sees each completion of
-    // a barrier in order, so a parity names exactly one completion.
-    __shared__ uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_free[2], p_full[2], o_done[2],
-        drain;
+    // o_done[g & 1] completes when O GEMM g is done; it also frees P tile g & 1.
+    // Every waiter sees each completion of a barrier in order, so a parity
+    // names exactly one completion.
+    __shared__ uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages], s_full[2],
+        s_free[2], p_full[2], o_done[2], drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // longest query tiles first: block L takes tile q_tiles - 1 - L / (H B)
-    const int per = a.H * a.B;
-    const int qt = a.q_tiles - 1 - (int)(blockIdx.x / per);
-    const int hb = (int)(blockIdx.x % per);
-    const int h = hb % a.H, b = hb / a.H;
+    // head by head, then sequence, then query tile (longest first)
+    const int per_head = a.q_tiles * a.B;
+    const int h = (int)(blockIdx.x / per_head);
+    const int rem = (int)(blockIdx.x % per_head);
+    const int b = rem / a.q_tiles, qt = a.q_tiles - 1 - rem % a.q_tiles;
     const int q0 = qt * kQ;
     const int64_t len = a.seq_lens[b];
     const bool seq_ok = len_ok(len, a.n_q, a.capacity, a.max_len);
@@ -250,9 +257,13 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
 
     if (threadIdx.x == 0) {
         mbar_init(&q_full, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
-            mbar_init(&kv_empty[s], 1);
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
@@ -296,28 +307,40 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
             tma_load_3d(smem + kQBox, &map_qn, &q_full, 64, h, qrow);
             tma_load_3d(smem + 2 * kQBox, &map_qr, &q_full, 0, h, qrow);
             const int krow = b * (int)a.max_len, crow = b * (int)a.capacity;
-            int i = 0;
-            for (; i < n_tiles; ++i) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait(&kv_empty[s], ((i / kStages) - 1) & 1, abort)) {
-                    fail();
+            // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
+            // tensor they are zero filled
+            int nk = 0, nv = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_tiles; ++i) {
+                const int t0 = i * kKeys;
+                const int sk = i % kKStages, sv = i % kVStages;
+                if (i >= kKStages && !mbar_wait(&k_empty[sk], ((i / kKStages) - 1) & 1, abort)) {
+                    ok = false;
                     break;
                 }
-                uint8_t* st = smem + kOffStage + s * kStageBytes;
-                const int t0 = i * kKeys;
-                // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
-                // tensor they are zero filled
-                mbar_expect_tx(&kv_full[s], kStageBytes);
-                tma_load_3d(st, &map_kn, &kv_full[s], 0, h, krow + t0);
-                tma_load_3d(st + kBox, &map_kn, &kv_full[s], 64, h, krow + t0);
-                tma_load_2d(st + 2 * kBox, &map_kr, &kv_full[s], 512, crow + t0);
-                tma_load_3d(st + 3 * kBox, &map_v, &kv_full[s], 0, h, krow + t0);
-                tma_load_3d(st + 4 * kBox, &map_v, &kv_full[s], 64, h, krow + t0);
+                uint8_t* kt = smem + kOffK + sk * kKBytes;
+                mbar_expect_tx(&k_full[sk], kKBytes);
+                tma_load_3d(kt, &map_kn, &k_full[sk], 0, h, krow + t0);
+                tma_load_3d(kt + kBox, &map_kn, &k_full[sk], 64, h, krow + t0);
+                tma_load_2d(kt + 2 * kBox, &map_kr, &k_full[sk], 512, crow + t0);
+                ++nk;
+                if (i >= kVStages && !mbar_wait(&v_empty[sv], ((i / kVStages) - 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* vt = smem + kOffV + sv * kVBytes;
+                mbar_expect_tx(&v_full[sv], kVBytes);
+                tma_load_3d(vt, &map_v, &v_full[sv], 0, h, krow + t0);
+                tma_load_3d(vt + kBox, &map_v, &v_full[sv], 64, h, krow + t0);
+                ++nv;
             }
+            if (!ok) fail();
             // no copy of this CTA may still be in flight when it exits
             mbar_wait(&q_full, 0, nullptr);
-            for (int k = i > kStages ? i - kStages : 0; k < i; ++k)
-                mbar_wait(&kv_full[k % kStages], (k / kStages) & 1, nullptr);
+            for (int k = nk > kKStages ? nk - kKStages : 0; k < nk; ++k)
+                mbar_wait(&k_full[k % kKStages], (k / kKStages) & 1, nullptr);
+            for (int k = nv > kVStages ? nv - kVStages : 0; k < nv; ++k)
+                mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1, nullptr);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -327,25 +350,25 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idO = idesc_bf16(128, 128, false, true);
             const uint64_t dQ = sdesc(sbase, 16, 1024, kSwizzle128);                          // K-major
-            const uint64_t dK = sdesc(sbase + kOffStage, 16, 1024, kSwizzle128);              // K-major
-            const uint64_t dV = sdesc(sbase + kOffStage + 3 * kBox, kBox, 1024, kSwizzle128);  // MN-major
+            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);                  // K-major
+            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);                 // MN-major
             const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);                  // K-major
             auto issue_o = [&](int g) -> bool {
-                const int pb = g & 1, s = g % kStages;
-                if (!wait_w(&p_full[pb], (g >> 1) & 1)) return false;
+                const int pb = g & 1, sv = g % kVStages;
+                if (!wait_w(&p_full[pb], (g >> 1) & 1) || !wait_w(&v_full[sv], (g / kVStages) & 1)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_ss_w(tmem + kColO, sdesc_add(dP, pb * kQBox + ks * 32),
-                             sdesc_add(dV, s * kStageBytes + ks * 2048), idO, (g | ks) ? 1u : 0u);
-                mma_commit_w(&kv_empty[s]);
+                             sdesc_add(dV, sv * kVBytes + ks * 2048), idO, (g | ks) ? 1u : 0u);
+                mma_commit_w(&v_empty[sv]);
                 mma_commit_w(&o_done[pb]);
                 return true;
             };
             bool ok = wait_w(&q_full, 0);
             for (int i = 0; ok && i < n_tiles; ++i) {
-                const int s = i % kStages, sb = i & 1;
-                ok = wait_w(&kv_full[s], (i / kStages) & 1) && (i < 2 || wait_w(&s_free[sb], ((i >> 1) - 1) & 1));
+                const int sk = i % kKStages, sb = i & 1;
+                ok = wait_w(&k_full[sk], (i / kKStages) & 1) && (i < 2 || wait_w(&s_free[sb], ((i >> 1) - 1) & 1));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dS = tmem + kColS + 64 * sb;
@@ -354,7 +377,8 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_ss_w(dS, sdesc_add(dQ, kb * kQBox + ks * 32),
-                                 sdesc_add(dK, s * kStageBytes + kb * kBox + ks * 32), idS, (kb | ks) ? 1u : 0u);
+                                 sdesc_add(dK, sk * kKBytes + kb * kBox + ks * 32), idS, (kb | ks) ? 1u : 0u);
+                mma_commit_w(&k_empty[sk]);
                 mma_commit_w(&s_full[sb]);
                 if (i >= 1) ok = issue_o(i - 1);
             }
