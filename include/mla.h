@@ -223,7 +223,7 @@ MLA_API int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t 
  * Arguments as for mla_decode; workspace >= mla_prefill_workspace_bytes(),
  * 256-byte aligned.  bf16 with d_c 512, d_rope 64, qk_nope 128, v_dim 128 and
  * any head count; other dims return MLA_ERR_UNSUPPORTED, as do sizes whose
- * batch * n_q, batch * max_len or batch * capacity reach 2^31.  A sequence with
+ * batch * n_q, heads * batch * max_len or batch * capacity reach 2^31.  A sequence with
  * a bad length sets MLA_ERR_LEN and gets zero outputs. */
 MLA_API size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len);
 MLA_API int mla_prefill(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_nope, const void* q_rope,

@@ -189,7 +189,8 @@ int mla_prefill(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_
         return MLA_ERR_ARG;
     if (!prefill_dims_ok(dims)) return MLA_ERR_UNSUPPORTED;
     const int64_t lim = (int64_t)1 << 31;
-    if ((int64_t)batch * n_q >= lim || (int64_t)batch * max_len >= lim || (int64_t)batch * capacity >= lim)
+    if ((int64_t)batch * n_q >= lim || (int64_t)dims->heads * batch * max_len >= lim ||
+        (int64_t)batch * capacity >= lim)
         return MLA_ERR_UNSUPPORTED;
     if (workspace_bytes < mla_prefill_workspace_bytes(dims, batch, n_q, max_len)) return MLA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MLA_ERR_ALIGN;

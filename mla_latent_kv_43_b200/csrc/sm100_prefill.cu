@@ -16,7 +16,9 @@
 // Steps of one call (same inputs and outputs as the absorbed decode):
 //   1. q_rot[t][h] = RoPE(q_rope[t][h], p(t))                       (CUDA cores)
 //   2. Kn = c W_uk, V = c W_uv for rows t < max_len of each sequence,
-//      rows at or past the sequence's length zeroed                  (expand_kernel)
+//      rows at or past the sequence's length zeroed, stored head-major
+//      [H][B][max_len][128] so that a head's key tile is one contiguous
+//      16 KB block                                                    (expand_kernel)
 //   3. causal flash attention per (128-query tile, head, sequence)   (this file)
 //
 // Attention kernel.  One CTA: 128 queries (the TMEM lanes / M of both GEMMs)
@@ -126,8 +128,8 @@ constexpr int kExSmem = kExStages * kExStageBytes;
 
 struct ExpandArgs {
     const int32_t* seq_lens;
-    int H, max_len, row_tiles;                     // row tiles of 128 per sequence
-    __nv_bfloat16 *kn, *v;                         // [B * max_len][H][128]
+    int B, max_len, row_tiles;                     // row tiles of 128 per sequence
+    __nv_bfloat16 *kn, *v;                         // [H][B][max_len][128]
     int32_t* status;
 };
 
@@ -207,7 +209,7 @@ expand_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const bool row_ok = t < a.max_len;
     const bool zero = !flag || t >= a.seq_lens[b];
-    const int64_t orow = ((int64_t)b * a.max_len + t) * a.H + h;
+    const int64_t orow = ((int64_t)h * a.B + b) * a.max_len + t;
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
         uint32_t rr[32];
@@ -306,7 +308,7 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
             tma_load_3d(smem, &map_qn, &q_full, 0, h, qrow);
             tma_load_3d(smem + kQBox, &map_qn, &q_full, 64, h, qrow);
             tma_load_3d(smem + 2 * kQBox, &map_qr, &q_full, 0, h, qrow);
-            const int krow = b * (int)a.max_len, crow = b * (int)a.capacity;
+            const int krow = (h * a.B + b) * (int)a.max_len, crow = b * (int)a.capacity;
             // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
             // tensor they are zero filled
             int nk = 0, nv = 0;
@@ -320,8 +322,8 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 }
                 uint8_t* kt = smem + kOffK + sk * kKBytes;
                 mbar_expect_tx(&k_full[sk], kKBytes);
-                tma_load_3d(kt, &map_kn, &k_full[sk], 0, h, krow + t0);
-                tma_load_3d(kt + kBox, &map_kn, &k_full[sk], 64, h, krow + t0);
+                tma_load_2d(kt, &map_kn, &k_full[sk], 0, krow + t0);
+                tma_load_2d(kt + kBox, &map_kn, &k_full[sk], 64, krow + t0);
                 tma_load_2d(kt + 2 * kBox, &map_kr, &k_full[sk], 512, crow + t0);
                 ++nk;
                 if (i >= kVStages && !mbar_wait(&v_empty[sv], ((i / kVStages) - 1) & 1, abort)) {
@@ -330,8 +332,8 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 }
                 uint8_t* vt = smem + kOffV + sv * kVBytes;
                 mbar_expect_tx(&v_full[sv], kVBytes);
-                tma_load_3d(vt, &map_v, &v_full[sv], 0, h, krow + t0);
-                tma_load_3d(vt + kBox, &map_v, &v_full[sv], 64, h, krow + t0);
+                tma_load_2d(vt, &map_v, &v_full[sv], 0, krow + t0);
+                tma_load_2d(vt + kBox, &map_v, &v_full[sv], 64, krow + t0);
                 ++nv;
             }
             if (!ok) fail();
@@ -561,7 +563,7 @@ int prefill_launch(const PrefillCall& c, int* launches) {
         }
         ExpandArgs e{};
         e.seq_lens = c.seq_lens;
-        e.H = H;
+        e.B = B;
         e.max_len = (int)c.max_len;
         e.row_tiles = (int)((c.max_len + 127) / 128);
         e.kn = kn;
@@ -594,10 +596,11 @@ int prefill_launch(const PrefillCall& c, int* launches) {
         if (!make_map(&mqr, q_rot, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
-        const uint64_t dims[3] = {128, (uint64_t)H, (uint64_t)B * c.max_len}, str[2] = {256, (uint64_t)H * 256};
-        const uint32_t box[3] = {64, 1, (uint32_t)kKeys};
-        if (!make_map(&mkn, kn, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-        if (!make_map(&mv, v, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        // head-major rows: (h * B + b) * max_len + t
+        const uint64_t dims[2] = {128, (uint64_t)H * B * c.max_len}, str[1] = {256};
+        const uint32_t box[2] = {64, (uint32_t)kKeys};
+        if (!make_map(&mkn, kn, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mv, v, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
         const uint64_t dims[2] = {576, (uint64_t)B * c.capacity}, str[1] = {576 * 2};
