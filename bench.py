@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
     ap.add_argument("--min-warmup-s", type=float, default=1.5, help="minimum warm-up wall time")
+    ap.add_argument("--crossover", action="store_true",
+                    help="time the absorbed and the materialised attention for a range of query counts "
+                         "behind a 4096-token context (one GPU) and print one JSON line")
     a = ap.parse_args()
     a.warmup = max(a.warmup, 3)
     return a
@@ -423,8 +426,60 @@ def run_ours(a, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- crossover
+CROSSOVER_NQ = (1, 4, 16, 64, 128, 256, 512, 1024, 2048, 4096)
+
+
+def crossover_workload(n_q: int, context: int = 4096):
+    """One sequence of `context` cached tokens whose last n_q are queries (a
+    decode step for n_q = 1, a chunk of prefill otherwise), DeepSeek-V3 shapes."""
+    return gen.Workload(name=f"v3_b1_ctx{context}_nq{n_q}", dtype="bf16", batch=1, n_q=n_q, lens=(context,),
+                        capacity=context, latent_rms_norm=True, seed=7, **gen.V3)
+
+
+def run_crossover(a):
+    """Absorbed (mla_decode) against materialised (mla_prefill) attention for
+    the same inputs: where the per-pair cost of the 576-wide absorbed form
+    overtakes the one-off expansion of the latents ("Understanding MLA",
+    section 6: the crossover between the two factorisations)."""
+    from mla_latent_kv_43_b200.runner import DeviceProblem
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    rows = []
+    for n_q in CROSSOVER_NQ:
+        w = crossover_workload(n_q)
+        host = gen.generate(w)
+        lens = host["seq_lens"].tolist()
+        row = {"n_q": n_q}
+        for name, wv in (("absorbed", w), ("materialised", w.with_(prefill=True))):
+            prob = DeviceProblem(wv, host, device=dev)
+            for _ in range(3):
+                prob.step()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+            for s, e in ev:
+                flush.zero_()
+                s.record(stream)
+                prob.step()
+                e.record(stream)
+            torch.cuda.synchronize()
+            if prob.get_status() != 0:
+                raise RuntimeError(f"{name} n_q={n_q}: status {B.STATUS.get(prob.get_status())}")
+            row[name + "_us"] = sorted(s.elapsed_time(e) for s, e in ev)[len(ev) // 2] * 1e3
+            row[name + "_tflop"] = RF.step_work(wv, lens)["flops"] / 1e12
+            del prob
+        row["faster"] = "materialised" if row["materialised_us"] < row["absorbed_us"] else "absorbed"
+        rows.append(row)
+    print(json.dumps({"crossover": rows, "context": 4096, "dtype": "bf16",
+                      "timing": "median of 5 steps, CUDA events, L2 flushed before each"}), flush=True)
+
+
 def main():
     a = parse()
+    if a.crossover:
+        run_crossover(a)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -66,3 +66,17 @@ def test_prefill_flop_counts():
     step = RF.step_work(w, lens)
     assert step["flops"] == RF.kernel_flops("sm100_prefill_attend", w, lens) + \
         RF.kernel_flops("sm100_prefill_expand", w, lens)
+
+
+def test_crossover_workloads():
+    """The crossover sweep's workloads: one 4096-token sequence whose last n_q
+    tokens are queries; the absorbed form's FLOPs grow with n_q faster than the
+    materialised form's, which pays the expansion once."""
+    lens = [4096]
+    f = {}
+    for n in bench.CROSSOVER_NQ:
+        w = bench.crossover_workload(n)
+        assert w.batch == 1 and w.lens == (4096,) and w.n_q == n and not w.prefill
+        f[n] = (RF.step_work(w, lens)["flops"], RF.step_work(w.with_(prefill=True), lens)["flops"])
+    assert f[1][0] < f[1][1]            # one query: absorbing is cheaper
+    assert f[4096][0] > f[4096][1]      # a whole prompt: materialising is cheaper
