@@ -49,6 +49,7 @@ KERNEL_SOURCES = {  # kernel name prefix -> source file whose hash keys committe
     "sm100_attend": "mla_latent_kv_43_b200/csrc/sm100_attend.cu",
     "generic_attend": "mla_latent_kv_43_b200/csrc/generic.cu",
     "sm100_oproj": "mla_latent_kv_43_b200/csrc/sm100_append.cu",
+    "sm100_prefill_attend": "mla_latent_kv_43_b200/csrc/sm100_prefill.cu",
 }
 
 
