@@ -80,3 +80,27 @@ def test_crossover_workloads():
         f[n] = (RF.step_work(w, lens)["flops"], RF.step_work(w.with_(prefill=True), lens)["flops"])
     assert f[1][0] < f[1][1]            # one query: absorbing is cheaper
     assert f[4096][0] > f[4096][1]      # a whole prompt: materialising is cheaper
+
+
+def test_generated_scores_have_unit_variance():
+    """Scale sanity of the input recipe: with the drawn distributions the scaled
+    score q.k / sqrt(qk_nope + d_rope) has variance 1 (latent rows of unit RMS
+    or unit variance, W ~ N(0, 1/d_c), queries and rope keys ~ N(0, 1)), so a
+    mis-scaled weight or a wrong scale shows up here.  RoPE preserves norms and
+    is left out."""
+    for w in (gen.WORKLOADS["tiny_fp32"],
+              gen.tiny("fp32", lens=(600, 600), heads=4, d_c=512, d_rope=64, qk_nope=128, v_dim=128,
+                       latent_rms_norm=True, seed=9)):
+        host = gen.generate(w)
+        c = host["c_kv"].double().numpy()          # [B][cap][d_c]
+        kr = host["k_rope"].double().numpy()
+        qn = host["q_nope"].double().numpy()       # [B][n_q][H][qk_nope]
+        qr = host["q_rope"].double().numpy()
+        Wuk = host["W_uk"].double().numpy()        # [H][d_c][qk_nope]
+        s = []
+        for h in range(w.heads):
+            K = c @ Wuk[h]                         # [B][cap][qk_nope]
+            sc = (np.einsum("bk,bnk->bn", qn[:, 0, h], K) + np.einsum("bk,bnk->bn", qr[:, 0, h], kr))
+            s.append(sc.ravel() * w.softmax_scale)
+        std = float(np.std(np.concatenate(s)))
+        assert 0.85 < std < 1.15, (w.name, std)
