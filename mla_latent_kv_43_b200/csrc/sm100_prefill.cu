@@ -21,8 +21,9 @@
 //      16 KB block                                                    (expand_kernel)
 //   3. causal flash attention per (128-query tile, head, sequence)   (this file)
 //
-// Attention kernel.  One CTA: 128 queries (the TMEM lanes / M of both GEMMs)
-// of one head.  Per 64-key tile: S = [q_nope || q_rot] [Kn || k_rope]^T
+// Attention kernel.  One CTA: 256 queries of one head in two groups of 128
+// (each group's rows are the TMEM lanes / M of its GEMMs); the two groups
+// share every key and value tile.  Per 64-key tile and group: S = [q_nope || q_rot] [Kn || k_rope]^T
 // (M 128, N 64, K 192) into one of two TMEM score buffers; the softmax warps
 // (one thread per query row) mask keys past the row's position, keep a
 // base-2 running maximum that moves only when it grows by more than 2^8
@@ -33,8 +34,13 @@
 // run several tiles ahead of the softmax.  The grid runs head by head (the
 // query tiles of one head, longest first, then the next head), so the CTAs
 // in flight share a few heads' keys and values in L2.
-// Roles (192 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax.
-// TMEM: O [0,128), S double buffer [128,256).
+// The MMA warp issues both groups' score GEMMs of tile i, then their value
+// GEMMs of tile i - 1, so one group's softmax runs while the tensor core
+// works for the other.
+// Roles (320 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax of
+// group 0, warps 6-9 of group 1.
+// TMEM: O of group g at [128 g, 128 g + 128), S double buffers at
+// [256 + 128 g, 256 + 128 g + 128).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -49,19 +55,20 @@ namespace sm100 {
 
 namespace {
 
-constexpr int kQ = 128;                            // queries per CTA
+constexpr int kQ = 128;                            // queries per group
+constexpr int kGroups = 2;                         // query groups per CTA
 constexpr int kKeys = 64;                          // keys per tile
-constexpr int kKStages = 3, kVStages = 4;
+constexpr int kKStages = 2, kVStages = 2;
 constexpr int kBox = 8192;                         // 64 rows x 128 B
 constexpr int kQBox = 16384;                       // 128 rows x 128 B
-constexpr int kOffK = 3 * kQBox;                   // Q: q_nope[0:64], q_nope[64:128], q_rot
+constexpr int kOffK = kGroups * 3 * kQBox;         // Q per group: q_nope[0:64], q_nope[64:128], q_rot
 constexpr int kKBytes = 3 * kBox;                  // key tile: Kn[0:64], Kn[64:128], k_rope
 constexpr int kVBytes = 2 * kBox;                  // value tile: V[0:64], V[64:128]
 constexpr int kOffV = kOffK + kKStages * kKBytes;
 constexpr int kOffP = kOffV + kVStages * kVBytes;
-constexpr int kSmemBytes = kOffP + 2 * kQBox;      // two P tiles (128 queries x 64 keys, bf16)
-constexpr int kThreads = 192;
-constexpr uint32_t kColO = 0, kColS = 128, kTmemCols = 256;
+constexpr int kSmemBytes = kOffP + kGroups * kQBox;  // one P tile per group (128 queries x 64 keys, bf16)
+constexpr int kThreads = 320;
+constexpr uint32_t kColO = 0, kColS = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
 struct PrefillArgs {
@@ -236,11 +243,12 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                       const __grid_constant__ CUtensorMap map_v, PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // o_done[g & 1] completes when O GEMM g is done; it also frees P tile g & 1.
+    // Per group g: s_full/s_free[g][b] guard score buffer b, p_full[g] the P
+    // tile, o_done[g][t & 1] completes when O GEMM t of the group is done.
     // Every waiter sees each completion of a barrier in order, so a parity
     // names exactly one completion.
-    __shared__ uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages], s_full[2],
-        s_free[2], p_full[2], o_done[2], drain;
+    __shared__ uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+    __shared__ uint64_t s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups], o_done[kGroups][2], drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -250,12 +258,16 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
     const int h = (int)(blockIdx.x / per_head);
     const int rem = (int)(blockIdx.x % per_head);
     const int b = rem / a.q_tiles, qt = a.q_tiles - 1 - rem % a.q_tiles;
-    const int q0 = qt * kQ;
+    const int q0 = qt * kGroups * kQ;
     const int64_t len = a.seq_lens[b];
     const bool seq_ok = len_ok(len, a.n_q, a.capacity, a.max_len);
-    // keys 0 .. p of the tile's last query are visible to some query of the tile
-    const int j_last = min(q0 + kQ, a.n_q) - 1;
-    const int n_tiles = seq_ok ? (int)((len - a.n_q + j_last) / kKeys) + 1 : 0;
+    // key tiles of group g: keys 0 .. p of its last query (none for a group past n_q)
+    auto tiles_of = [&](int g) -> int {
+        const int first = q0 + g * kQ, last = min(first + kQ, a.n_q) - 1;
+        return (seq_ok && first < a.n_q) ? (int)((len - a.n_q + last) / kKeys) + 1 : 0;
+    };
+    const int n_g0 = tiles_of(0), n_g1 = tiles_of(1);
+    const int n_all = max(n_g0, n_g1);
 
     if (threadIdx.x == 0) {
         mbar_init(&q_full, 1);
@@ -267,11 +279,13 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
             mbar_init(&v_full[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 4);      // the four softmax warps have read the score tile
-            mbar_init(&p_full[i], 4);      // ... have written their P rows
-            mbar_init(&o_done[i], 1);
+        for (int g = 0; g < kGroups; ++g) {
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&s_full[g][i], 1);
+                mbar_init(&s_free[g][i], 4);   // the group's four softmax warps have read the score tile
+                mbar_init(&o_done[g][i], 1);
+            }
+            mbar_init(&p_full[g], 4);          // ... have written their P rows
         }
         mbar_init(&drain, 1);
         abort_flag = 0;
@@ -300,20 +314,25 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (n_tiles > 0 && elect_one()) {
+        if (n_all > 0 && elect_one()) {
             tma_prefetch(&map_kn);
             tma_prefetch(&map_v);
             const int qrow = b * a.n_q + q0;
-            mbar_expect_tx(&q_full, 3 * kQBox);
-            tma_load_3d(smem, &map_qn, &q_full, 0, h, qrow);
-            tma_load_3d(smem + kQBox, &map_qn, &q_full, 64, h, qrow);
-            tma_load_3d(smem + 2 * kQBox, &map_qr, &q_full, 0, h, qrow);
+            // both query tiles (rows past n_q belong to the next sequence or are zero filled)
+            mbar_expect_tx(&q_full, kGroups * 3 * kQBox);
+#pragma unroll
+            for (int g = 0; g < kGroups; ++g) {
+                uint8_t* qs = smem + g * 3 * kQBox;
+                tma_load_3d(qs, &map_qn, &q_full, 0, h, qrow + g * kQ);
+                tma_load_3d(qs + kQBox, &map_qn, &q_full, 64, h, qrow + g * kQ);
+                tma_load_3d(qs + 2 * kQBox, &map_qr, &q_full, 0, h, qrow + g * kQ);
+            }
             const int krow = (h * a.B + b) * (int)a.max_len, crow = b * (int)a.capacity;
             // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
             // tensor they are zero filled
             int nk = 0, nv = 0;
             bool ok = true;
-            for (int i = 0; ok && i < n_tiles; ++i) {
+            for (int i = 0; ok && i < n_all; ++i) {
                 const int t0 = i * kKeys;
                 const int sk = i % kKStages, sv = i % kVStages;
                 if (i >= kKStages && !mbar_wait(&k_empty[sk], ((i / kKStages) - 1) & 1, abort)) {
@@ -346,56 +365,69 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        // S(i) is issued before O(i - 1), so the softmax of tile i overlaps the
-        // value GEMM of tile i - 1.
-        if (n_tiles > 0) {
+        // Per key tile i: the score GEMMs of both groups, then the value GEMMs
+        // of tile i - 1, so each group's softmax overlaps the other's GEMMs.
+        if (n_all > 0) {
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
             constexpr uint32_t idO = idesc_bf16(128, 128, false, true);
-            const uint64_t dQ = sdesc(sbase, 16, 1024, kSwizzle128);                          // K-major
-            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);                  // K-major
-            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);                 // MN-major
-            const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);                  // K-major
-            auto issue_o = [&](int g) -> bool {
-                const int pb = g & 1, sv = g % kVStages;
-                if (!wait_w(&p_full[pb], (g >> 1) & 1) || !wait_w(&v_full[sv], (g / kVStages) & 1)) return false;
-                tc_fence_after();
+            const uint64_t dQ = sdesc(sbase, 16, 1024, kSwizzle128);                   // K-major
+            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);           // K-major
+            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);         // MN-major
+            const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);           // K-major
+            auto issue_o = [&](int t) -> bool {
+                const int sv = t % kVStages;
+                if (!wait_w(&v_full[sv], (t / kVStages) & 1)) return false;
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ss_w(tmem + kColO, sdesc_add(dP, pb * kQBox + ks * 32),
-                             sdesc_add(dV, sv * kVBytes + ks * 2048), idO, (g | ks) ? 1u : 0u);
+                for (int g = 0; g < kGroups; ++g) {
+                    if (t >= (g == 0 ? n_g0 : n_g1)) continue;
+                    if (!wait_w(&p_full[g], t & 1)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss_w(tmem + kColO + 128 * g, sdesc_add(dP, g * kQBox + ks * 32),
+                                 sdesc_add(dV, sv * kVBytes + ks * 2048), idO, (t | ks) ? 1u : 0u);
+                    mma_commit_w(&o_done[g][t & 1]);
+                }
                 mma_commit_w(&v_empty[sv]);
-                mma_commit_w(&o_done[pb]);
                 return true;
             };
             bool ok = wait_w(&q_full, 0);
-            for (int i = 0; ok && i < n_tiles; ++i) {
+            for (int i = 0; ok && i < n_all; ++i) {
                 const int sk = i % kKStages, sb = i & 1;
-                ok = wait_w(&k_full[sk], (i / kKStages) & 1) && (i < 2 || wait_w(&s_free[sb], ((i >> 1) - 1) & 1));
+                if (!(ok = wait_w(&k_full[sk], (i / kKStages) & 1))) break;
+#pragma unroll
+                for (int g = 0; g < kGroups; ++g) {
+                    if (!ok || i >= (g == 0 ? n_g0 : n_g1)) continue;
+                    if (i >= 2 && !(ok = wait_w(&s_free[g][sb], ((i >> 1) - 1) & 1))) break;
+                    tc_fence_after();
+                    const uint32_t dS = tmem + kColS + 128 * g + 64 * sb;
+#pragma unroll
+                    for (int kb = 0; kb < 3; ++kb)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_ss_w(dS, sdesc_add(dQ, g * 3 * kQBox + kb * kQBox + ks * 32),
+                                     sdesc_add(dK, sk * kKBytes + kb * kBox + ks * 32), idS, (kb | ks) ? 1u : 0u);
+                    mma_commit_w(&s_full[g][sb]);
+                }
                 if (!ok) break;
-                tc_fence_after();
-                const uint32_t dS = tmem + kColS + 64 * sb;
-#pragma unroll
-                for (int kb = 0; kb < 3; ++kb)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss_w(dS, sdesc_add(dQ, kb * kQBox + ks * 32),
-                                 sdesc_add(dK, sk * kKBytes + kb * kBox + ks * 32), idS, (kb | ks) ? 1u : 0u);
                 mma_commit_w(&k_empty[sk]);
-                mma_commit_w(&s_full[sb]);
                 if (i >= 1) ok = issue_o(i - 1);
             }
-            if (ok) ok = issue_o(n_tiles - 1);
+            if (ok) ok = issue_o(n_all - 1);
             if (!ok && lane == 0) fail();
             mma_commit_w(&drain);
             if (lane == 0) mbar_wait(&drain, 0, nullptr);
             __syncwarp();
         }
     } else {
-        // ------------------------------------------------------------ softmax warps
+        // ------------------------------------------------------------ softmax groups
+        const int g = (warp - 2) >> 2;               // query group: rows q0 + 128 g ..
         const int q = warp & 3;                      // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;                 // query row of the tile
+        const int r = q * 32 + lane;                 // query row within the group
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const int j = q0 + r;
+        const uint32_t colO = kColO + 128 * g, colS = kColS + 128 * g;
+        const int n_tiles = g == 0 ? n_g0 : n_g1;
+        const int j = q0 + g * kQ + r;
         const bool row_ok = j < a.n_q;
         const int64_t p = (seq_ok && row_ok) ? query_pos(len, a.n_q, j) : -1;
         uint4* orow = reinterpret_cast<uint4*>(a.out + (((int64_t)b * a.n_q + j) * a.H + h) * 128);
@@ -403,58 +435,49 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
             if (row_ok)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
-            if (r == 0) set_status(a.status, MLA_ERR_LEN);
-        } else {
+            if (r == 0 && g == 0) set_status(a.status, MLA_ERR_LEN);
+        } else if (n_tiles > 0) {
             float m_used = -INFINITY, l = 0.f;
             bool ok = true;
             for (int i = 0; i < n_tiles; ++i) {
                 const int sb = i & 1;
-                if (!(ok = wait_w(&s_full[sb], (i >> 1) & 1))) break;
+                if (!(ok = wait_w(&s_full[g][sb], (i >> 1) & 1))) break;
                 tc_fence_after();
-                float x[64];
-                {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, rr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) x[k] = __uint_as_float(rr[k]);
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, rr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) x[32 + k] = __uint_as_float(rr[k]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[sb]);
-                // causal mask (selects, so whatever lies past the sequence never leaks in)
+                // The score row is read twice from TMEM (maximum, then exponentials), so
+                // only 32 scores are live at a time; the causal mask is a select, so
+                // whatever lies past the sequence never leaks in.
                 const int64_t key0 = (int64_t)i * kKeys;
-                if (key0 + kKeys - 1 > p) {
+                const bool masked = key0 + kKeys - 1 > p;
+                float mx = -INFINITY;
 #pragma unroll
-                    for (int n = 0; n < 64; ++n) x[n] = key0 + n <= p ? x[n] : -INFINITY;
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem + lane_off + colS + 64 * sb + 32 * half, rr);
+                    tmem_wait_ld();
+                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        float v = __uint_as_float(rr[k]);
+                        if (masked && key0 + 32 * half + k > p) v = -INFINITY;
+                        m4[k & 3] = fmaxf(m4[k & 3], v);
+                    }
+                    mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
                 }
-                float mx8[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mx8[k] = fmaxf(fmaxf(fmaxf(x[k], x[k + 8]), fmaxf(x[k + 16], x[k + 24])),
-                                   fmaxf(fmaxf(x[k + 32], x[k + 40]), fmaxf(x[k + 48], x[k + 56])));
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
-                const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
+                mx *= a.scale_log2;
                 // the maximum moves only when it grew by more than 2^8 (-inf + 8 is -inf)
                 const float m = mx > m_used + kRescaleThreshold ? mx : m_used;
-                // P tile sb is free once O GEMM i - 2 is done
-                if (i >= 2 && !(ok = wait_w(&o_done[sb], ((i - 2) >> 1) & 1))) break;
+                // the P tile and O are free once the group's O GEMM i - 1 is done
+                if (i >= 1 && !(ok = wait_w(&o_done[g][(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
                 // O holds tiles 0 .. i - 1 relative to m_used: rescale it when m moved.
                 // TMEM accesses are warp-collective, so lanes that need none multiply by 1.
                 const bool need = m_used != -INFINITY && m > m_used;
                 if (__any_sync(0xffffffffu, need)) {
-                    if (!(ok = wait_w(&o_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
                     tc_fence_after();
                     const float alpha = need ? ex2(m_used - m) : 1.f;
 #pragma unroll 1
                     for (int c = 0; c < 8; ++c) {
                         uint32_t rr[16];
-                        const uint32_t ta = tmem + lane_off + kColO + 16 * c;
+                        const uint32_t ta = tmem + lane_off + colO + 16 * c;
                         tmem_ld16(ta, rr);
                         tmem_wait_ld();
 #pragma unroll
@@ -467,27 +490,41 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 if (need) l *= ex2(m_used - m);
                 m_used = m;
                 const bool live = m_used != -INFINITY;      // a row with no visible key yet (or none at all)
-                const uint32_t prow = sbase + kOffP + sb * kQBox + r * 128;
+                const uint32_t prow = sbase + kOffP + g * kQBox + r * 128;
                 float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t pw[4];
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t rr[32];
+                    tmem_ld32(tmem + lane_off + colS + 64 * sb + 32 * half, rr);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float p0 = live ? ex2(fmaf(x[8 * c + 2 * k], a.scale_log2, -m_used)) : 0.f;
-                        const float p1 = live ? ex2(fmaf(x[8 * c + 2 * k + 1], a.scale_log2, -m_used)) : 0.f;
-                        ps4[k] += p0 + p1;
-                        pw[k] = pack_bf16(p0, p1);
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pw[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int n = 8 * c + 2 * k;            // column within the half
+                            const bool v0 = live && !(masked && key0 + 32 * half + n > p);
+                            const bool v1 = live && !(masked && key0 + 32 * half + n + 1 > p);
+                            const float p0 = v0 ? ex2(fmaf(__uint_as_float(rr[n]), a.scale_log2, -m_used)) : 0.f;
+                            const float p1 = v1 ? ex2(fmaf(__uint_as_float(rr[n + 1]), a.scale_log2, -m_used)) : 0.f;
+                            ps4[k] += p0 + p1;
+                            pw[k] = pack_bf16(p0, p1);
+                        }
+                        const int chunk = 4 * half + c;
+                        st_shared_u4(prow + ((chunk ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                     }
-                    st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                 }
+                // both reads of score buffer sb are done
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[g][sb]);
                 l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
                 fence_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[sb]);
+                if (lane == 0) mbar_arrive(&p_full[g]);
             }
-            // every O GEMM is done once the last one is
-            if (ok) ok = wait_w(&o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+            // every O GEMM of the group is done once its last one is
+            if (ok) ok = wait_w(&o_done[g][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
             if (!ok) {
                 if (lane == 0) fail();
             } else {
@@ -496,7 +533,7 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t rr[32];
-                    tmem_ld32(tmem + lane_off + kColO + 32 * c, rr);
+                    tmem_ld32(tmem + lane_off + colO + 32 * c, rr);
                     tmem_wait_ld();
                     uint32_t w[16];
 #pragma unroll
@@ -612,7 +649,7 @@ int prefill_launch(const PrefillCall& c, int* launches) {
     a.B = B;
     a.n_q = n_q;
     a.H = H;
-    a.q_tiles = (n_q + kQ - 1) / kQ;
+    a.q_tiles = (n_q + kGroups * kQ - 1) / (kGroups * kQ);
     a.capacity = c.capacity;
     a.max_len = c.max_len;
     a.scale_log2 = c.d.softmax_scale * 1.4426950408889634f;
