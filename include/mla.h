@@ -50,7 +50,7 @@ enum mla_status {
     MLA_ERR_ARG = 1,          /* null pointer, non-positive or odd size, bad dtype */
     MLA_ERR_ALIGN = 2,        /* a pointer the kernels load with TMA is not 16-byte aligned */
     MLA_ERR_WORKSPACE = 3,    /* workspace_bytes below mla_decode_workspace_bytes() */
-    MLA_ERR_UNSUPPORTED = 4,  /* a valid request this build does not implement */
+    MLA_ERR_UNSUPPORTED = 4,  /* a valid request the library does not implement */
     MLA_ERR_CUDA = 5,         /* a CUDA launch or API call failed */
     MLA_ERR_LEN = 6,          /* device: len_b < n_q, len_b > capacity or len_b > max_len */
     MLA_ERR_POS = 7,          /* device: an append position outside [0, capacity) */
