@@ -19,24 +19,24 @@
 //      rows at or past the sequence's length zeroed, stored head-major
 //      [H][B][max_len][128] so that a head's key tile is one contiguous
 //      16 KB block                                                    (expand_kernel)
-//   3. causal flash attention per (128-query tile, head, sequence)   (this file)
+//   3. causal flash attention per (256-query tile, head, sequence)   (this file)
 //
 // Attention kernel.  One CTA: 256 queries of one head in two groups of 128
 // (each group's rows are the TMEM lanes / M of its GEMMs); the two groups
-// share every key and value tile.  Per 64-key tile and group: S = [q_nope || q_rot] [Kn || k_rope]^T
-// (M 128, N 64, K 192) into one of two TMEM score buffers; the softmax warps
-// (one thread per query row) mask keys past the row's position, keep a
-// base-2 running maximum that moves only when it grows by more than 2^8
-// (O and the row sum are rescaled then), write P as bf16 into one of two
-// shared-memory tiles; O += P V (M 128, N 128, K 64) with V read MN-major.
-// Keys and values have rings of their own: a key tile is released when its
-// score GEMM completes, a value tile when its value GEMM does, so the loads
-// run several tiles ahead of the softmax.  The grid runs head by head (the
-// query tiles of one head, longest first, then the next head), so the CTAs
-// in flight share a few heads' keys and values in L2.
-// The MMA warp issues both groups' score GEMMs of tile i, then their value
-// GEMMs of tile i - 1, so one group's softmax runs while the tensor core
-// works for the other.
+// share every key and value tile.  Per 64-key tile and group:
+// S = [q_nope || q_rot] [Kn || k_rope]^T (M 128, N 64, K 192) into one of the
+// group's two TMEM score buffers; the softmax warps (one thread per query
+// row) mask keys past the row's position, keep a base-2 running maximum that
+// moves only when it grows by more than 2^8 (O and the row sum are rescaled
+// then) and write P as bf16 into the group's shared-memory tile;
+// O += P V (M 128, N 128, K 64) with V read MN-major.  Keys and values have
+// rings of their own: a key tile is released when its last score GEMM
+// completes, a value tile when its last value GEMM does.  The grid runs head
+// by head (the query tiles of one head, longest first, then the next head),
+// so the CTAs in flight share a few heads' keys and values in L2.  The MMA
+// warp issues both groups' score GEMMs of tile i, then their value GEMMs of
+// tile i - 1, so one group's softmax runs while the tensor core works for the
+// other.
 // Roles (320 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax of
 // group 0, warps 6-9 of group 1.
 // TMEM: O of group g at [128 g, 128 g + 128), S double buffers at
