@@ -104,3 +104,30 @@ def test_generated_scores_have_unit_variance():
             s.append(sc.ravel() * w.softmax_scale)
         std = float(np.std(np.concatenate(s)))
         assert 0.85 < std < 1.15, (w.name, std)
+
+
+def test_step_work_matches_hand_counts():
+    """Per-step algorithmic bytes and FLOPs of the DeepSeek-V3 workloads,
+    counted by hand from the shapes: 1152 B per cached key read once per
+    sequence, W_uk + W_uv = 33.55 MB, 49,152 B of queries and 32,768 B of
+    outputs per query token, 278,528 FLOPs per visible (query, key) pair and
+    33.55 MFLOPs of projections per query token (+ W_dkv, x and the new rows
+    and 2 * 64 * 7168 * 576 FLOPs for the two appended tokens of 32
+    sequences)."""
+    W, QO, PAIR, PROJ = 33_554_432, 49_152 + 32_768, 278_528, 33_554_432
+    cases = {
+        "v3_b1_ctx8192": ([8192], 8192 * 1152 + W + QO, 8192 * PAIR + PROJ),
+        "v3_b4_ctx131072": ([131072] * 4, 4 * 131072 * 1152 + W + 4 * QO, 4 * 131072 * PAIR + 4 * PROJ),
+        # two causal queries per sequence see 4097 and 4098 keys
+        "v3_b32_append2": ([4098] * 32,
+                           32 * 4098 * 1152 + W + 7168 * 576 * 2 + 64 * 7168 * 2 + 64 * 576 * 2 + 64 * QO,
+                           32 * (4097 + 4098) * PAIR + 64 * PROJ + 2 * 64 * 7168 * 576),
+    }
+    for name, (lens, nbytes, flops) in cases.items():
+        r = RF.step_work(gen.WORKLOADS[name], lens)
+        assert r["bytes"] == nbytes, (name, r["bytes"], nbytes)
+        assert r["flops"] == flops, (name, r["flops"], flops)
+    # the rounded figures: 43.07 MB / 2.32 GFLOP, 637.9 MB / 146.2 GFLOP, 199.1 MB / 75.7 GFLOP
+    assert round(cases["v3_b1_ctx8192"][1] / 1e4) == 4307 and round(cases["v3_b32_append2"][2] / 1e8) == 757
+    assert RF.cache_bytes_per_token(512, 64, 2) == 1152
+    assert RF.cache_bytes_per_token(512, 64, 2, layers=61) == 70272
