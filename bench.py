@@ -266,6 +266,61 @@ def workload_config(w, host, world):
             "parallelism": f"dp{world} (independent sequence shards)"}
 
 
+# ----------------------------------------------------------------- end to end, overlapped
+L2_BYTES = 126e6        # B200 L2; steps reading more than this need no flush between them
+
+
+def e2e_pipelined(prob, h_in, h_outs, steps):
+    """End to end with the steps overlapped the way a serving loop overlaps
+    them: step k + 1's inputs are copied in (one copy stream) and step k - 1's
+    result read back (another) while step k computes (a third); inputs and the
+    result are double-buffered.  Every step's host-to-device and
+    device-to-host copies lie inside the timed region, which runs from the
+    first copy to the last read-back.  Returns milliseconds per step."""
+    res = "y" if prob.has_oproj else "out"
+    bufs = []
+    for k in range(2):
+        d = {n: getattr(prob, n) if k == 0 else torch.empty_like(getattr(prob, n)) for n in [*h_in, res]}
+        bufs.append(d)
+    up, comp, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    read_back = [torch.cuda.Event() for _ in range(2)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def copy_in(k):
+        with torch.cuda.stream(up):
+            if k >= 2:
+                up.wait_event(computed[k % 2])          # step k - 2 no longer reads these inputs
+            for n, h in h_in.items():
+                bufs[k % 2][n].copy_(h, non_blocking=True)
+            in_ready[k % 2].record(up)
+
+    torch.cuda.synchronize()
+    start.record(up)
+    copy_in(0)
+    for k in range(steps):
+        if k + 1 < steps:
+            copy_in(k + 1)
+        with torch.cuda.stream(comp):
+            comp.wait_event(in_ready[k % 2])
+            if k >= 2:
+                comp.wait_event(read_back[k % 2])       # step k - 2's result has been read back
+            for n, t in bufs[k % 2].items():
+                setattr(prob, n, t)
+            prob.step()
+            computed[k % 2].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[k % 2])
+            h_outs[k % 2].copy_(bufs[k % 2][res], non_blocking=True)
+            read_back[k % 2].record(down)
+    end.record(down)
+    end.synchronize()
+    for n, t in bufs[0].items():
+        setattr(prob, n, t)
+    return start.elapsed_time(end) / steps
+
+
 # ----------------------------------------------------------------- our arm
 def run_ours(a, rank, world, local):
     from mla_latent_kv_43_b200.runner import DeviceProblem
@@ -360,6 +415,23 @@ def run_ours(a, rank, world, local):
     if st != 0:
         raise RuntimeError(f"device status after timing: {B.STATUS.get(st, st)}")
 
+    # pass D: the same copies with consecutive steps overlapped (when a step reads
+    # more than L2 holds, so that no flush is needed between overlapped steps)
+    e2e_pipe_ms = None
+    # every rank takes the same branch (each has its own lengths): all must qualify
+    if max_over_ranks(0.0 if work["bytes"] > L2_BYTES else 1.0, world) == 0.0:
+        h_in = {"q_nope": h_qn, "q_rope": h_qr, "seq_lens": h_len}
+        if prob.has_append:
+            h_in["x"] = h_x
+        if prob.sparse:
+            h_in["sel"], h_in["n_sel"] = h_sel, h_nsel
+        h_outs = [h_out, torch.empty_like(h_out).pin_memory()]
+        barrier(world)
+        e2e_pipe_ms = max_over_ranks(e2e_pipelined(prob, h_in, h_outs, a.steps), world)
+        st = prob.get_status()
+        if st != 0:
+            raise RuntimeError(f"device status after the overlapped pass: {B.STATUS.get(st, st)}")
+
     clocks = sampler.summary(t0, t1) if sampler else None
     if sampler:
         sampler.stop()
@@ -415,9 +487,16 @@ def run_ours(a, rank, world, local):
         "roofline": roof,
         "kernels": kernels,
         "gpu_launches": launches,
-        "e2e": {"value": qtok / (e2e_ms / a.steps * 1e-3), "unit": "query-tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / a.steps},
+        "e2e": ({"value": qtok / (e2e_pipe_ms * 1e-3), "unit": "query-tokens/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_pipe_ms,
+                 "mode": "consecutive steps overlapped (copy in, compute, read back on three streams, "
+                         "double-buffered); no L2 flush: each step reads more than L2 holds"}
+                if e2e_pipe_ms is not None else
+                {"value": qtok / (e2e_ms / a.steps * 1e-3), "unit": "query-tokens/s",
+                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / a.steps,
+                 "mode": "one step at a time, L2 flushed before each"}),
+        "e2e_serial": {"value": qtok / (e2e_ms / a.steps * 1e-3), "unit": "query-tokens/s",
+                       "ms_per_step": e2e_ms / a.steps},
         "clocks": clocks,
     }
     if world == 1 and a.cpu_seconds > 0:
