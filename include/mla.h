@@ -1,5 +1,8 @@
 /*
- * mla.h -- C ABI of the MLA absorbed-decode library (libmla.so).
+ * mla.h -- C ABI of libmla.so: Multi-head Latent Attention against the
+ * compressed latent cache -- absorbed decode (dense and over a top-k
+ * selection), cache append, output projection, and prefill in the
+ * materialised factorisation.
  *
  * Multi-head Latent Attention caches, per token and layer, one 576-wide entry:
  * a 512-wide latent c_KV followed by a 64-wide rope key that is already
@@ -49,7 +52,7 @@ enum mla_status {
     MLA_OK = 0,
     MLA_ERR_ARG = 1,          /* null pointer, non-positive or odd size, bad dtype */
     MLA_ERR_ALIGN = 2,        /* a pointer the kernels load with TMA is not 16-byte aligned */
-    MLA_ERR_WORKSPACE = 3,    /* workspace_bytes below mla_decode_workspace_bytes() */
+    MLA_ERR_WORKSPACE = 3,    /* workspace_bytes below the call's size (mla_*_workspace_bytes) */
     MLA_ERR_UNSUPPORTED = 4,  /* a valid request the library does not implement */
     MLA_ERR_CUDA = 5,         /* a CUDA launch or API call failed */
     MLA_ERR_LEN = 6,          /* device: len_b < n_q, len_b > capacity or len_b > max_len */
@@ -203,8 +206,9 @@ MLA_API int mla_decode_sparse(const mla_dims* dims, int32_t batch, int32_t n_q,
  *   W_O     (device) [heads * v_dim][hidden], dims->dtype.
  *   y       (device) [tokens][hidden], dims->dtype; float accumulation, one rounding.
  *   status  (device) int32 status word.
- * bf16 runs a tcgen05 GEMM with K split over clusters of eight CTAs; fp32
- * (or a width that is not a multiple of 8) runs on CUDA cores.
+ * bf16 runs a tcgen05 GEMM with K split over a cluster of 2, 4 or 8 CTAs (the
+ * widest split whose grid runs in one wave); fp32 (or a width that is not a
+ * multiple of 8) runs on CUDA cores.
  * Errors: MLA_ERR_ARG (tokens < 0, hidden <= 0, a null pointer when tokens > 0),
  * MLA_ERR_ALIGN (a bf16 tensor-core operand not 16-byte aligned),
  * MLA_ERR_UNSUPPORTED (more than 65535 * 256 tokens on the tensor-core path);
@@ -220,11 +224,14 @@ MLA_API int mla_output_projection(const mla_dims* dims, int32_t tokens, int32_t 
  * 192-wide key [c W_uk[h] || k_rope] and the 128-wide value ("Understanding MLA",
  * sections "Reference code vs serving engines" and 6; "Multi-Head Latent
  * Attention", section 3).  The materialised rows live in the workspace.
- * Arguments as for mla_decode; workspace >= mla_prefill_workspace_bytes(),
- * 256-byte aligned.  bf16 with d_c 512, d_rope 64, qk_nope 128, v_dim 128 and
- * any head count; other dims return MLA_ERR_UNSUPPORTED, as do sizes whose
- * batch * n_q, heads * batch * max_len or batch * capacity reach 2^31.  A sequence with
- * a bad length sets MLA_ERR_LEN and gets zero outputs. */
+ * Arguments as for mla_decode (without splits); workspace >=
+ * mla_prefill_workspace_bytes(dims, batch, n_q, max_len), 256-byte aligned.
+ * bf16 with d_c 512, d_rope 64, qk_nope 128, v_dim 128 and any head count;
+ * other dims return MLA_ERR_UNSUPPORTED, as do sizes whose batch * n_q,
+ * heads * batch * max_len or batch * capacity reach 2^31.  Host errors as for
+ * mla_decode (MLA_ERR_ARG, MLA_ERR_WORKSPACE, MLA_ERR_ALIGN for q_nope, q_rope,
+ * W_uk, W_uv, cache or out not 16-byte aligned).  A sequence with a bad length
+ * sets MLA_ERR_LEN and gets zero outputs. */
 MLA_API size_t mla_prefill_workspace_bytes(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len);
 MLA_API int mla_prefill(const mla_dims* dims, int32_t batch, int32_t n_q, const void* q_nope, const void* q_rope,
                         const void* W_uk, const void* W_uv, const void* cache, int64_t capacity,
