@@ -140,6 +140,11 @@ def shard_workload(w, rank: int):
     return w.with_(seed=w.seed + 1000 * rank) if rank else w
 
 
+def all_ranks(flag: bool, world: int, device="cuda") -> bool:
+    """True on every rank when the flag holds on every rank (one collective)."""
+    return max_over_ranks(0.0 if flag else 1.0, world, device) == 0.0
+
+
 def job_throughput(query_tokens_per_rank: int, world: int, ms_per_step_max: float) -> float:
     """Whole-job query tokens per second: every rank's tokens over the slowest rank's time."""
     return query_tokens_per_rank * world / (ms_per_step_max * 1e-3)
@@ -419,7 +424,7 @@ def run_ours(a, rank, world, local):
     # more than L2 holds, so that no flush is needed between overlapped steps)
     e2e_pipe_ms = None
     # every rank takes the same branch (each has its own lengths): all must qualify
-    if max_over_ranks(0.0 if work["bytes"] > L2_BYTES else 1.0, world) == 0.0:
+    if all_ranks(work["bytes"] > L2_BYTES, world):
         h_in = {"q_nope": h_qn, "q_rope": h_qr, "seq_lens": h_len}
         if prob.has_append:
             h_in["x"] = h_x

@@ -1,6 +1,7 @@
 """The multi-rank host logic of the benchmark on CPU: two gloo ranks, each with
 its own shard of sequences, agree on the slowest rank's time and on the
-whole-job throughput (weak scaling, no collective on the data path)."""
+whole-job throughput (weak scaling, no collective on the data path), and take
+a collective branch together when only one of them qualifies."""
 import os
 import socket
 import sys
@@ -35,7 +36,10 @@ def _rank_main(rank, world, port, out):
         csum = torch.tensor([float(host["q_nope"].double().sum())])
         allc = [torch.zeros(1) for _ in range(world)]
         dist.all_gather(allc, csum)
-        out[rank] = (slowest, value, shard.seed, [float(c) for c in allc])
+        # a branch every rank must take together: taken only when all ranks qualify
+        mixed = bench.all_ranks(rank == 0, world, device="cpu")
+        both = bench.all_ranks(True, world, device="cpu")
+        out[rank] = (slowest, value, shard.seed, [float(c) for c in allc], mixed, both)
     finally:
         dist.destroy_process_group()
 
@@ -45,8 +49,9 @@ def test_two_gloo_ranks_shard_and_reduce():
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
-    (s0, v0, seed0, c0), (s1, v1, seed1, c1) = out[0], out[1]
+    (s0, v0, seed0, c0, m0, b0), (s1, v1, seed1, c1, m1, b1) = out[0], out[1]
     assert s0 == s1 == 2.0                        # max over ranks
     assert v0 == v1 == 2 * 2 / 2e-3               # 2 query tokens per rank, 2 ranks, 2 ms
     assert seed0 != seed1                         # distinct shards
     assert c0 == c1 and c0[0] != c0[1]            # the shards' inputs differ
+    assert (m0, m1, b0, b1) == (False, False, True, True)
