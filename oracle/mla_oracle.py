@@ -13,7 +13,7 @@ What it computes, and where each step is stated:
   step B2) and of the query's rope half at the query's own position
   (Phase C, step C2).  The pair layout and base are not fixed by the pages;
   this oracle takes interleaved pairs (x[2i], x[2i+1]) rotated by
-  pos * base^(-2i/d_R), base 10000 (the stated reading of the build).
+  pos * base^(-2i/d_R), base 10000 (a reading: the pages leave it open).
 * Concatenation Q = [Q_nope || Q_rope], K = [K_nope || K_rope] and
   softmax(Q K^T / sqrt(qk_nope + d_R)) V (Phase D, steps D1-D2;
   "Multi-Head Latent Attention", section 3, the sketch's last two lines).
