@@ -195,3 +195,22 @@ def test_prefill_argument_checks():
     d = ctypes.byref(v3())
     need = L.mla_prefill_workspace_bytes(d, 2, 4, 100)
     assert need >= 2 * 4 * 128 * 64 * 2 + 2 * (2 * 100 * 128 * 128 * 2)
+
+
+def test_header_is_c_and_links_from_c(tmp_path):
+    """include/mla.h compiles as C99 and libmla.so links and answers from a C
+    program (host-checkable calls only: sizes, argument errors, strings)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    lib_dir = os.path.dirname(B.LIB_PATH)
+    exe = str(tmp_path / "abi_check")
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "abi_check.c"), "-L", lib_dir, "-lmla", f"-Wl,-rpath,{lib_dir}", "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAIL" not in r.stdout and r.stdout.count("ok ") == 11, r.stdout
