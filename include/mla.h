@@ -266,7 +266,15 @@ MLA_API int mla_selftest_wait_timeout(int32_t* status, int64_t limit_ns, void* s
  * exceed it returns MLA_ERR_WORKSPACE; pass a small `splits` (for example 4)
  * to fit larger batches, since split-KV partial results dominate the size.
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current).  With CUDA's lazy module loading that lookup is also
+ * what loads the library's device code on that device and reserves the
+ * array, and it may synchronise the device: make the first call during
+ * set-up, before any stream capture.  The address is cached per device for
+ * the life of the process; it is no longer valid after the device is reset
+ * (cudaDeviceReset), so do not call this entry point again after a reset.
+ * Argument checks and their order are mla_decode's (an empty problem returns
+ * MLA_OK without touching the device); a call that returns an error
+ * enqueued nothing and mla_last_launch_count then reports 0.
  * All calls share the one array and it keeps the last call's contents (no
  * region needs clearing: each is written before it is read), so calls whose
  * execution overlaps on the GPU -- on different streams, or from different

@@ -85,6 +85,10 @@ int generic_gemm_xw(mla_dtype dtype, const void* x, const void* W, int M, int K,
 // RMSNorm of the latent of every appended row (after either append kernel).
 int rms_norm_rows(const AppendCall& c, int* launches);
 
+// Sets the count mla_last_launch_count reports to 0 (for an entry point that
+// returns before enqueuing anything).
+void clear_last_launch_count();
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // RoPE pair frequencies theta_i = base^(-2i/d_rope), i < d_rope / 2, as

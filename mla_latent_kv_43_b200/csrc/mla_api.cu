@@ -43,6 +43,8 @@ int layout_for(const mla_dims* dims, int32_t batch, int32_t n_q, int64_t max_len
 
 namespace mla {
 
+void clear_last_launch_count() { g_last_launches = 0; }
+
 void rope_turn_table(float base, int d_rope, uint64_t* turn) {
     const long double two_pi = 6.283185307179586476925286766559005768L;
     for (int i = 0; i < d_rope / 2; ++i) {

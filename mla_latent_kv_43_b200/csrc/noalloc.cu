@@ -6,6 +6,7 @@
 
 #include <mutex>
 
+#include "internal.h"
 #include "mla.h"
 
 namespace {
@@ -39,13 +40,21 @@ extern "C" int mla_decode_noalloc(const mla_dims* dims, int32_t batch, int32_t n
                                   const void* q_rope, const void* W_uk, const void* W_uv, const void* cache,
                                   int64_t capacity, const int32_t* seq_lens, int64_t max_len, void* out,
                                   int32_t splits, int32_t* status, void* stream) {
-    if (batch == 0 || n_q == 0) return MLA_OK;
+    // The layout call checks dims and sizes exactly as mla_decode does.
     mla_ws_layout L;
-    const int rc = mla_decode_workspace_layout(dims, batch, n_q, max_len, splits, &L);
-    if (rc != MLA_OK) return rc;
-    if (L.total > kScratchBytes) return MLA_ERR_WORKSPACE;
+    int rc = mla_decode_workspace_layout(dims, batch, n_q, max_len, splits, &L);
+    if (rc == MLA_OK && (batch == 0 || n_q == 0)) {
+        // the empty problem: mla_decode's own answer, without touching the device
+        return mla_decode(dims, batch, n_q, q_nope, q_rope, W_uk, W_uv, cache, capacity, seq_lens, max_len, out,
+                          nullptr, 0, splits, status, stream);
+    }
+    if (rc == MLA_OK && L.total > kScratchBytes) rc = MLA_ERR_WORKSPACE;
     void* scratch = nullptr;
-    if (scratch_address(&scratch) != MLA_OK) return MLA_ERR_CUDA;
+    if (rc == MLA_OK && scratch_address(&scratch) != MLA_OK) rc = MLA_ERR_CUDA;
+    if (rc != MLA_OK) {
+        mla::clear_last_launch_count();     // nothing was enqueued by this call
+        return rc;
+    }
     // Every region of the workspace is written before it is read within one
     // call, so nothing left by an earlier call needs clearing.
     return mla_decode(dims, batch, n_q, q_nope, q_rope, W_uk, W_uv, cache, capacity, seq_lens, max_len, out, scratch,

@@ -177,6 +177,10 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     // softmax: the running row maximum after tile g (slot g & 1) and its
     // per-quarter barriers; per-item meeting of the two groups' row sums
     __shared__ uint64_t m_ready[2][4], ep_ready[4];
+    // ep_done: both groups' warps of a lane quarter have read their half of O
+    // (the next item's first value GEMM overwrites it); item_done: the item's
+    // last value GEMM has completed (one completion per item)
+    __shared__ uint64_t ep_done[4], item_done;
     __shared__ float m_pub[2][128];
     __shared__ float ep_m[2][2][128], ep_l[2][2][128];
     __shared__ __align__(16) uint32_t ep_scratch[8][32 * 16];   // per softmax warp: 32 rows x 64 bytes
@@ -207,7 +211,9 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             mbar_init(&m_ready[0][i], 1);   // warp of lane quarter i in the group of an even tile
             mbar_init(&m_ready[1][i], 1);   // ... of an odd tile
             mbar_init(&ep_ready[i], 2);     // the two groups' warps of lane quarter i, once per item
+            mbar_init(&ep_done[i], 2);      // ... after their epilogue reads of O, once per item
         }
+        mbar_init(&item_done, 1);           // committed after each item's last O GEMM
         mbar_init(&drain, 1);
         abort_flag = 0;
         fence_mbar_init();
@@ -338,6 +344,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 mma_commit_mc_w(&rx_done[gO % kXBufs], (uint16_t)(1u << peer));
                 ++gO;
                 if (++kO == itO.t1 - itO.t0) {
+                    mma_commit_w(&item_done);
                     kO = 0;
                     haveO = iterO.next(itO);
                 }
@@ -497,9 +504,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         const int gtid = (warp - 6 - 4 * grp) * 32 + lane;   // 0..127 within the group
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const bool xleader = (warp == 6 + 4 * grp) && lane == 0;   // the expect_tx of this group's tiles
-        // O GEMM of global tile n has completed.  Completions alternate between two
-        // barriers; the next completion on o_done[n & 1] (tile n + 2) needs a P tile
-        // that cannot have been written when this is called, so the parity is exact.
+        // O GEMM of global tile n = g - 1 has completed (the rescale before P of tile
+        // g).  Completions alternate between two barriers, so the parity is exact
+        // only if O(g - 3) is done and O(g + 1) is not: the peer's partial scores of
+        // tile g (waited for above) are sent only after this CTA's O GEMM of tile
+        // g - 3 released that exchange buffer, and O(g + 1) follows O(g), which
+        // needs the P tile this thread has yet to write.
         // Exchange buffer g % 3 holds the peer's partial scores of tile g, then this
         // CTA's P tile g (each thread overwrites exactly the chunks it read); the
         // commit of O GEMM g hands it back to the peer (for its tile g + 3).
@@ -640,7 +650,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             // epilogue: both groups' sums meet; group c writes O columns [128c, 128c + 128)
             // of this CTA's latent half (normalised, or a partial plus log2-sum-exp)
             bool ok = true;
-            if (lane == 0) ok = wait_o(it + T - 1);
+            if (lane == 0) ok = mbar_wait(&item_done, n_item & 1, abort);
             if (!lane0(ok)) break;
             const int eb = n_item & 1;
             ep_m[eb][grp][h] = m_used;
@@ -694,7 +704,15 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 }
                 if (item.slot >= 0 && rank == 0 && grp == 0) a.part_lse[item.slot * 128 + h] = mf + __log2f(lsum);
             }
+            // the next item's first O GEMM (accumulate = 0) may start only after both
+            // groups' reads of this item's O
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&ep_done[q]);
+                ok = mbar_wait(&ep_done[q], n_item & 1, abort);
+            }
+            if (!lane0(ok)) break;
             it += T;
             ++n_item;
         }

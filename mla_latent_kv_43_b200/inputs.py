@@ -213,3 +213,47 @@ def tiny(dtype: str = "fp32", *, batch=None, heads=3, d_c=8, d_rope=4, qk_nope=6
                     lens=tuple(lens), capacity=cap, latent_rms_norm=latent_rms_norm,
                     hidden=hidden, n_new=n_new, top_k=top_k, hidden_out=hidden_out, prefill=prefill,
                     seed=seed)
+
+
+def sharpen(host: Dict[str, torch.Tensor], *, gain: int = 4, late=None, late_gain: int = 2,
+            dominant=None, dominant_gain: int = 4, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Reshape generated inputs into a large-score, peaky-softmax case.
+
+    * ``W_uk[h]`` becomes a signed selection times ``gain``: latent row i of
+      head h holds +-gain at one q_nope column (a seeded permutation, every
+      column used d_c / qk_nope times) and zeros elsewhere, so each absorbed
+      query entry is +-gain times one stored q_nope value -- exactly
+      representable in the storage dtype when ``gain`` is a power of two;
+    * ``q_rope`` is multiplied by ``gain``;
+    * the cache rows ``late[b] = (lo, hi)`` of sequence b (latent and raw rope
+      key) are multiplied by ``late_gain``, and row ``dominant[b]`` by
+      ``dominant_gain``.
+
+    With power-of-two gains every reshaped value is the stored value times a
+    power of two, so no rounding is added.  Returns a new dict; ``host`` is
+    left unchanged.
+    """
+    for g in (gain, late_gain, dominant_gain):
+        assert g > 0 and (g & (g - 1)) == 0, "gains must be powers of two"
+    out = dict(host)
+    H, d_c, qk = host["W_uk"].shape
+    assert d_c % qk == 0
+    rng = np.random.default_rng(seed)
+    W = np.zeros((H, d_c, qk), dtype=np.float32)
+    for h in range(H):
+        cols = rng.permutation(np.repeat(np.arange(qk), d_c // qk))
+        signs = rng.choice(np.array([-1.0, 1.0], dtype=np.float32), size=d_c)
+        W[h, np.arange(d_c), cols] = signs * gain
+    out["W_uk"] = _cast(W, host["W_uk"].dtype)
+    out["q_rope"] = host["q_rope"] * gain
+    c, kr = host["c_kv"].clone(), host["k_rope"].clone()
+    for b in range(c.shape[0]):
+        if late is not None and late[b] is not None:
+            lo, hi = late[b]
+            c[b, lo:hi] *= late_gain
+            kr[b, lo:hi] *= late_gain
+        if dominant is not None and dominant[b] is not None:
+            c[b, dominant[b]] *= dominant_gain
+            kr[b, dominant[b]] *= dominant_gain
+    out["c_kv"], out["k_rope"] = c, kr
+    return out

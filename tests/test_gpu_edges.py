@@ -131,3 +131,69 @@ def test_rope_kernel_matches_oracle(dtype):
     assert np.array_equal(got[:, :16], xt.double().numpy()[:, :16])
     tol = 2e-6 if dtype == "fp32" else 8e-3
     assert rel_err(got[:, 16:], ref) <= tol
+
+
+def _scaled_scores(w, host, b, h):
+    """Scaled scores of query (b, last) head h against its visible keys (fp64,
+    from the oracle's absorbed query and rotated cache keys)."""
+    L = int(host["seq_lens"][b])
+    p = L - w.n_q + (w.n_q - 1)
+    q = O.absorbed_query(host["q_nope"][b, -1, h].double().numpy(), host["q_rope"][b, -1, h].double().numpy(),
+                         host["W_uk"][h].double().numpy(), p, w.rope_base)
+    k_rot = O.rope_cache(host["k_rope"][b:b + 1, :L].double().numpy(), [L], w.rope_base)[0]
+    K = np.concatenate([host["c_kv"][b, :L].double().numpy(), k_rot], axis=1)
+    return (K @ q) * w.softmax_scale
+
+
+def test_large_logits_peaky_softmax_many_pieces():
+    """Tensor-core path with scaled scores spanning more than +-40, a handful of
+    keys holding most of each head's softmax weight, a row maximum that grows
+    by more than 2^8 (base 2) late in the sequence, and each sequence cut into
+    many split-KV pieces, every (batch, head) row compared at the bf16 bar.
+    The absorbed query is exactly representable in bf16 (a signed selection
+    of q_nope times a power of two), so the comparison measures the kernel's
+    own arithmetic rather than the rounding of the query, whose effect grows
+    with the score magnitude for any bf16-operand kernel.  ("Understanding
+    MLA", Phase D step D2: softmax(Q K^T / sqrt(192)) V.)"""
+    lens = (8192, 2600)
+    w, host = make("bf16_v3", lens=lens, capacity=8192, seed=11)
+    late = [(lens[0] - 700, lens[0] - 600), (lens[1] - 300, lens[1] - 200)]
+    host = gen.sharpen(host, gain=4, late=late, late_gain=2, dominant=[1000, 100], dominant_gain=4, seed=12)
+    # the inputs are what the docstring says (checked on a few heads, fp64)
+    grew, span = 0, 0.0
+    for h in (0, 37, 64, 90):
+        s = _scaled_scores(w, host, 0, h)
+        span = max(span, float(np.abs(s).max()))
+        wts = np.exp(s - s.max())
+        wts /= wts.sum()
+        assert np.sort(wts)[-8:].sum() > 0.5
+        l2 = s * np.log2(np.e)
+        grew += l2[late[0][0]:].max() > l2[: late[0][0]].max() + 8
+    assert span > 40 and grew >= 1, (span, grew)
+    splits = 48
+    prob = DeviceProblem(w, host, splits=splits)
+    assert prob.layout["splits"] == splits
+    prob.step()
+    torch.cuda.synchronize()
+    assert prob.get_status() == 0
+    got = gpu_out(prob)
+    assert np.isfinite(got).all()
+    ref = oracle_out(w, host)
+    err = rel_err(got, ref)
+    print(f"large logits: max|d|/max|ref| = {err:.3e}")
+    assert err <= TOL["bf16"], err
+
+
+def test_one_sequence_in_74_pieces():
+    """One 32768-key sequence cut into 74 split-KV pieces (one per cluster of
+    the B200's 148 SMs): the log-sum-exp merge of many pieces per token."""
+    w, host = make("bf16_v3", lens=(32768,), capacity=32768, seed=13)
+    prob = DeviceProblem(w, host, splits=74)
+    assert prob.layout["splits"] == 74
+    prob.step()
+    torch.cuda.synchronize()
+    assert prob.get_status() == 0
+    hs = list(range(0, 128, 8))
+    ref = oracle_out(w, host, batches=[0], heads=hs)
+    err = rel_err(sampled(gpu_out(prob), [0], hs), sampled(ref, [0], hs))
+    assert err <= TOL["bf16"], err

@@ -1,7 +1,8 @@
 """CUDA path against the fp64 oracle on the five workloads and the top-k
-sparse workload (same seeded
-inputs; full outputs where the oracle is quick, sampled (batch, head)
-outputs at full size, in the launch configuration the benchmark times)."""
+sparse workload (same seeded inputs, in the launch configuration the
+benchmark times).  Every (batch, head) output row is compared for the tiny
+workload, the batched headline workload and the append workload; the
+single-sequence and top-k workloads compare sampled (batch, head) rows."""
 import os
 import sys
 
@@ -20,9 +21,9 @@ pytestmark = pytest.mark.gpu
 CASES = [
     ("tiny_fp32", None, None),
     ("v3_b1_ctx8192", [0], list(range(0, 128, 4))),
-    ("v3_b64_ragged", [0, 9, 17, 33, 48, 63], [0, 5, 77, 127]),
+    ("v3_b64_ragged", None, None),
     ("v3_b4_ctx131072", [0, 3], [0, 64, 127]),
-    ("v3_b32_append2", [0, 13, 31], [0, 33, 100]),
+    ("v3_b32_append2", None, None),
     ("v3_b32_topk2048", [0, 17, 31], [0, 64, 127]),
 ]
 
