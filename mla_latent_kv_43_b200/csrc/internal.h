@@ -38,6 +38,10 @@ struct AppendCall {
     cudaStream_t stream;
 };
 
+// Dense tensor-core decode: the CTA-pair attention kernel over 128-key tiles
+// (true) or the single-CTA-pair latent-split kernel over 64-key tiles (false).
+constexpr bool kDecodePairKernel = false;
+
 // True when the tensor-core path serves these dims: bf16 with the
 // DeepSeek-V3 head geometry (128 heads, latent 512, rope 64, nope 128, value 128).
 bool sm100_decode_supported(const mla_dims& d);

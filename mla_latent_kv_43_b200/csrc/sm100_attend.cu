@@ -290,9 +290,8 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                                         rows[4 * g4 + 1], rows[4 * g4 + 2], rows[4 * g4 + 3]);
                         }
                     } else {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            tma_load_3d(st + i * kLatBox, &map_lat, &full[s], 256 * rank + 64 * i, key0, b);
+                        // this CTA's four latent column groups in one copy (see launch_attend)
+                        tma_load_4d(st, &map_lat, &full[s], 0, key0, 4 * (int)rank, b);
                         tma_load_3d(st + 4 * kLatBox, &map_rope, &full[s], 512 + 32 * rank, key0, b);
                     }
                 }
@@ -741,10 +740,18 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
         if (!make_map(&ml, c.cache, 2, dims, str, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
         if (!make_map(&mr, c.cache, 2, dims, str, box_r, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
     } else {
+        // latent: rows viewed as 9 groups of 64 columns (group stride 128 bytes,
+        // placed after the key dimension), one box = 64 keys x 4 groups landing
+        // group-major: a whole latent half per tensor copy.  A single thread
+        // issues about one tensor copy per 0.3 us whatever its size up to 16 KB,
+        // so one copy instead of four keeps the loads at HBM speed.
+        const uint64_t dl[4] = {64, (uint64_t)c.capacity, 9, (uint64_t)c.batch};
+        const uint64_t sl[3] = {576 * 2, 64 * 2, (uint64_t)c.capacity * 576 * 2};
+        const uint32_t box_l[4] = {64, 64, 4, 1};
+        if (!make_map(&ml, c.cache, 4, dl, sl, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
         const uint64_t dims[3] = {576, (uint64_t)c.capacity, (uint64_t)c.batch};
         const uint64_t str[2] = {576 * 2, (uint64_t)c.capacity * 576 * 2};
-        const uint32_t box_l[3] = {64, 64, 1}, box_r[3] = {32, 64, 1};
-        if (!make_map(&ml, c.cache, 3, dims, str, box_l, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        const uint32_t box_r[3] = {32, 64, 1};
         if (!make_map(&mr, c.cache, 3, dims, str, box_r, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
     }
     AttnArgs a{};

@@ -1,0 +1,691 @@
+// Absorbed MLA attention against the latent cache on a CTA pair
+// (tcgen05 cta_group::2): the dense decode's core kernel.
+//
+// For one query token (b, j) and a range of 128-key tiles of its sequence,
+// with q_lat = [W_uk q_nope || RoPE(q_rope)] (576 wide, all 128 heads):
+//     S[h][n] = <q_lat[h], cache[b][n][0:576]>                    (score)
+//     online softmax over n (base 2, scale folded in), fp32 state
+//     O[h][0:512] += P[h][n] cache[b][n][0:512]                    (weighted latent)
+// i.e. the score of "Understanding MLA (Multi-head Latent Attention)",
+// section 4 (content part through the absorbed query, position part through
+// the shared rope key), weighted over the cached latents as on aicassindra
+// "Multi-head latent attention", "End-to-end flow".
+//
+// Work split.  A cluster of two CTAs on two SMs is one MMA unit.  All 128
+// heads of a token are the M dimension of both contractions, split 64 / 64:
+// CTA r holds the query rows and the softmax of heads [64r, 64r + 64).
+//  * Score GEMM (M 128 heads, N 128 keys, K 576): CTA r stages keys
+//    [64r, 64r + 64) of the tile, all 576 columns; each CTA's S holds its 64
+//    heads against all 128 keys -- complete scores, no partial sums to
+//    exchange.
+//  * Value GEMM (M 128 heads, N 256 latent columns, twice, K 128 keys): CTA r
+//    stages latent columns [128r, 128r + 128) and [256 + 128r, 256 + 128r +
+//    128) of all 128 keys.  These are re-read from L2 (the score stage of the
+//    same tile brought them there from HBM a tile period earlier), so each
+//    cache byte crosses HBM once; no load is multicast.
+// Each CTA keeps its 64 heads x 512 latent fp32 O in TMEM.
+//
+// TMEM per CTA (512 columns): O [0, 256), S double buffer [256, 320) and
+// [320, 384).  In the pair layout (M = 128 over two CTAs) a CTA's 64 rows
+// fill all 128 lanes: lane i and lane i + 64 both hold row i, the first and
+// the second half of the N columns.
+//
+// Shared memory per CTA: the query rows (9 groups of 64 columns x 64 rows,
+// 72 KB), two P buffers (64 heads x 128 keys bf16), a ring of key units (3
+// column groups x 64 keys, 24 KB) for the score GEMM and a ring of value
+// units (2 column groups x 64 keys, 16 KB) for the value GEMM.  Every staged
+// unit arrives in ONE tensor copy: the maps view a cache row as 9 groups of
+// 64 columns (a dimension of stride 128 bytes placed after the key
+// dimension), so a box of several groups lands as consecutive 8 KB
+// group-major blocks, the layout both GEMMs read.  (A single thread issues
+// about one tensor copy per 0.3 us whatever its size up to 16 KB, so fewer,
+// larger copies are what keeps the loads at HBM speed.)
+//
+// Roles (256 threads): warp 0 key / query loads, warp 1 MMA issue (even CTA;
+// TMEM allocation in both), warp 2 value loads (and the zeroing of value rows
+// past the visible keys), warps 4-7 softmax and epilogue (thread t <-> TMEM
+// lane t: head 64r + t % 64, key / column half t / 64).
+//
+// Work items as in the single-CTA kernel: the 128-key tiles of all query
+// tokens are concatenated and cut into one contiguous range per pair.  A
+// token whose tiles all fall in one pair's range is finished there
+// (normalised latent output, bf16); a token cut across pairs leaves partial
+// outputs plus log2-sum-exp per piece for the merge before the up-projection.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "profile.h"
+#include "sm100_host.h"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace sm100 {
+
+namespace {
+
+constexpr int kKeys = 128;                   // keys per tile (the pair)
+constexpr int kBox = 8192;                   // one column group of 64 rows
+constexpr int kQBoxes = 9;                   // 576 / 64 column groups
+constexpr int kKU = 3;                       // column groups per key unit
+constexpr int kKUnits = kQBoxes / kKU;       // key units per tile
+constexpr int kKS = 3;                       // key-unit ring slots
+constexpr int kVS = 3;                       // value-unit ring slots
+constexpr int kVUnits = 4;                   // value units per tile: 2 latent halves x 2 key halves
+constexpr int kOffQ = 0;
+constexpr int kOffP = kOffQ + kQBoxes * kBox;         // 2 buffers x 2 boxes (64 keys each)
+constexpr int kOffK = kOffP + 4 * kBox;
+constexpr int kOffV = kOffK + kKS * kKU * kBox;
+constexpr int kSmemBytes = kOffV + kVS * 2 * kBox;
+constexpr int kThreads = 256;
+constexpr uint32_t kColO = 0, kColS = 256, kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// value units of tile g may be fetched once the first key unit of tile g + 1
+// has been requested (tile g's latent columns are then in L2)
+constexpr int kVLagUnits = 1;
+
+struct PairArgs {
+    const __nv_bfloat16* q_lat;   // [BJ][128][576]
+    const int32_t* cum;           // [BJ + 1] 128-key tile prefix
+    const int32_t* first_bj;      // [pairs] first query token of each pair's range
+    const int32_t* seq_lens;
+    int BJ, n_q, pairs;
+    float scale_log2;             // softmax_scale * log2(e)
+    __nv_bfloat16* o_lat;         // [BJ][128][512]
+    __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
+    float* part_lse;              // [2 * pairs][128], log2 domain
+    int32_t* status;
+};
+
+struct Item {
+    int bj, t0, t1, n_vis, slot;  // slot < 0: finished here; n_vis: keys this token attends
+};
+
+// Pieces of the concatenated tile range [s0, s1) of one pair, in order.
+struct ItemIter {
+    const int32_t* cum;
+    const int32_t* lens;
+    int BJ, n_q, bj, s0, s1, pair;
+    __device__ void init(const PairArgs& a, int p) {
+        cum = a.cum;
+        BJ = a.BJ;
+        n_q = a.n_q;
+        lens = a.seq_lens;
+        pair = p;
+        const int T = cum[BJ];
+        s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
+        s1 = (int)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
+        bj = a.first_bj[p];
+    }
+    __device__ bool next(Item& it) {
+        while (bj < BJ) {
+            const int c0 = cum[bj], c1 = cum[bj + 1];
+            if (c0 >= s1) return false;
+            const int cur = bj++;
+            if (c1 == c0) continue;
+            const int lo = max(c0, s0), hi = min(c1, s1);
+            if (hi <= lo) continue;
+            it.bj = cur;
+            it.t0 = lo - c0;
+            it.t1 = hi - c0;
+            const int b = cur / n_q, j = cur % n_q;
+            it.n_vis = (int)query_pos(lens[b], n_q, j) + 1;
+            it.slot = (c0 >= s0 && c1 <= s1) ? -1 : (c0 < s0 ? 2 * pair : 2 * pair + 1);
+            return true;
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, PairArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // waited on by the even CTA's MMA warp (arrivals and bytes from both CTAs)
+    __shared__ uint64_t kfull[kKS], vready[kVS], qfull, sfree[2], pfull[2], ep_done;
+    // completed by the pair's MMA commits in both CTAs, or local
+    __shared__ uint64_t kempty[kKS], vempty[kVS], vland[kVS], qempty, sfull[2], pfree[2], o_done[2], item_done,
+        drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+    __shared__ int k_issued;                  // key units this CTA has requested (value-load pacing)
+    __shared__ float xch[2][128];             // partner exchange of the softmax (row max, row sum)
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kKS; ++s) {
+            mbar_init(&kfull[s], 1);          // the even CTA's expect_tx; bytes of both CTAs
+            mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < kVS; ++s) {
+            mbar_init(&vready[s], 2);         // each CTA's value loader, after landing (and zeroing)
+            mbar_init(&vempty[s], 1);
+            mbar_init(&vland[s], 1);
+        }
+        mbar_init(&qfull, 1);
+        mbar_init(&qempty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfree[i], 2);          // each CTA's softmax has read S
+            mbar_init(&pfull[i], 2);          // each CTA's softmax has written P
+            mbar_init(&sfull[i], 1);
+            mbar_init(&pfree[i], 1);
+            mbar_init(&o_done[i], 1);
+        }
+        mbar_init(&ep_done, 2);               // each CTA's epilogue has read O
+        mbar_init(&item_done, 1);
+        mbar_init(&drain, 1);
+        abort_flag = 0;
+        k_issued = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();          // both CTAs' barriers are initialised before any remote access
+    tc_fence_after();
+    grid_dep_wait();         // q_lat and the tile plan come from the previous kernel
+    grid_dep_trigger();
+    const uint32_t tmem = tmem_base;
+    const uint32_t sbase = smem_u32(smem);
+    volatile int* abort = &abort_flag;
+    volatile int* kiss = &k_issued;
+    auto fail = [&]() {
+        *abort = 1;
+        set_status(a.status, MLA_ERR_TIMEOUT);
+    };
+    // barriers of the even CTA, as shared::cluster addresses
+    auto lead = [&](uint64_t* bar) { return map_peer(smem_u32(bar), 0); };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ query and key loads
+        if (elect_one()) {
+            tma_prefetch(&map_q);
+            tma_prefetch(&map_k);
+            ItemIter iter;
+            iter.init(a, pair);
+            Item item;
+            uint32_t kc = 0, n = 0;
+            bool ok = true;
+            while (ok && iter.next(item)) {
+                const int b = item.bj / a.n_q;
+                // the query rows of this item once every score GEMM of the previous one is done
+                if (n > 0 && !mbar_wait(&qempty, (n - 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                if (rank == 0) mbar_expect_tx(&qfull, 2 * kQBoxes * kBox);
+                tma_load_3d_pair(smem + kOffQ, &map_q, lead(&qfull), 0, item.bj * 128 + 64 * (int)rank, 0);
+                for (int t = item.t0; t < item.t1 && ok; ++t) {
+                    const int key0 = t * kKeys + 64 * (int)rank;
+                    for (int u = 0; u < kKUnits; ++u, ++kc) {
+                        const int s = kc % kKS;
+                        if (kc >= (uint32_t)kKS && !mbar_wait(&kempty[s], ((kc / kKS) - 1) & 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        if (rank == 0) mbar_expect_tx(&kfull[s], 2 * kKU * kBox);
+                        tma_load_4d_pair(smem + kOffK + s * kKU * kBox, &map_k, lead(&kfull[s]), 0, key0, kKU * u, b);
+                        *kiss = (int)kc + 1;
+                    }
+                }
+                ++n;
+            }
+            *kiss = 0x7fffffff;               // no more key chunks: value loads need not wait
+            if (!ok) fail();
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue (even CTA)
+        // Two streams in tile order, advanced one staged unit at a time: score
+        // GEMMs S(g) (3 key units of 3 column groups, 4 K-steps per group) and
+        // value GEMMs O(g) (4 value units, 4 K-steps each).  The whole warp runs the loop (decisions are
+        // lane 0's observations, broadcast); one elected lane issues.
+        if (rank == 0) {
+            constexpr uint32_t idS = idesc_bf16(128, kKeys, false, false);
+            constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
+            const uint64_t dQ = sdesc(sbase + kOffQ, 16, 1024, kSwizzle128);     // query rows, K-major
+            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);     // key chunk, K-major
+            const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);     // P rows, K-major
+            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);   // value unit, MN-major
+            ItemIter iterS, iterO;
+            iterS.init(a, pair);
+            iterO.init(a, pair);
+            Item itS, itO;
+            bool haveS = iterS.next(itS), haveO = iterO.next(itO);
+            int kS = 0, kO = 0;                    // tile index within the current item
+            uint32_t gS = 0, gO = 0;               // global tile counters
+            uint32_t cS = 0, cO = 0;               // chunk within the current tile
+            uint32_t kc = 0, vc = 0;               // ring chunk counters
+            uint32_t nS = 0, nO = 0;               // item counters
+            bool qS = false;                       // query rows of the current S item landed
+            uint32_t idle = 0;
+            uint64_t t_idle = 0;
+            bool ok = true;
+            while (ok && haveO) {
+                bool progressed = false;
+                // value chunk of O(gO): needs P(gO) from both CTAs, its value chunk in both,
+                // and (first tile of an item after the first) both epilogues done with O
+                if (gO < gS) {
+                    bool ready = true;
+                    if (cO == 0) {
+                        ready = mbar_ready_cluster_w(&pfull[gO & 1], (gO >> 1) & 1) &&
+                                (kO != 0 || nO == 0 || mbar_ready_cluster_w(&ep_done, (nO - 1) & 1));
+                    }
+                    const int vs = vc % kVS;
+                    if (ready && mbar_ready_cluster_w(&vready[vs], (vc / kVS) & 1)) {
+                        tc_fence_after();
+                        const int half = cO >> 1, kh = cO & 1;               // latent half, key half
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint32_t pa = (gO & 1) * 2 * kBox + kh * kBox + ks * 32;
+                            mma_pair_ss_w(tmem + kColO + 128 * half, sdesc_add(dP, pa),
+                                          sdesc_add(dV, vs * 2 * kBox + ks * 2048), idO,
+                                          (kO == 0 && kh == 0 && ks == 0) ? 0u : 1u);
+                        }
+                        mma_commit_pair_w(&vempty[vs]);
+                        ++vc;
+                        if (++cO == kVUnits) {
+                            cO = 0;
+                            mma_commit_pair_w(&pfree[gO & 1]);
+                            mma_commit_pair_w(&o_done[gO & 1]);
+                            ++gO;
+                            if (++kO == itO.t1 - itO.t0) {
+                                mma_commit_pair_w(&item_done);
+                                kO = 0;
+                                ++nO;
+                                haveO = iterO.next(itO);
+                            }
+                        }
+                        progressed = true;
+                    }
+                }
+                // key chunk of S(gS): needs the item's query rows, a free S buffer and the chunk
+                if (haveS) {
+                    if (!qS) qS = mbar_ready_w(&qfull, nS & 1);
+                    bool ready = qS;
+                    if (ready && cS == 0 && gS >= 2) ready = mbar_ready_cluster_w(&sfree[gS & 1], ((gS >> 1) - 1) & 1);
+                    const int s = kc % kKS;
+                    if (ready && mbar_ready_w(&kfull[s], (kc / kKS) & 1)) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int gi = 0; gi < kKU; ++gi)
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_pair_ss_w(tmem + kColS + 64 * (gS & 1),
+                                              sdesc_add(dQ, (kKU * cS + gi) * kBox + ks * 32),
+                                              sdesc_add(dK, (s * kKU + gi) * kBox + ks * 32), idS,
+                                              (cS == 0 && gi == 0 && ks == 0) ? 0u : 1u);
+                        mma_commit_pair_w(&kempty[s]);
+                        ++kc;
+                        if (++cS == kKUnits) {
+                            cS = 0;
+                            mma_commit_pair_w(&sfull[gS & 1]);
+                            ++gS;
+                            if (++kS == itS.t1 - itS.t0) {
+                                mma_commit_pair_w(&qempty);
+                                kS = 0;
+                                qS = false;
+                                ++nS;
+                                haveS = iterS.next(itS);
+                            }
+                        }
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    idle = 0;
+                } else if ((++idle & 255u) == 0) {
+                    const uint64_t now = globaltimer();
+                    if (idle == 256) t_idle = now;
+                    const int quit = (*abort || now - t_idle > kWaitLimitNs) ? 1 : 0;
+                    if (__shfl_sync(0xffffffffu, quit, 0)) ok = false;
+                }
+            }
+            if (!ok && lane == 0) fail();
+            mma_commit_pair_w(&drain);
+            mbar_wait(&drain, 0, nullptr);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ value loads
+        // Value unit (half h, key half kh) of tile g: latent columns
+        // [256h + 128r, +128) (column groups 4h + 2r and 4h + 2r + 1) of keys
+        // [64 kh, 64 kh + 64), one tensor copy.  A unit is requested once its
+        // slot is free and the first key unit of tile g + 1 has been requested;
+        // once it lands, rows past the visible keys (last tile of an item) are
+        // zeroed, then the even CTA's MMA warp is told.
+        // The warp runs one loop; lane 0 decides, every lane zeroes.
+        ItemIter it_req, it_rel;                 // the request and the relay side walk the same items
+        it_req.init(a, pair);
+        it_rel.init(a, pair);
+        Item req, rel;
+        bool have_req = it_req.next(req), have_rel = it_rel.next(rel);
+        int tile_req = have_req ? req.t0 : 0, tile_rel = have_rel ? rel.t0 : 0;
+        uint32_t c_req = 0, c_rel = 0;           // unit within the tile
+        uint32_t g_req = 0;                      // global tile of the next request
+        uint32_t vq = 0, vr = 0;                 // ring counters: requested, relayed
+        uint32_t idle = 0;
+        uint64_t t_idle = 0;
+        bool ok = true;
+        while (ok && have_rel) {
+            bool progressed = false;
+            if (have_req && vq < vr + kVS) {
+                const int vs = vq % kVS;
+                const bool lagged = *kiss >= (int)(kKUnits * (g_req + 1) + kVLagUnits);
+                const bool free_ = vq < (uint32_t)kVS || mbar_ready(&vempty[vs], ((vq / kVS) - 1) & 1);
+                if (__shfl_sync(0xffffffffu, (lagged && free_) ? 1 : 0, 0)) {
+                    if (lane == 0) {
+                        const int b = req.bj / a.n_q;
+                        const int half = c_req >> 1, kh = c_req & 1;
+                        const int key0 = tile_req * kKeys + 64 * kh;
+                        mbar_expect_tx(&vland[vs], 2 * kBox);
+                        tma_load_4d(smem + kOffV + vs * 2 * kBox, &map_v, &vland[vs], 0, key0, 4 * half + 2 * (int)rank, b);
+                    }
+                    ++vq;
+                    if (++c_req == kVUnits) {
+                        c_req = 0;
+                        ++g_req;
+                        if (++tile_req == req.t1) {
+                            have_req = it_req.next(req);
+                            if (have_req) tile_req = req.t0;
+                        }
+                    }
+                    progressed = true;
+                }
+            }
+            if (vr < vq && mbar_ready_w(&vland[vr % kVS], (vr / kVS) & 1)) {
+                const int vs = vr % kVS;
+                // keys of this unit: [tile * 128 + 64 kh, +64); rows of keys >= n_vis are zeroed
+                const int first = tile_rel * kKeys + 64 * (int)(c_rel & 1);
+                const int keep = max(0, min(64, rel.n_vis - first));
+                if (keep < 64) {
+                    const uint32_t base = sbase + kOffV + vs * 2 * kBox;
+                    const int nrows = 64 - keep;           // rows keep..63 of both column groups
+                    for (int i = lane; i < nrows * 16; i += 32) {
+                        const int r = keep + (i >> 4), grp = (i >> 3) & 1, ch = i & 7;
+                        st_shared_u4(base + grp * kBox + r * 128 + ch * 16, 0u, 0u, 0u, 0u);
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                }
+                if (lane == 0) mbar_arrive_peer(lead(&vready[vs]));
+                ++vr;
+                if (++c_rel == kVUnits) {
+                    c_rel = 0;
+                    if (++tile_rel == rel.t1) {
+                        have_rel = it_rel.next(rel);
+                        if (have_rel) tile_rel = rel.t0;
+                    }
+                }
+                progressed = true;
+            }
+            if (progressed) {
+                idle = 0;
+            } else if ((++idle & 255u) == 0) {
+                const uint64_t now = globaltimer();
+                if (idle == 256) t_idle = now;
+                const int quit = (*abort || now - t_idle > kWaitLimitNs) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, quit, 0)) ok = false;
+            }
+        }
+        if (!ok && lane == 0) fail();
+        // every requested chunk has landed before the CTA may exit
+        for (uint32_t i = vr; i < vq; ++i)
+            if (lane == 0) mbar_wait(&vland[i % kVS], (i / kVS) & 1, nullptr);
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax and epilogue
+        // Thread t (0..127) <-> TMEM lane t: head 64r + t % 64 of this CTA, the
+        // t / 64 half of the tile's keys in S and of each 256-column latent half
+        // in O.  Partners t and t ^ 64 share a head: their tile maxima and, at
+        // the end of an item, their row sums meet through xch.
+        const int t = threadIdx.x - 128;
+        const int q = warp & 3;
+        const int hl = t & 63, part = t >> 6;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const bool leader = t == 0;
+        auto lane0 = [&](bool ok) -> bool { return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0; };
+        auto group_sync = [&]() { named_barrier(1, 128); };
+        ItemIter iter;
+        iter.init(a, pair);
+        Item item;
+        uint32_t g = 0, n_item = 0;
+        bool stop = false;
+        while (!stop && iter.next(item)) {
+            const int T = item.t1 - item.t0;
+            float m_used = -INFINITY, l = 0.f;     // this thread's part of the row sum, relative to m_used
+            for (int k = 0; k < T && !stop; ++k, ++g) {
+                const int sb = g & 1;
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait(&sfull[sb], (g >> 1) & 1, abort);
+                if (!lane0(ok)) { stop = true; break; }
+                tc_fence_after();
+                float x[64];
+                {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[32 + i] = __uint_as_float(r[i]);
+                }
+                tc_fence_before();
+                // keys past the visible ones (last tile) take no weight, whatever they hold
+                const int key0 = (item.t0 + k) * kKeys + 64 * part;
+                const int valid = min(64, item.n_vis - key0);
+                if (valid < 64) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) x[i] = i < valid ? x[i] : -INFINITY;
+                }
+                float mx8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mx8[i] = fmaxf(fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24])),
+                                   fmaxf(fmaxf(x[i + 32], x[i + 40]), fmaxf(x[i + 48], x[i + 56])));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
+                // base 2: scores scaled by scale * log2(e) (> 0, so the raw maximum serves)
+                const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
+                xch[sb][t] = mx;
+                group_sync();                        // every S read of this tile is done, maxima published
+                if (leader) mbar_arrive_peer(lead(&sfree[sb]));
+                const float m_tile = fmaxf(mx, xch[sb][t ^ 64]);
+                // Lazy rescaling: the maximum moves only when it grew by more than 2^8
+                // (an item's first tile takes its maximum as it is).
+                const float m_cand = fmaxf(m_used, m_tile);
+                const float m = (k == 0 || m_cand > m_used + kRescaleThreshold) ? m_cand : m_used;
+                // P buffer sb is free once O(g - 2) has completed
+                if (g >= 2) {
+                    if (lane == 0) ok = mbar_wait(&pfree[sb], ((g >> 1) - 1) & 1, abort);
+                    if (!lane0(ok)) { stop = true; break; }
+                }
+                // O holds the item's tiles before g relative to m_used: rescale it when m
+                // moved (after O(g - 1) completed).  Warp-collective TMEM access: lanes
+                // that need none multiply by 1.
+                const bool need = k > 0 && m > m_used;
+                if (__any_sync(0xffffffffu, need)) {
+                    if (lane == 0) ok = mbar_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort);
+                    if (!lane0(ok)) { stop = true; break; }
+                    tc_fence_after();
+                    const float alpha = need ? ex2(m_used - m) : 1.f;
+#pragma unroll 1
+                    for (int c = 0; c < 16; ++c) {
+                        uint32_t r[16];
+                        const uint32_t ta = tmem + lane_off + kColO + 16 * c;
+                        tmem_ld16(ta, r);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st16(ta, r);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+                if (m > m_used) {
+                    if (m_used != -INFINITY) l *= ex2(m_used - m);
+                    m_used = m;
+                }
+                // P row: head hl, keys [64 part, 64 part + 64) -> box `part` of buffer sb
+                const uint32_t prow = sbase + kOffP + sb * 2 * kBox + part * kBox + hl * 128;
+                float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t pw[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float p0 = ex2(fmaf(x[8 * c + 2 * i], a.scale_log2, -m));
+                        const float p1 = ex2(fmaf(x[8 * c + 2 * i + 1], a.scale_log2, -m));
+                        ps4[i] += p0 + p1;
+                        pw[i] = pack_bf16(p0, p1);
+                    }
+                    st_shared_u4(prow + ((c ^ (hl & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                }
+                l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
+                fence_async_smem();
+                group_sync();
+                if (leader) mbar_arrive_peer(lead(&pfull[sb]));
+            }
+            if (stop) break;
+            // epilogue: the two halves of each head's row sum meet; every thread writes
+            // its 2 x 128 latent columns (normalised, or a partial plus log2-sum-exp)
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&item_done, n_item & 1, abort);
+            if (!lane0(ok)) break;
+            xch[n_item & 1][t] = l;
+            group_sync();
+            const float lsum = l + xch[n_item & 1][t ^ 64];
+            tc_fence_after();
+            const float inv = 1.f / lsum;
+            const int head = 64 * (int)rank + hl;
+            // each warp stages 32 rows x 64 bytes in its quarter of the P area so one
+            // store instruction covers eight contiguous 64-byte row segments
+            const uint32_t scr = sbase + kOffP + q * 2048;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                const int half = c >> 2, sub = c & 3;             // 32 columns per step
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_off + kColO + 128 * half + 32 * sub, r);
+                tmem_wait_ld();
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    st_shared_u4(scr + lane * 64 + ((j ^ (lane & 3)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2],
+                                 w[4 * j + 3]);
+                __syncwarp();
+                // lane i of this warp holds row (thread) 32 q + i: head 64 r + (32 q + i) % 64,
+                // columns 256 half + 128 part + 32 sub
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int rr = 8 * kk + (lane >> 2), pc = lane & 3;
+                    const int tt = 32 * q + rr;
+                    const int hh = 64 * (int)rank + (tt & 63);
+                    const uint4 v = ld_shared_u4(scr + rr * 64 + ((pc ^ (rr & 3)) << 4));
+                    __nv_bfloat16* rowp = (item.slot < 0 ? a.o_lat + ((int64_t)item.bj * 128 + hh) * 512
+                                                         : a.part_o + ((int64_t)item.slot * 128 + hh) * 512);
+                    *reinterpret_cast<uint4*>(rowp + 256 * half + 128 * (tt >> 6) + 32 * sub + 8 * pc) = v;
+                }
+                __syncwarp();
+            }
+            if (item.slot >= 0 && part == 0) a.part_lse[item.slot * 128 + head] = m_used + __log2f(lsum);
+            // the next item's first value GEMM (accumulate = 0) may start only after
+            // both CTAs' reads of this item's O
+            tc_fence_before();
+            group_sync();
+            if (leader) mbar_arrive_peer(lead(&ep_done));
+            ++n_item;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort) {
+        // a wait expired: loads already requested may still be landing in this
+        // CTA's shared memory; give them time before the CTA exits
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) __nanosleep(1000);
+    }
+    cluster_sync();          // no CTA leaves while its peer may still access it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+int launch_attend_pair(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
+                       __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches) {
+    // Rows of 576 columns viewed as 9 groups of 64: (column in group, row,
+    // group, ...) with the group dimension's stride 128 bytes, so one box of
+    // several groups lands group-major (each group a 64-row x 128-byte block).
+    CUtensorMap mq, mk, mv;
+    {
+        // query rows: [BJ * 128][576]; one box = 64 rows x all 9 groups
+        const uint64_t dims[3] = {64, (uint64_t)c.batch * c.n_q * 128, 9};
+        const uint64_t str[2] = {576 * 2, 64 * 2};
+        const uint32_t box[3] = {64, 64, 9};
+        if (!make_map(&mq, q_lat, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        // cache [batch][capacity][576]; key units 64 keys x 3 groups, value units 64 keys x 2 groups
+        const uint64_t dims[4] = {64, (uint64_t)c.capacity, 9, (uint64_t)c.batch};
+        const uint64_t str[3] = {576 * 2, 64 * 2, (uint64_t)c.capacity * 576 * 2};
+        const uint32_t box_k[4] = {64, 64, kKU, 1}, box_v[4] = {64, 64, 2, 1};
+        if (!make_map(&mk, c.cache, 4, dims, str, box_k, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mv, c.cache, 4, dims, str, box_v, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    PairArgs a{};
+    a.q_lat = q_lat;
+    a.cum = cum;
+    a.first_bj = first_bj;
+    a.seq_lens = c.seq_lens;
+    a.BJ = c.batch * c.n_q;
+    a.n_q = c.n_q;
+    a.pairs = pairs;
+    a.scale_log2 = c.d.softmax_scale * 1.4426950408889634f;
+    a.o_lat = o_lat;
+    a.part_o = part_o;
+    a.part_lse = part_lse;
+    a.status = c.status;
+    const size_t smem = kSmemBytes + 1024;
+    if (cudaFuncSetAttribute(attend_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MLA_ERR_CUDA;
+    prof_begin(c.stream, "sm100_attend");
+    const cudaError_t e = launch_pdl(attend_pair_kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, mq, mk, mv, a);
+    prof_end(c.stream);
+    if (launches) ++*launches;
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace sm100
+}  // namespace mla

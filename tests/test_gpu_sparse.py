@@ -4,8 +4,9 @@ a top-k selection of the cached latents per query).
 
 * against the oracle's decode over the same selection (bf16 bar), with
   ragged counts, tail tiles and two causal queries;
-* selecting every visible key in order reproduces mla_decode bit for bit
-  (the gathered tiles are the contiguous tiles);
+* selecting every visible key reproduces mla_decode (the dense decode runs
+  another kernel, so the two agree within the bf16 bar, and both match the
+  oracle's dense decode);
 * a count outside 1..min(max_sel, p + 1) sets MLA_ERR_LEN and zeroes that
   query's outputs; a slot past the query's position sets MLA_ERR_INDEX."""
 import os
@@ -73,7 +74,14 @@ def test_sparse_full_selection_equals_dense():
     dense.step()
     torch.cuda.synchronize()
     assert dense.get_status() == 0
-    assert torch.equal(sparse_out, dense.out)
+    s_np = sparse_out.double().cpu().numpy()
+    d_np = dense.out.double().cpu().numpy()
+    assert np.isfinite(s_np).all() and np.isfinite(d_np).all()
+    assert rel_err(s_np, d_np) <= TOL["bf16"]
+    k_rot = O.rope_cache(host["k_rope"], host["seq_lens"], w.rope_base)
+    ref = O.decode_naive(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"], host["c_kv"], k_rot,
+                         host["seq_lens"], n_q, w.softmax_scale, w.rope_base)
+    assert rel_err(s_np, ref) <= TOL["bf16"] and rel_err(d_np, ref) <= TOL["bf16"]
 
 
 def test_sparse_bad_count_zeroes_the_query():
