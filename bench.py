@@ -550,8 +550,9 @@ def run_ours(a, rank, world, local):
         achieved = kbytes / avg_s / 1e9
         roof = {"kernel": kname, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": committed_traffic(kname),
-                "algorithmic_bytes_per_launch": kbytes, "avg_launch_us": avg_s * 1e6,
-                "peak_source": peaks["source"]}
+                "algorithmic_bytes_per_launch": kbytes,
+                "intermediate_bytes_per_launch": RF.kernel_intermediate_bytes(kname, w_rank, q_el, q_el),
+                "avg_launch_us": avg_s * 1e6, "peak_source": peaks["source"]}
     kernels = {}
     for n, (c, t) in sorted(prof.items()):
         kb = RF.kernel_bytes(n, w_rank, lens, q_el, q_el)

@@ -52,6 +52,20 @@ __device__ __forceinline__ void rope_pair_turn(float x0, float x1, int64_t pos, 
     *y1 = x0 * s + x1 * c;
 }
 
+// The same rotation for results stored in bf16: the hardware sine / cosine
+// (__sincosf, absolute error about 2^-21 on [-pi, pi), far below bf16's 2^-9
+// relative rounding) instead of the correctly reduced sincosf, which costs
+// microseconds per token in the absorb and prefill kernels.
+__device__ __forceinline__ void rope_pair_turn_bf16(float x0, float x1, int64_t pos, uint64_t turn, float* y0,
+                                                    float* y1) {
+    const uint64_t t = (uint64_t)pos * turn;
+    const float ang = (float)(int32_t)(uint32_t)(t >> 32) * 1.46291807926715968e-9f;   // 2 pi / 2^32
+    float s, c;
+    __sincosf(ang, &s, &c);
+    *y0 = x0 * c - x1 * s;
+    *y1 = x0 * s + x1 * c;
+}
+
 // Query position of token j of a sequence holding len keys (its queries'
 // entries included): p = len - n_q + j.
 __device__ __forceinline__ int64_t query_pos(int64_t len, int n_q, int j) { return len - n_q + j; }

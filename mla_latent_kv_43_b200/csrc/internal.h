@@ -38,8 +38,8 @@ struct AppendCall {
     cudaStream_t stream;
 };
 
-// Dense tensor-core decode: the CTA-pair attention kernel over 128-key tiles
-// (true) or the single-CTA-pair latent-split kernel over 64-key tiles (false).
+// Dense tensor-core decode: the CTA-pair attention kernel (heads split across
+// the pair, cta_group::2 MMAs; true) or the latent-split kernel (false).
 constexpr bool kDecodePairKernel = false;
 
 // True when the tensor-core path serves these dims: bf16 with the

@@ -199,7 +199,7 @@ append_kernel(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ 
                 continue;
             }
             float y0 = v0[i], y1 = v1[i];
-            if (n >= 512) rope_pair_turn(v0[i], v1[i], pos, a.rope_turn[(n - 512) >> 1], &y0, &y1);
+            if (n >= 512) rope_pair_turn_bf16(v0[i], v1[i], pos, a.rope_turn[(n - 512) >> 1], &y0, &y1);
             const int b = m / a.n_new;
             *reinterpret_cast<uint32_t*>(a.cache + ((int64_t)b * a.capacity + pos) * kFeatures + n) = pack_bf16(y0, y1);
         }

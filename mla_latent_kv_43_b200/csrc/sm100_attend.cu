@@ -78,7 +78,7 @@ struct AttnArgs {
     float scale_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* o_lat;         // [BJ][128][512]
     __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
-    float* part_lse;              // [2 * pairs][128], log2 domain
+    float* part_lse;              // [2 * pairs][2 latent halves][128], log2 domain
     int32_t* status;
     // sparse decode: the selected slots of each query token and their count
     const int32_t* sel;           // [BJ][max_sel]
@@ -701,7 +701,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                         w[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
                     put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 32 * c) * 2; });
                 }
-                if (item.slot >= 0 && rank == 0 && grp == 0) a.part_lse[item.slot * 128 + h] = mf + __log2f(lsum);
+                if (item.slot >= 0 && grp == 0) a.part_lse[(item.slot * 2 + rank) * 128 + h] = mf + __log2f(lsum);
             }
             // the next item's first O GEMM (accumulate = 0) may start only after both
             // groups' reads of this item's O
@@ -729,7 +729,8 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 }  // namespace
 
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches) {
+                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs,
+                  int* launches) {
     const bool sparse = c.n_sel != nullptr;
     CUtensorMap ml, mr;
     if (sparse) {

@@ -1,7 +1,7 @@
 // Absorbed MLA attention against the latent cache on a CTA pair
 // (tcgen05 cta_group::2): the dense decode's core kernel.
 //
-// For one query token (b, j) and a range of 128-key tiles of its sequence,
+// For one query token (b, j) and a range of 64-key tiles of its sequence,
 // with q_lat = [W_uk q_nope || RoPE(q_rope)] (576 wide, all 128 heads):
 //     S[h][n] = <q_lat[h], cache[b][n][0:576]>                    (score)
 //     online softmax over n (base 2, scale folded in), fp32 state
@@ -14,39 +14,42 @@
 // Work split.  A cluster of two CTAs on two SMs is one MMA unit.  All 128
 // heads of a token are the M dimension of both contractions, split 64 / 64:
 // CTA r holds the query rows and the softmax of heads [64r, 64r + 64).
-//  * Score GEMM (M 128 heads, N 128 keys, K 576): CTA r stages keys
-//    [64r, 64r + 64) of the tile, all 576 columns; each CTA's S holds its 64
-//    heads against all 128 keys -- complete scores, no partial sums to
+//  * Score GEMM (M 128 heads, N 64 keys, K 576): CTA r stages keys
+//    [32r, 32r + 32) of the tile, all 576 columns; each CTA's S holds its 64
+//    heads against all 64 keys -- complete scores, no partial sums to
 //    exchange.
-//  * Value GEMM (M 128 heads, N 256 latent columns, twice, K 128 keys): CTA r
+//  * Value GEMM (M 128 heads, N 256 latent columns, twice, K 64 keys): CTA r
 //    stages latent columns [128r, 128r + 128) and [256 + 128r, 256 + 128r +
-//    128) of all 128 keys.  These are re-read from L2 (the score stage of the
+//    128) of all 64 keys.  These are re-read from L2 (the score stage of the
 //    same tile brought them there from HBM a tile period earlier), so each
 //    cache byte crosses HBM once; no load is multicast.
 // Each CTA keeps its 64 heads x 512 latent fp32 O in TMEM.
 //
-// TMEM per CTA (512 columns): O [0, 256), S double buffer [256, 320) and
-// [320, 384).  In the pair layout (M = 128 over two CTAs) a CTA's 64 rows
+// TMEM per CTA (512 columns): O [0, 256), S double buffer [256, 288) and
+// [288, 320).  In the pair layout (M = 128 over two CTAs) a CTA's 64 rows
 // fill all 128 lanes: lane i and lane i + 64 both hold row i, the first and
 // the second half of the N columns.
 //
 // Shared memory per CTA: the query rows (9 groups of 64 columns x 64 rows,
-// 72 KB), two P buffers (64 heads x 128 keys bf16), a ring of key units (3
-// column groups x 64 keys, 24 KB) for the score GEMM and a ring of value
-// units (2 column groups x 64 keys, 16 KB) for the value GEMM.  Every staged
-// unit arrives in ONE tensor copy: the maps view a cache row as 9 groups of
+// 72 KB), two P buffers (64 heads x 64 keys bf16), a ring of two key tiles
+// (this CTA's 32 keys x 9 column groups, 36 KB each) for the score GEMM and
+// a ring of four value units (2 column groups x 64 keys, 16 KB; two per tile)
+// for the value GEMM, so both rings hold two tiles.  Every staged unit
+// arrives in ONE tensor copy: the maps view a cache row as 9 groups of
 // 64 columns (a dimension of stride 128 bytes placed after the key
 // dimension), so a box of several groups lands as consecutive 8 KB
 // group-major blocks, the layout both GEMMs read.  (A single thread issues
 // about one tensor copy per 0.3 us whatever its size up to 16 KB, so fewer,
 // larger copies are what keeps the loads at HBM speed.)
 //
-// Roles (256 threads): warp 0 key / query loads, warp 1 MMA issue (even CTA;
+// Roles (384 threads): warp 0 key / query loads, warp 1 MMA issue (even CTA;
 // TMEM allocation in both), warp 2 value loads (and the zeroing of value rows
-// past the visible keys), warps 4-7 softmax and epilogue (thread t <-> TMEM
-// lane t: head 64r + t % 64, key / column half t / 64).
+// past the visible keys), warps 4-11 softmax and epilogue: thread t of
+// warps 4-7 and of warps 8-11 reads TMEM lane t (head 64r + t % 64, key /
+// column half t / 64), the two warp sets splitting each lane's columns, so
+// every tile's softmax runs on 256 threads of 16 scores each.
 //
-// Work items as in the single-CTA kernel: the 128-key tiles of all query
+// Work items as in the single-CTA kernel: the 64-key tiles of all query
 // tokens are concatenated and cut into one contiguous range per pair.  A
 // token whose tiles all fall in one pair's range is finished there
 // (normalised latent output, bf16); a token cut across pairs leaves partial
@@ -65,36 +68,36 @@ namespace sm100 {
 
 namespace {
 
-constexpr int kKeys = 128;                   // keys per tile (the pair)
+constexpr int kKeys = 64;                    // keys per tile (the pair); 32 staged by each CTA for the score
 constexpr int kBox = 8192;                   // one column group of 64 rows
 constexpr int kQBoxes = 9;                   // 576 / 64 column groups
-constexpr int kKU = 3;                       // column groups per key unit
-constexpr int kKUnits = kQBoxes / kKU;       // key units per tile
-constexpr int kKS = 3;                       // key-unit ring slots
-constexpr int kVS = 3;                       // value-unit ring slots
-constexpr int kVUnits = 4;                   // value units per tile: 2 latent halves x 2 key halves
+constexpr int kKTile = kQBoxes * 4096;       // one CTA's key tile: 9 groups x 32 keys
+constexpr int kKS = 2;                       // key-tile ring slots
+constexpr int kVS = 4;                       // value-unit ring slots
+constexpr int kVUnits = 2;                   // value units per tile: 2 latent halves
 constexpr int kOffQ = 0;
-constexpr int kOffP = kOffQ + kQBoxes * kBox;         // 2 buffers x 2 boxes (64 keys each)
-constexpr int kOffK = kOffP + 4 * kBox;
-constexpr int kOffV = kOffK + kKS * kKU * kBox;
+constexpr int kOffP = kOffQ + kQBoxes * kBox;         // 2 buffers of 64 heads x 64 keys
+constexpr int kOffK = kOffP + 2 * kBox;
+constexpr int kOffV = kOffK + kKS * kKTile;
 constexpr int kSmemBytes = kOffV + kVS * 2 * kBox;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr uint32_t kColO = 0, kColS = 256, kTmemCols = 512;
+constexpr uint32_t kSCols = kKeys / 2;        // S columns per buffer (64 heads x 64 keys in the pair layout)
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
-// value units of tile g may be fetched once the first key unit of tile g + 1
-// has been requested (tile g's latent columns are then in L2)
-constexpr int kVLagUnits = 1;
+// value units of tile g may be fetched once the key tile g + 1 has been
+// requested (tile g's latent columns are then in L2)
+constexpr int kVLagTiles = 1;
 
 struct PairArgs {
     const __nv_bfloat16* q_lat;   // [BJ][128][576]
-    const int32_t* cum;           // [BJ + 1] 128-key tile prefix
+    const int32_t* cum;           // [BJ + 1] 64-key tile prefix
     const int32_t* first_bj;      // [pairs] first query token of each pair's range
     const int32_t* seq_lens;
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* o_lat;         // [BJ][128][512]
     __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
-    float* part_lse;              // [2 * pairs][128], log2 domain
+    float* part_lse;              // [2 * pairs][2 latent halves][128], log2 domain
     int32_t* status;
 };
 
@@ -167,8 +170,11 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         drain;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
-    __shared__ int k_issued;                  // key units this CTA has requested (value-load pacing)
-    __shared__ float xch[2][128];             // partner exchange of the softmax (row max, row sum)
+    __shared__ int k_issued;                  // key tiles this CTA has requested (value-load pacing)
+    // the four threads of a head exchange tile maxima and row sums; every read
+    // of one use precedes a group barrier that precedes the next write
+    __shared__ float xch[256];
+    __shared__ int group_ok[2];               // softmax group: outcome of the leader's bounded waits
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -226,6 +232,7 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         if (elect_one()) {
             tma_prefetch(&map_q);
             tma_prefetch(&map_k);
+            const uint64_t keep_l2 = l2_policy_evict_last();
             ItemIter iter;
             iter.init(a, pair);
             Item item;
@@ -240,18 +247,17 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 }
                 if (rank == 0) mbar_expect_tx(&qfull, 2 * kQBoxes * kBox);
                 tma_load_3d_pair(smem + kOffQ, &map_q, lead(&qfull), 0, item.bj * 128 + 64 * (int)rank, 0);
-                for (int t = item.t0; t < item.t1 && ok; ++t) {
-                    const int key0 = t * kKeys + 64 * (int)rank;
-                    for (int u = 0; u < kKUnits; ++u, ++kc) {
-                        const int s = kc % kKS;
-                        if (kc >= (uint32_t)kKS && !mbar_wait(&kempty[s], ((kc / kKS) - 1) & 1, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        if (rank == 0) mbar_expect_tx(&kfull[s], 2 * kKU * kBox);
-                        tma_load_4d_pair(smem + kOffK + s * kKU * kBox, &map_k, lead(&kfull[s]), 0, key0, kKU * u, b);
-                        *kiss = (int)kc + 1;
+                for (int t = item.t0; t < item.t1; ++t, ++kc) {
+                    const int key0 = t * kKeys + 32 * (int)rank;
+                    const int s = kc % kKS;
+                    if (kc >= (uint32_t)kKS && !mbar_wait(&kempty[s], ((kc / kKS) - 1) & 1, abort)) {
+                        ok = false;
+                        break;
                     }
+                    if (rank == 0) mbar_expect_tx(&kfull[s], 2 * kKTile);
+                    // kept in L2 for the value re-read of the same tile
+                    tma_load_4d_pair_hint(smem + kOffK + s * kKTile, &map_k, lead(&kfull[s]), 0, key0, 0, b, keep_l2);
+                    *kiss = (int)kc + 1;
                 }
                 ++n;
             }
@@ -260,15 +266,15 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issue (even CTA)
-        // Two streams in tile order, advanced one staged unit at a time: score
-        // GEMMs S(g) (3 key units of 3 column groups, 4 K-steps per group) and
-        // value GEMMs O(g) (4 value units, 4 K-steps each).  The whole warp runs the loop (decisions are
+        // Two streams in tile order: score GEMMs S(g) (one key tile, 9 column
+        // groups x 4 K-steps) and value GEMMs O(g) (2 value units, 4 K-steps
+        // each), the latter advanced one unit at a time.  The whole warp runs the loop (decisions are
         // lane 0's observations, broadcast); one elected lane issues.
         if (rank == 0) {
-            constexpr uint32_t idS = idesc_bf16(128, kKeys, false, false);
+            constexpr uint32_t idS = idesc_bf16(128, kKeys, false, false);      // pair: 32 keys from each CTA
             constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
             const uint64_t dQ = sdesc(sbase + kOffQ, 16, 1024, kSwizzle128);     // query rows, K-major
-            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);     // key chunk, K-major
+            const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);     // key tile, K-major
             const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);     // P rows, K-major
             const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);   // value unit, MN-major
             ItemIter iterS, iterO;
@@ -278,7 +284,7 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             bool haveS = iterS.next(itS), haveO = iterO.next(itO);
             int kS = 0, kO = 0;                    // tile index within the current item
             uint32_t gS = 0, gO = 0;               // global tile counters
-            uint32_t cS = 0, cO = 0;               // chunk within the current tile
+            uint32_t cO = 0;                       // value unit within the current tile
             uint32_t kc = 0, vc = 0;               // ring chunk counters
             uint32_t nS = 0, nO = 0;               // item counters
             bool qS = false;                       // query rows of the current S item landed
@@ -298,13 +304,13 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     const int vs = vc % kVS;
                     if (ready && mbar_ready_cluster_w(&vready[vs], (vc / kVS) & 1)) {
                         tc_fence_after();
-                        const int half = cO >> 1, kh = cO & 1;               // latent half, key half
+                        const int half = cO;                                 // latent half
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) {
-                            const uint32_t pa = (gO & 1) * 2 * kBox + kh * kBox + ks * 32;
+                            const uint32_t pa = (gO & 1) * kBox + ks * 32;
                             mma_pair_ss_w(tmem + kColO + 128 * half, sdesc_add(dP, pa),
                                           sdesc_add(dV, vs * 2 * kBox + ks * 2048), idO,
-                                          (kO == 0 && kh == 0 && ks == 0) ? 0u : 1u);
+                                          (kO == 0 && ks == 0) ? 0u : 1u);
                         }
                         mma_commit_pair_w(&vempty[vs]);
                         ++vc;
@@ -323,35 +329,31 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                         progressed = true;
                     }
                 }
-                // key chunk of S(gS): needs the item's query rows, a free S buffer and the chunk
+                // S(gS): needs the item's query rows, a free S buffer and the key tile
                 if (haveS) {
                     if (!qS) qS = mbar_ready_w(&qfull, nS & 1);
                     bool ready = qS;
-                    if (ready && cS == 0 && gS >= 2) ready = mbar_ready_cluster_w(&sfree[gS & 1], ((gS >> 1) - 1) & 1);
+                    if (ready && gS >= 2) ready = mbar_ready_cluster_w(&sfree[gS & 1], ((gS >> 1) - 1) & 1);
                     const int s = kc % kKS;
                     if (ready && mbar_ready_w(&kfull[s], (kc / kKS) & 1)) {
                         tc_fence_after();
 #pragma unroll
-                        for (int gi = 0; gi < kKU; ++gi)
+                        for (int gi = 0; gi < kQBoxes; ++gi)
 #pragma unroll
                             for (int ks = 0; ks < 4; ++ks)
-                                mma_pair_ss_w(tmem + kColS + 64 * (gS & 1),
-                                              sdesc_add(dQ, (kKU * cS + gi) * kBox + ks * 32),
-                                              sdesc_add(dK, (s * kKU + gi) * kBox + ks * 32), idS,
-                                              (cS == 0 && gi == 0 && ks == 0) ? 0u : 1u);
+                                mma_pair_ss_w(tmem + kColS + kSCols * (gS & 1), sdesc_add(dQ, gi * kBox + ks * 32),
+                                              sdesc_add(dK, s * kKTile + gi * 4096 + ks * 32), idS,
+                                              (gi == 0 && ks == 0) ? 0u : 1u);
                         mma_commit_pair_w(&kempty[s]);
+                        mma_commit_pair_w(&sfull[gS & 1]);
                         ++kc;
-                        if (++cS == kKUnits) {
-                            cS = 0;
-                            mma_commit_pair_w(&sfull[gS & 1]);
-                            ++gS;
-                            if (++kS == itS.t1 - itS.t0) {
-                                mma_commit_pair_w(&qempty);
-                                kS = 0;
-                                qS = false;
-                                ++nS;
-                                haveS = iterS.next(itS);
-                            }
+                        ++gS;
+                        if (++kS == itS.t1 - itS.t0) {
+                            mma_commit_pair_w(&qempty);
+                            kS = 0;
+                            qS = false;
+                            ++nS;
+                            haveS = iterS.next(itS);
                         }
                         progressed = true;
                     }
@@ -371,13 +373,14 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         }
     } else if (warp == 2) {
         // ------------------------------------------------------------ value loads
-        // Value unit (half h, key half kh) of tile g: latent columns
-        // [256h + 128r, +128) (column groups 4h + 2r and 4h + 2r + 1) of keys
-        // [64 kh, 64 kh + 64), one tensor copy.  A unit is requested once its
-        // slot is free and the first key unit of tile g + 1 has been requested;
+        // Value unit (half h) of tile g: latent columns [256h + 128r, +128)
+        // (column groups 4h + 2r and 4h + 2r + 1) of the tile's 64 keys, one
+        // tensor copy.  A unit is requested once its slot is free and the key
+        // tile g + 1 has been requested;
         // once it lands, rows past the visible keys (last tile of an item) are
         // zeroed, then the even CTA's MMA warp is told.
         // The warp runs one loop; lane 0 decides, every lane zeroes.
+        const uint64_t last_use = l2_policy_evict_first();     // the cache rows' last read
         ItemIter it_req, it_rel;                 // the request and the relay side walk the same items
         it_req.init(a, pair);
         it_rel.init(a, pair);
@@ -394,15 +397,16 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             bool progressed = false;
             if (have_req && vq < vr + kVS) {
                 const int vs = vq % kVS;
-                const bool lagged = *kiss >= (int)(kKUnits * (g_req + 1) + kVLagUnits);
+                const bool lagged = *kiss >= (int)(g_req + 1 + kVLagTiles);
                 const bool free_ = vq < (uint32_t)kVS || mbar_ready(&vempty[vs], ((vq / kVS) - 1) & 1);
                 if (__shfl_sync(0xffffffffu, (lagged && free_) ? 1 : 0, 0)) {
                     if (lane == 0) {
                         const int b = req.bj / a.n_q;
-                        const int half = c_req >> 1, kh = c_req & 1;
-                        const int key0 = tile_req * kKeys + 64 * kh;
+                        const int half = c_req;
+                        const int key0 = tile_req * kKeys;
                         mbar_expect_tx(&vland[vs], 2 * kBox);
-                        tma_load_4d(smem + kOffV + vs * 2 * kBox, &map_v, &vland[vs], 0, key0, 4 * half + 2 * (int)rank, b);
+                        tma_load_4d_hint(smem + kOffV + vs * 2 * kBox, &map_v, &vland[vs], 0, key0, 4 * half + 2 * (int)rank,
+                                         b, last_use);
                     }
                     ++vq;
                     if (++c_req == kVUnits) {
@@ -418,8 +422,8 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             }
             if (vr < vq && mbar_ready_w(&vland[vr % kVS], (vr / kVS) & 1)) {
                 const int vs = vr % kVS;
-                // keys of this unit: [tile * 128 + 64 kh, +64); rows of keys >= n_vis are zeroed
-                const int first = tile_rel * kKeys + 64 * (int)(c_rel & 1);
+                // keys of this unit: [tile * 64, +64); rows of keys >= n_vis are zeroed
+                const int first = tile_rel * kKeys;
                 const int keep = max(0, min(64, rel.n_vis - first));
                 if (keep < 64) {
                     const uint32_t base = sbase + kOffV + vs * 2 * kBox;
@@ -458,17 +462,44 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
         __syncwarp();
     } else if (warp >= 4) {
         // ------------------------------------------------------------ softmax and epilogue
-        // Thread t (0..127) <-> TMEM lane t: head 64r + t % 64 of this CTA, the
-        // t / 64 half of the tile's keys in S and of each 256-column latent half
-        // in O.  Partners t and t ^ 64 share a head: their tile maxima and, at
-        // the end of an item, their row sums meet through xch.
-        const int t = threadIdx.x - 128;
+        // st (0..255): TMEM lane t = st % 128 (head 64r + t % 64, key / column half
+        // part = t / 64) and column half cv = st / 128 of that lane: keys
+        // [32 part + 16 cv, +16) of each tile, O columns [128 cv, 128 cv + 128).
+        // The four threads of a head meet through xch (tile maxima; row sums at the
+        // end of an item).
+        const int st = threadIdx.x - 128;
+        const int t = st & 127, cv = st >> 7;
         const int q = warp & 3;
         const int hl = t & 63, part = t >> 6;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const bool leader = t == 0;
-        auto lane0 = [&](bool ok) -> bool { return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0; };
-        auto group_sync = [&]() { named_barrier(1, 128); };
+        const bool leader = st == 0;
+        auto group_sync = [&]() { named_barrier(1, 256); };
+        // true when the predicate holds in any thread of the group (a group barrier)
+        auto group_any = [&](bool v) -> bool {
+            uint32_t r;
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, 1, 256, p;\n\t"
+                "selp.u32 %0, 1, 0, q;\n\t}"
+                : "=r"(r)
+                : "r"((uint32_t)v)
+                : "memory");
+            return r != 0;
+        };
+        // One thread waits (bounded) and the group barrier hands its outcome to all
+        // eight warps, so they leave together on a timeout and no warp is left at a
+        // group barrier.  Alternate flag slots: a thread reads use i before the
+        // barrier of use i + 1, which precedes the leader's write of use i + 2.
+        uint32_t n_wait = 0;
+        auto group_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            const int slot = n_wait++ & 1;
+            if (leader) group_ok[slot] = mbar_wait(bar, parity, abort) ? 1 : 0;
+            group_sync();
+            return group_ok[slot] != 0;
+        };
+        auto head_sum = [&](const float* v) { return (v[hl] + v[hl + 64]) + (v[hl + 128] + v[hl + 192]); };
+        auto head_max = [&](const float* v) {
+            return fmaxf(fmaxf(v[hl], v[hl + 64]), fmaxf(v[hl + 128], v[hl + 192]));
+        };
         ItemIter iter;
         iter.init(a, pair);
         Item item;
@@ -479,65 +510,52 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             float m_used = -INFINITY, l = 0.f;     // this thread's part of the row sum, relative to m_used
             for (int k = 0; k < T && !stop; ++k, ++g) {
                 const int sb = g & 1;
-                bool ok = true;
-                if (lane == 0) ok = mbar_wait(&sfull[sb], (g >> 1) & 1, abort);
-                if (!lane0(ok)) { stop = true; break; }
+                if (!group_wait(&sfull[sb], (g >> 1) & 1)) { stop = true; break; }
                 tc_fence_after();
-                float x[64];
+                float x[16];
                 {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, r);
+                    uint32_t r[16];
+                    tmem_ld16(tmem + lane_off + kColS + kSCols * sb + 16 * cv, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 16; ++i) x[i] = __uint_as_float(r[i]);
                 }
                 tc_fence_before();
                 // keys past the visible ones (last tile) take no weight, whatever they hold
-                const int key0 = (item.t0 + k) * kKeys + 64 * part;
-                const int valid = min(64, item.n_vis - key0);
-                if (valid < 64) {
+                const int key0 = (item.t0 + k) * kKeys + 32 * part + 16 * cv;
+                const int valid = min(16, item.n_vis - key0);
+                if (valid < 16) {
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) x[i] = i < valid ? x[i] : -INFINITY;
+                    for (int i = 0; i < 16; ++i) x[i] = i < valid ? x[i] : -INFINITY;
                 }
-                float mx8[8];
+                float mx4[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mx8[i] = fmaxf(fmaxf(fmaxf(x[i], x[i + 8]), fmaxf(x[i + 16], x[i + 24])),
-                                   fmaxf(fmaxf(x[i + 32], x[i + 40]), fmaxf(x[i + 48], x[i + 56])));
-#pragma unroll
-                for (int i = 0; i < 4; ++i) mx8[i] = fmaxf(mx8[i], mx8[i + 4]);
+                for (int i = 0; i < 4; ++i) mx4[i] = fmaxf(fmaxf(x[i], x[i + 4]), fmaxf(x[i + 8], x[i + 12]));
                 // base 2: scores scaled by scale * log2(e) (> 0, so the raw maximum serves)
-                const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * a.scale_log2;
-                xch[sb][t] = mx;
+                const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * a.scale_log2;
+                xch[st] = mx;
                 group_sync();                        // every S read of this tile is done, maxima published
                 if (leader) mbar_arrive_peer(lead(&sfree[sb]));
-                const float m_tile = fmaxf(mx, xch[sb][t ^ 64]);
+                const float m_tile = head_max(xch);
                 // Lazy rescaling: the maximum moves only when it grew by more than 2^8
                 // (an item's first tile takes its maximum as it is).
                 const float m_cand = fmaxf(m_used, m_tile);
                 const float m = (k == 0 || m_cand > m_used + kRescaleThreshold) ? m_cand : m_used;
                 // P buffer sb is free once O(g - 2) has completed
-                if (g >= 2) {
-                    if (lane == 0) ok = mbar_wait(&pfree[sb], ((g >> 1) - 1) & 1, abort);
-                    if (!lane0(ok)) { stop = true; break; }
-                }
+                if (g >= 2 && !group_wait(&pfree[sb], ((g >> 1) - 1) & 1)) { stop = true; break; }
                 // O holds the item's tiles before g relative to m_used: rescale it when m
                 // moved (after O(g - 1) completed).  Warp-collective TMEM access: lanes
-                // that need none multiply by 1.
+                // that need none multiply by 1.  Whether any head of the group
+                // rescales is itself a group decision (the barrier below is group-wide).
                 const bool need = k > 0 && m > m_used;
-                if (__any_sync(0xffffffffu, need)) {
-                    if (lane == 0) ok = mbar_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort);
-                    if (!lane0(ok)) { stop = true; break; }
+                if (group_any(need)) {
+                    if (!group_wait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) { stop = true; break; }
                     tc_fence_after();
                     const float alpha = need ? ex2(m_used - m) : 1.f;
 #pragma unroll 1
-                    for (int c = 0; c < 16; ++c) {
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t r[16];
-                        const uint32_t ta = tmem + lane_off + kColO + 16 * c;
+                        const uint32_t ta = tmem + lane_off + kColO + 128 * cv + 16 * c;
                         tmem_ld16(ta, r);
                         tmem_wait_ld();
 #pragma unroll
@@ -551,20 +569,21 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     if (m_used != -INFINITY) l *= ex2(m_used - m);
                     m_used = m;
                 }
-                // P row: head hl, keys [64 part, 64 part + 64) -> box `part` of buffer sb
-                const uint32_t prow = sbase + kOffP + sb * 2 * kBox + part * kBox + hl * 128;
+                // P row: head hl, keys [32 part + 16 cv, +16) -> 16-byte chunks
+                // 4 part + 2 cv and 4 part + 2 cv + 1 of row hl of buffer sb
+                const uint32_t prow = sbase + kOffP + sb * kBox + hl * 128;
                 float ps4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
                     uint32_t pw[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const float p0 = ex2(fmaf(x[8 * c + 2 * i], a.scale_log2, -m));
-                        const float p1 = ex2(fmaf(x[8 * c + 2 * i + 1], a.scale_log2, -m));
+                        const float p0 = ex2(fmaf(x[8 * cc + 2 * i], a.scale_log2, -m));
+                        const float p1 = ex2(fmaf(x[8 * cc + 2 * i + 1], a.scale_log2, -m));
                         ps4[i] += p0 + p1;
                         pw[i] = pack_bf16(p0, p1);
                     }
-                    st_shared_u4(prow + ((c ^ (hl & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                    st_shared_u4(prow + (((4 * part + 2 * cv + cc) ^ (hl & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                 }
                 l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
                 fence_async_smem();
@@ -572,25 +591,22 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 if (leader) mbar_arrive_peer(lead(&pfull[sb]));
             }
             if (stop) break;
-            // epilogue: the two halves of each head's row sum meet; every thread writes
-            // its 2 x 128 latent columns (normalised, or a partial plus log2-sum-exp)
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&item_done, n_item & 1, abort);
-            if (!lane0(ok)) break;
-            xch[n_item & 1][t] = l;
+            // epilogue: the four parts of each head's row sum meet; every thread writes
+            // its 128 latent columns (normalised, or a partial plus log2-sum-exp)
+            if (!group_wait(&item_done, n_item & 1)) break;
+            xch[st] = l;
             group_sync();
-            const float lsum = l + xch[n_item & 1][t ^ 64];
+            const float lsum = head_sum(xch);
             tc_fence_after();
             const float inv = 1.f / lsum;
             const int head = 64 * (int)rank + hl;
-            // each warp stages 32 rows x 64 bytes in its quarter of the P area so one
+            // each warp stages 32 rows x 64 bytes in its eighth of the P area so one
             // store instruction covers eight contiguous 64-byte row segments
-            const uint32_t scr = sbase + kOffP + q * 2048;
+            const uint32_t scr = sbase + kOffP + (warp - 4) * 2048;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                const int half = c >> 2, sub = c & 3;             // 32 columns per step
+            for (int sub = 0; sub < 4; ++sub) {                   // 32 columns per step
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_off + kColO + 128 * half + 32 * sub, r);
+                tmem_ld32(tmem + lane_off + kColO + 128 * cv + 32 * sub, r);
                 tmem_wait_ld();
                 uint32_t w[16];
 #pragma unroll
@@ -601,8 +617,8 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     st_shared_u4(scr + lane * 64 + ((j ^ (lane & 3)) << 4), w[4 * j], w[4 * j + 1], w[4 * j + 2],
                                  w[4 * j + 3]);
                 __syncwarp();
-                // lane i of this warp holds row (thread) 32 q + i: head 64 r + (32 q + i) % 64,
-                // columns 256 half + 128 part + 32 sub
+                // lane i of this warp holds TMEM lane 32 q + i: head 64 r + (32 q + i) % 64,
+                // latent columns 256 cv + 128 part + 32 sub
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const int rr = 8 * kk + (lane >> 2), pc = lane & 3;
@@ -611,11 +627,16 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     const uint4 v = ld_shared_u4(scr + rr * 64 + ((pc ^ (rr & 3)) << 4));
                     __nv_bfloat16* rowp = (item.slot < 0 ? a.o_lat + ((int64_t)item.bj * 128 + hh) * 512
                                                          : a.part_o + ((int64_t)item.slot * 128 + hh) * 512);
-                    *reinterpret_cast<uint4*>(rowp + 256 * half + 128 * (tt >> 6) + 32 * sub + 8 * pc) = v;
+                    *reinterpret_cast<uint4*>(rowp + 256 * cv + 128 * (tt >> 6) + 32 * sub + 8 * pc) = v;
                 }
                 __syncwarp();
             }
-            if (item.slot >= 0 && part == 0) a.part_lse[item.slot * 128 + head] = m_used + __log2f(lsum);
+            if (item.slot >= 0 && part == 0 && cv == 0) {
+                // the same log-sum-exp for both latent halves of the piece
+                const float lse = m_used + __log2f(lsum);
+                a.part_lse[item.slot * 256 + head] = lse;
+                a.part_lse[item.slot * 256 + 128 + head] = lse;
+            }
             // the next item's first value GEMM (accumulate = 0) may start only after
             // both CTAs' reads of this item's O
             tc_fence_before();
@@ -656,10 +677,10 @@ int launch_attend_pair(const DecodeCall& c, const __nv_bfloat16* q_lat, const in
         if (!make_map(&mq, q_lat, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
-        // cache [batch][capacity][576]; key units 64 keys x 3 groups, value units 64 keys x 2 groups
+        // cache [batch][capacity][576]; key tiles 32 keys x 9 groups, value units 64 keys x 2 groups
         const uint64_t dims[4] = {64, (uint64_t)c.capacity, 9, (uint64_t)c.batch};
         const uint64_t str[3] = {576 * 2, 64 * 2, (uint64_t)c.capacity * 576 * 2};
-        const uint32_t box_k[4] = {64, 64, kKU, 1}, box_v[4] = {64, 64, 2, 1};
+        const uint32_t box_k[4] = {64, 32, kQBoxes, 1}, box_v[4] = {64, 64, 2, 1};
         if (!make_map(&mk, c.cache, 4, dims, str, box_k, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
         if (!make_map(&mv, c.cache, 4, dims, str, box_v, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }

@@ -31,7 +31,7 @@ constexpr int kMaxPairs = 256;              // clusters per launch
 // cluster at least kMinTiles key tiles of the largest possible total
 // (batch * n_q * ceil(max_len / 64)): fewer, longer pieces when there are few
 // long sequences, all 74 clusters otherwise.
-constexpr int64_t kMinTiles = 8;
+constexpr int64_t kMinTiles = 2;
 int pairs_for(int splits, int64_t BJ, int64_t max_len) {
     const int max_pairs = std::max(1, std::min(sm_count() / 2, kMaxPairs));
     if (splits > 0) return std::min(splits, max_pairs);
@@ -60,7 +60,7 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
     take(BJ * d.heads * (d.d_c + d.d_rope) * 2, &L->q_lat, &L->q_lat_bytes);
     take(BJ * d.heads * d.d_c * 2, &L->o_lat, &L->o_lat_bytes);
     take((size_t)2 * P * d.heads * d.d_c * 2, &L->part_o, &L->part_o_bytes);   // bf16
-    take((size_t)2 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);
+    take((size_t)4 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);   // [2P pieces][2 latent halves][H]
     take((BJ + 1 + P) * 4, &L->sched, &L->sched_bytes);   // tile prefix, then each cluster's first token
     L->total = off;
     L->compute_dtype = MLA_BF16;
@@ -84,8 +84,9 @@ int sm100_decode(const DecodeCall& c, int* launches) {
     int rc;
     int32_t* first_bj = cum + BJ + 1;
     if ((rc = sm100::launch_absorb(c, q_lat, cum, first_bj, P, launches))) return rc;
-    // dense decode: the CTA-pair kernel over 128-key tiles; decode over a
-    // selection: the gather kernel over 64-key tiles (the plan above uses the same size)
+    // dense decode: the CTA-pair kernel or the latent-split kernel; decode over a
+    // selection: the latent-split kernel gathering its rows (64-key tiles throughout).
+    // The up-projection merges the split-KV pieces of each token.
     rc = (c.n_sel || !kDecodePairKernel)
              ? sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, P, launches)
              : sm100::launch_attend_pair(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, P, launches);

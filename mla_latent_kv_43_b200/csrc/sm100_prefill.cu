@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(128) prefill_qrope_kernel(const __nv_bfloat16*
         for (int k = 0; k < 4; ++k) {
             const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
             float y0, y1;
-            rope_pair_turn(x.x, x.y, p, rt.turn[4 * c + k], &y0, &y1);
+            rope_pair_turn_bf16(x.x, x.y, p, rt.turn[4 * c + k], &y0, &y1);
             w[k] = pack_bf16(y0, y1);
         }
         dst[c] = make_uint4(w[0], w[1], w[2], w[3]);

@@ -43,7 +43,7 @@ struct ProjArgs {
     int pairs;
     const int32_t* n_sel;    // sparse decode: selected keys per query token (nullptr: dense)
     int max_sel;
-    int tile_keys;           // keys per attention tile: 128 (dense, CTA-pair kernel) or 64 (sparse)
+    int tile_keys;           // keys per attention tile (64)
     // upproj
     __nv_bfloat16* out;
     int32_t* status;
@@ -70,9 +70,12 @@ __device__ __forceinline__ int32_t tiles_of(const ProjArgs& a, int bj, bool* bad
     return (int32_t)((p + a.tile_keys) / a.tile_keys);
 }
 
-__device__ void plan_tiles(const ProjArgs& a, int tid) {
+// Key-tile plan, for any number of query tokens: per-thread token ranges and
+// global loads throughout (used when the tokens do not fit the staged plan).
+__device__ void plan_tiles_long(const ProjArgs& a, int tid) {
+
     // Tiles of tile_keys keys each query token attends; 0 for an invalid length.
-    __shared__ int32_t part[kThreads / 32];
+    __shared__ int32_t part_l[kThreads / 32];
     const int per = (a.BJ + kThreads - 1) / kThreads;
     const int lo = min(a.BJ, tid * per), hi = min(a.BJ, lo + per);
     int32_t sum = 0;
@@ -88,10 +91,10 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
         const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
         if (lane >= d) incl += v;
     }
-    if (lane == 31) part[warp] = incl;
+    if (lane == 31) part_l[warp] = incl;
     __syncthreads();
     int32_t run = incl - sum;
-    for (int w = 0; w < warp; ++w) run += part[w];
+    for (int w = 0; w < warp; ++w) run += part_l[w];
     if (tid == 0) a.cum[0] = 0;
     const int32_t run_lo = run;                 // cum[lo]
     bool ignored = false;
@@ -104,7 +107,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
     // range [cum[lo], cum[hi]) holds that start answers from its own values: those
     // are the clusters p with ceil(cum[lo] pairs / T) <= p < ceil(cum[hi] pairs / T).
     int32_t T = 0;
-    for (int w = 0; w < kThreads / 32; ++w) T += part[w];
+    for (int w = 0; w < kThreads / 32; ++w) T += part_l[w];
     if (T == 0) {
         for (int p = tid; p < a.pairs; p += kThreads) a.first_bj[p] = a.BJ;
         return;
@@ -121,6 +124,71 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
                 break;
             }
         }
+    }
+}
+
+constexpr int kPlanTokens = 512;           // tokens the staged plan holds in shared memory (2 KB: the absorb CTAs stay four per SM)
+
+// The key-tile plan of the attention kernel: cum[bj + 1] = key tiles of query
+// tokens 0..bj, and the first token of every cluster's tile range.  Each
+// token's length is loaded once (all loads of a thread issued together), the
+// prefix and the cluster starts are then computed from shared memory.
+__device__ void plan_tiles(const ProjArgs& a, int tid) {
+    if (a.BJ > kPlanTokens) {
+        plan_tiles_long(a, tid);
+        return;
+    }
+    __shared__ int32_t part[kThreads / 32];
+    __shared__ int32_t s_cum[kPlanTokens + 1];
+    constexpr int kPer = kPlanTokens / kThreads;
+    const int per = (a.BJ + kThreads - 1) / kThreads;
+    const int lo = min(a.BJ, tid * per), hi = min(a.BJ, lo + per);
+    int32_t t[kPer];
+    int32_t sum = 0;
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        t[i] = lo + i < hi ? tiles_of(a, lo + i, &bad) : 0;
+        sum += t[i];
+    }
+    if (bad) set_status(a.status, MLA_ERR_LEN);
+    // exclusive prefix of the per-thread sums: shuffle scan in each warp, then
+    // the four warp totals
+    const int lane = tid & 31, warp = tid >> 5;
+    int32_t incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    if (lane == 31) part[warp] = incl;
+    __syncthreads();
+    int32_t run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += part[w];
+    if (tid == 0) {
+        a.cum[0] = 0;
+        s_cum[0] = 0;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        run += t[i];
+        if (lo + i < hi) {
+            a.cum[lo + i + 1] = run;
+            s_cum[lo + i + 1] = run;
+        }
+    }
+    __syncthreads();
+    // First query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
+    // the first bj with cum[bj + 1] > floor(p T / pairs) (BJ when there is none).
+    const int32_t T = s_cum[a.BJ];
+    for (int p = tid; p < a.pairs; p += kThreads) {
+        const int32_t s0 = (int32_t)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
+        int l = 0, r = a.BJ;
+        while (l < r) {
+            const int mid = (l + r) >> 1;
+            if (s_cum[mid + 1] > s0) r = mid; else l = mid + 1;
+        }
+        a.first_bj[p] = T == 0 ? a.BJ : l;
     }
 }
 
@@ -156,6 +224,15 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     __shared__ uint32_t tmem_base;
     __shared__ int flag;
     const int h = blockIdx.x, mt = blockIdx.y, nt = blockIdx.z;
+    if (h == a.H) {
+        // the extra column of the grid: one CTA builds the attention kernel's
+        // key-tile plan, off the critical path of the projection CTAs
+        if (mt == 0 && nt == 0) {
+            grid_dep_wait();
+            plan_tiles(a, threadIdx.x);
+        }
+        return;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = a.n_tile;
     const uint32_t ncols = tmem_cols_for(N);
@@ -203,8 +280,8 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     __syncwarp();
     grid_dep_trigger();
 
-    // query RoPE (CTAs of row tile 0; one thread per token row, N <= kThreads)
-    // and the key-tile plan while the MMAs run
+    // query RoPE while the MMAs run (CTAs of row tile 0; one thread per token
+    // row, N <= kThreads)
     const int n_row = nt * N + threadIdx.x;
     if (mt == 0 && threadIdx.x < N && n_row < a.BJ) {
         const int b = n_row / a.n_q, j = n_row % a.n_q;
@@ -221,13 +298,12 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
             for (int i = 0; i < 4; ++i) {
                 const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
                 float y0, y1;
-                rope_pair_turn(x.x, x.y, p, a.rope_turn[4 * c + i], &y0, &y1);
+                rope_pair_turn_bf16(x.x, x.y, p, a.rope_turn[4 * c + i], &y0, &y1);
                 w[i] = pack_bf16(y0, y1);
             }
             dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
-    if (h == 0 && mt == 0 && nt == 0) plan_tiles(a, threadIdx.x);
 
     if (block_wait(&done, &flag, a.status)) {
         // TMEM row m holds q_lat[n][h][128 mt + m] for the N tokens; stage as
@@ -339,113 +415,281 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, ProjArgs a, MergeArgs mg
     grid_dep_wait();         // the attention kernel's latents and pieces
     grid_dep_trigger();
 
-    // B operand: row n (token nt * N + n), 64-column block kb at sB + kb * N * 128,
-    // 16-byte chunk c of the 128-byte row at ((c ^ (n & 7)) << 4).
-    // Phase 1: one thread per token finds its pieces and their log-sum-exp.
     const int nvalid = min(N, a.BJ - nt * N);
-    __shared__ int m_pf[64], m_pl[64], m_mode[64];      // mode 0: zeros, 1: o_lat as is, 2: merge
-    __shared__ float m_M[64], m_inv[64];
-    const PieceRange pr{mg.cum[mg.BJ], mg.pairs};
-    if (threadIdx.x < N) {
-        const int n = threadIdx.x;
-        int mode = 0, pf = 0, pl = -1;
-        float M = -INFINITY, S = 0.f;
-        if (n < nvalid) {
+    {
+        // B operand: row n (token nt * N + n), 64-column block kb at sB + kb * N * 128,
+        // 16-byte chunk c of the 128-byte row at ((c ^ (n & 7)) << 4).
+        // Phase 1: the pieces (slots) of each token and their log-sum-exp.  Many
+        // tokens (the usual case: one or two pieces each): one thread per token, up
+        // to kFast pieces' log-sum-exps loaded together.  Few tokens (typically
+        // cut into many pieces): one warp per token, lanes over pieces.
+        // Phase 2 (see below) then assembles the merged rows.
+        constexpr int kFast = 4;
+        const bool few = nvalid <= 8;
+        __shared__ int m_mode[64], m_np[64], m_pf[64], m_pl[64], m_slot[64][kFast];   // mode 0: zeros, 1: o_lat as is, 2: merge
+        __shared__ float m_w[64][kFast], m_M[64], m_inv[64];
+        const PieceRange pr{mg.cum[mg.BJ], mg.pairs};
+        auto token_range = [&](int n, int& mode, int& pf, int& pl) {
+            mode = 0;
+            pf = 0;
+            pl = -1;
+            if (n >= nvalid) return;
             const int bj = nt * N + n;
             const int c0 = mg.cum[bj], c1 = mg.cum[bj + 1];
-            if (c1 > c0) {
-                pf = pr.pair_of(c0);
-                pl = pr.pair_of(c1 - 1);
-                mode = pf == pl ? 1 : 2;
+            if (c1 == c0) return;
+            pf = pr.pair_of(c0);
+            pl = pr.pair_of(c1 - 1);
+            mode = pf == pl ? 1 : 2;
+        };
+        if (few) {
+            if (warp < nvalid) {
+                const int n = warp;
+                int mode, pf, pl;
+                token_range(n, mode, pf, pl);
+                float M = -INFINITY, S = 0.f;
                 if (mode == 2) {
-                    for (int p = pf; p <= pl; ++p)
-                        if (p == pf || !pr.empty(p)) M = fmaxf(M, mg.part_lse[PieceRange::slot(p, pf) * 128 + h]);
-                    for (int p = pf; p <= pl; ++p)
-                        if (p == pf || !pr.empty(p)) S += exp2f(mg.part_lse[PieceRange::slot(p, pf) * 128 + h] - M);
+                    for (int p0 = pf; p0 <= pl; p0 += 32) {
+                        const int p = p0 + lane;
+                        if (p <= pl && (p == pf || !pr.empty(p))) M = fmaxf(M, mg.part_lse[PieceRange::slot(p, pf) * 256 + h]);
+                    }
+    #pragma unroll
+                    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+                    for (int p0 = pf; p0 <= pl; p0 += 32) {
+                        const int p = p0 + lane;
+                        if (p <= pl && (p == pf || !pr.empty(p))) S += exp2f(mg.part_lse[PieceRange::slot(p, pf) * 256 + h] - M);
+                    }
+    #pragma unroll
+                    for (int d = 16; d > 0; d >>= 1) S += __shfl_xor_sync(0xffffffffu, S, d);
+                }
+                if (lane == 0) {
+                    m_mode[n] = mode;
+                    m_pf[n] = pf;
+                    m_pl[n] = pl;
+                    m_M[n] = M;
+                    m_inv[n] = mode == 2 ? 1.f / S : 0.f;
                 }
             }
+        } else if (threadIdx.x < N) {
+            const int n = threadIdx.x;
+            int mode, np = 0, pf, pl;
+            token_range(n, mode, pf, pl);
+            float M = -INFINITY, S = 0.f;
+            if (mode == 2) {
+                int sl[kFast];
+                for (int p = pf; p <= pl; ++p) {
+                    if (p != pf && pr.empty(p)) continue;
+                    if (np < kFast) sl[np] = PieceRange::slot(p, pf);
+                    ++np;
+                }
+                float lse[kFast];
+    #pragma unroll
+                for (int i = 0; i < kFast; ++i) lse[i] = i < np ? mg.part_lse[sl[i] * 256 + h] : -INFINITY;
+    #pragma unroll
+                for (int i = 0; i < kFast; ++i) M = fmaxf(M, lse[i]);
+                if (np > kFast) {            // more pieces: the rest one by one
+                    int k = 0;
+                    for (int p = pf; p <= pl; ++p) {
+                        if (p != pf && pr.empty(p)) continue;
+                        if (k++ >= kFast) M = fmaxf(M, mg.part_lse[PieceRange::slot(p, pf) * 256 + h]);
+                    }
+                }
+    #pragma unroll
+                for (int i = 0; i < kFast; ++i) {
+                    const float w = i < np ? exp2f(lse[i] - M) : 0.f;
+                    S += w;
+                    m_w[n][i] = w;
+                    m_slot[n][i] = i < np ? sl[i] : 0;
+                }
+                if (np > kFast) {
+                    int k = 0;
+                    for (int p = pf; p <= pl; ++p) {
+                        if (p != pf && pr.empty(p)) continue;
+                        if (k++ >= kFast) S += exp2f(mg.part_lse[PieceRange::slot(p, pf) * 256 + h] - M);
+                    }
+                }
+            }
+            m_mode[n] = mode;
+            m_np[n] = np;
+            m_pf[n] = pf;
+            m_pl[n] = pl;
+            m_M[n] = M;
+            m_inv[n] = mode == 2 ? 1.f / S : 0.f;
         }
-        m_pf[n] = pf;
-        m_pl[n] = pl;
-        m_mode[n] = mode;
-        m_M[n] = M;
-        m_inv[n] = mode == 2 ? 1.f / S : 0.f;
-    }
-    __syncthreads();
-    // Phase 2: one (token, 64-column block) per thread and pass; a piece's eight
-    // 16-byte loads are issued together, two pieces at a time.
-    for (int item = threadIdx.x; item < N * 8; item += kUpThreads) {
-        const int n = item >> 3, kb = item & 7;
-        const int mode = m_mode[n];
-        uint32_t w[32];
-        const int bj = nt * N + n;
-        uint4* orow = reinterpret_cast<uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512 + 64 * kb);
-        if (mode == 0) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = 0u;
-            if (n < nvalid) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) orow[c] = make_uint4(0u, 0u, 0u, 0u);
+        __syncthreads();
+        // row n of the B operand: 64-column block kb at sB + (kb * N + n) * 128, 16-byte chunk c at ((c ^ (n & 7)) << 4);
+        // lane l holds columns [16 l, 16 l + 16): block l / 4, chunks 2 (l % 4) and 2 (l % 4) + 1
+        auto put_row = [&](int n, const uint32_t (&w)[8]) {
+            const int kb = lane >> 2, c = (lane & 3) * 2;
+            const uint32_t row = smem_u32(sB + (kb * N + n) * 128);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((c ^ (n & 7)) << 4)), "r"(w[0]), "r"(w[1]),
+                         "r"(w[2]), "r"(w[3]) : "memory");
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((c + 1) ^ (n & 7)) << 4)), "r"(w[4]),
+                         "r"(w[5]), "r"(w[6]), "r"(w[7]) : "memory");
+        };
+        auto accumulate = [&](float (&acc)[16], float wt, const uint4& v0, const uint4& v1) {
+            const uint32_t pw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
+                acc[2 * j] = fmaf(wt, f.x, acc[2 * j]);
+                acc[2 * j + 1] = fmaf(wt, f.y, acc[2 * j + 1]);
             }
-        } else if (mode == 1) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = orow[c];
-                w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-            }
-        } else {
-            const int pf = m_pf[n], pl = m_pl[n];
-            const float M = m_M[n];
-            float acc[64];
-#pragma unroll
-            for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-            int p = pf;
-            while (p <= pl) {
-                int sl[2] = {-1, -1};
-                for (int k = 0; k < 2 && p <= pl; ++p) {
-                    if (p == pf || !pr.empty(p)) {
-                        if (k == 0) sl[0] = PieceRange::slot(p, pf); else sl[1] = PieceRange::slot(p, pf);
-                        ++k;
+        };
+        if (few) {
+            // Few tokens: warp w assembles 64-column block w of every token row, lanes
+            // over pieces (each lane one piece's 128-byte segment, weighted), then a
+            // butterfly sum across the lanes; rows of tokens past nvalid stay zero.
+            const int kb = warp;
+            for (int n = 0; n < N; ++n) {
+                const int mode = n < nvalid ? m_mode[n] : 0;
+                const int bj = nt * N + n;
+                float acc[64];
+    #pragma unroll
+                for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+                if (mode == 1 && lane == 0) {
+                    const uint4* src = reinterpret_cast<const uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512 + 64 * kb);
+    #pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = src[c];
+                        const uint32_t pw[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
+                            acc[8 * c + 2 * j] = f.x;
+                            acc[8 * c + 2 * j + 1] = f.y;
+                        }
                     }
-                }
-                uint4 v[2][8];
-                float wt[2] = {0.f, 0.f};
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (sl[i] >= 0) {
-                        const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)sl[i] * 128 + h) * 512 + 64 * kb);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) v[i][c] = src[c];
-                        wt[i] = exp2f(mg.part_lse[sl[i] * 128 + h] - M);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (sl[i] >= 0) {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const uint32_t pw[4] = {v[i][c].x, v[i][c].y, v[i][c].z, v[i][c].w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
-                                acc[8 * c + 2 * j] = fmaf(wt[i], f.x, acc[8 * c + 2 * j]);
-                                acc[8 * c + 2 * j + 1] = fmaf(wt[i], f.y, acc[8 * c + 2 * j + 1]);
+                } else if (mode == 2) {
+                    const int pf = m_pf[n], pl = m_pl[n];
+                    const float M = m_M[n], inv = m_inv[n];
+                    for (int p0 = pf; p0 <= pl; p0 += 32) {
+                        const int p = p0 + lane;
+                        if (p <= pl && (p == pf || !pr.empty(p))) {
+                            const int sl = PieceRange::slot(p, pf);
+                            const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)sl * 128 + h) * 512 + 64 * kb);
+                            uint4 v[8];
+    #pragma unroll
+                            for (int c = 0; c < 8; ++c) v[c] = src[c];
+                            const float wt = exp2f(mg.part_lse[sl * 256 + h] - M) * inv;
+    #pragma unroll
+                            for (int c = 0; c < 8; ++c) {
+                                const uint32_t pw[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+    #pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
+                                    acc[8 * c + 2 * j] = fmaf(wt, f.x, acc[8 * c + 2 * j]);
+                                    acc[8 * c + 2 * j + 1] = fmaf(wt, f.y, acc[8 * c + 2 * j + 1]);
+                                }
                             }
                         }
                     }
                 }
+                if (mode == 2) {
+    #pragma unroll
+                    for (int d = 16; d > 0; d >>= 1)
+    #pragma unroll
+                        for (int i = 0; i < 64; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], d);
+                }
+                // lane c (< 8) writes 16-byte chunk c of the 128-byte block: every lane holds
+                // the full sums after the butterfly (mode 1: lane 0 only, broadcast below)
+                if (mode == 1) {
+    #pragma unroll
+                    for (int i = 0; i < 64; ++i) acc[i] = __shfl_sync(0xffffffffu, acc[i], 0);
+                }
+                if (lane < 8) {
+                    uint32_t w[4];
+    #pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float lo = 0.f, hi = 0.f;
+    #pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c == lane) { lo = acc[8 * c + 2 * j]; hi = acc[8 * c + 2 * j + 1]; }
+                        w[j] = pack_bf16(lo, hi);
+                    }
+                    const uint32_t row = smem_u32(sB + (kb * N + n) * 128);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((lane ^ (n & 7)) << 4)), "r"(w[0]),
+                                 "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+                    if (n < nvalid && mode != 1)
+                        reinterpret_cast<uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512 + 64 * kb)[lane] =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
-            const float inv = m_inv[n];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) w[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) orow[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        } else {
+        // four tokens per warp and round, the first two pieces of each loaded
+        // together (most tokens have one or two); further pieces follow one by one
+        constexpr int kTok = 4;
+        for (int n0 = kTok * warp; n0 < N; n0 += kTok * (kUpThreads / 32)) {
+            uint4 v[kTok][2][2];
+            int mode[kTok];
+    #pragma unroll
+            for (int u = 0; u < kTok; ++u) {
+                const int n = n0 + u;
+                mode[u] = n < N ? m_mode[n] : 0;
+                const int bj = nt * N + n;
+                if (mode[u] == 1) {
+                    const uint4* src = reinterpret_cast<const uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512) + 2 * lane;
+                    v[u][0][0] = src[0];
+                    v[u][0][1] = src[1];
+                } else if (mode[u] == 2) {
+    #pragma unroll
+                    for (int i = 0; i < 2; ++i) {            // a merged token has at least two pieces
+                        const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)m_slot[n][i] * 128 + h) * 512) + 2 * lane;
+                        v[u][i][0] = src[0];
+                        v[u][i][1] = src[1];
+                    }
+                }
+            }
+    #pragma unroll
+            for (int u = 0; u < kTok; ++u) {
+                const int n = n0 + u;
+                if (n >= N) continue;
+                const int bj = nt * N + n;
+                uint4* orow = reinterpret_cast<uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512) + 2 * lane;
+                uint32_t w[8];
+                if (mode[u] == 0) {
+    #pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = 0u;
+                    if (n < nvalid) {
+                        orow[0] = make_uint4(0u, 0u, 0u, 0u);
+                        orow[1] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                } else if (mode[u] == 1) {
+                    w[0] = v[u][0][0].x; w[1] = v[u][0][0].y; w[2] = v[u][0][0].z; w[3] = v[u][0][0].w;
+                    w[4] = v[u][0][1].x; w[5] = v[u][0][1].y; w[6] = v[u][0][1].z; w[7] = v[u][0][1].w;
+                } else {
+                    float acc[16];
+    #pragma unroll
+                    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                    accumulate(acc, m_w[n][0], v[u][0][0], v[u][0][1]);
+                    accumulate(acc, m_w[n][1], v[u][1][0], v[u][1][1]);
+                    const int np = m_np[n];
+                    for (int i = 2; i < min(np, kFast); ++i) {
+                        const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)m_slot[n][i] * 128 + h) * 512) + 2 * lane;
+                        accumulate(acc, m_w[n][i], src[0], src[1]);
+                    }
+                    if (np > kFast) {              // the rest one by one
+                        const int pf = m_pf[n];
+                        const float M = m_M[n];
+                        int k = 0;
+                        for (int p = pf; ; ++p) {
+                            if (p != pf && pr.empty(p)) continue;
+                            if (k++ < kFast) continue;
+                            const int sl = PieceRange::slot(p, pf);
+                            const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)sl * 128 + h) * 512) + 2 * lane;
+                            accumulate(acc, exp2f(mg.part_lse[sl * 256 + h] - M), src[0], src[1]);
+                            if (k == np) break;
+                        }
+                    }
+                    const float inv = m_inv[n];
+    #pragma unroll
+                    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+                    orow[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    orow[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+                put_row(n, w);
+            }
         }
-        const uint32_t row = smem_u32(sB + (kb * N + n) * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((c ^ (n & 7)) << 4)), "r"(w[4 * c]),
-                         "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3]) : "memory");
+        }
     }
     fence_async_smem();      // generic-proxy writes, read by the tensor core
     __syncthreads();
@@ -518,8 +762,8 @@ int launch(K kernel, const CUtensorMap& A, const CUtensorMap& B, const ProjArgs&
 }  // namespace
 
 // absorb + q-RoPE + plan.  q_nope [BJ][H][128], W_uk [H][512][128], q_rope [BJ][H][64]
-int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32_t* first_bj, int pairs,
-                  int* launches) {
+int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32_t* first_bj,
+                  int pairs, int* launches) {
     // (sparse decode: c.n_sel / c.max_sel give the tile counts)
     const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 128);
     // The 128-wide rows are viewed as 2 groups of 64 columns (group stride 128
@@ -554,9 +798,9 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
     a.pairs = pairs;
     a.n_sel = c.n_sel;
     a.max_sel = c.max_sel;
-    a.tile_keys = (c.n_sel || !kDecodePairKernel) ? 64 : 128;
+    a.tile_keys = 64;                     // both attention kernels take 64-key tiles
     a.status = c.status;
-    const dim3 grid(H, 4, (BJ + N - 1) / N);
+    const dim3 grid(H + 1, 4, (BJ + N - 1) / N);      // column H: the plan CTA
     return launch(absorb_kernel, A, B, a, grid, 2 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches);
 }
 

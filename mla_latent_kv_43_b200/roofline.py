@@ -92,9 +92,11 @@ def step_work(w, lens: Sequence[int]) -> Dict[str, float]:
 def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_elem: int) -> float:
     """Algorithmic bytes of one launch of a kernel of the step.
 
-    The attention kernel moves the visible cache rows once per sequence, the
-    absorbed queries in and the latent outputs out; absorb/up-projection move
-    their weight and activations; append moves W_dkv, x and the new rows.
+    The attention kernel's are the cache rows it must read, once per sequence
+    (what the method's compressed cache shrinks); its absorbed queries in and
+    latent outputs out are workspace intermediates, counted separately by
+    kernel_intermediate_bytes.  Absorb/up-projection move their weight and
+    activations; append moves W_dkv, x and the new rows.
     """
     es = 4 if w.dtype == "fp32" else 2
     D = w.d_c + w.d_rope
@@ -106,7 +108,7 @@ def kernel_bytes(kernel: str, w, lens: Sequence[int], q_lat_elem: int, o_lat_ele
         keys = sum(int(L) for L in lens)
         if w.top_k:
             keys = sum(sum(min(w.top_k, int(L) - w.n_q + j + 1) for j in range(w.n_q)) for L in lens)
-        return keys * D * es + qt * H * D * q_lat_elem + qt * H * w.d_c * o_lat_elem
+        return keys * D * es
     if "absorb" in kernel:
         return H * w.d_c * w.qk_nope * es + qt * H * (w.qk_nope + w.d_rope) * es + qt * H * D * q_lat_elem
     if "upproj" in kernel:
@@ -135,4 +137,14 @@ def kernel_flops(kernel: str, w, lens: Sequence[int]) -> float:
         return 2.0 * H * (w.qk_nope + w.d_rope + w.v_dim) * visible_pairs(w, lens)
     if "prefill_expand" in kernel:
         return 2.0 * sum(int(L) for L in lens) * w.d_c * H * (w.qk_nope + w.v_dim)
+    return 0.0
+
+
+def kernel_intermediate_bytes(kernel: str, w, q_lat_elem: int, o_lat_elem: int) -> float:
+    """Workspace intermediates a launch moves besides its algorithmic bytes:
+    for the attention kernel, the absorbed queries read and the weighted
+    latents written (split-KV partials not included)."""
+    if "attend" in kernel or "core" in kernel:
+        qt = w.batch * w.n_q
+        return qt * w.heads * (w.d_c + w.d_rope) * q_lat_elem + qt * w.heads * w.d_c * o_lat_elem
     return 0.0

@@ -131,3 +131,14 @@ def test_step_work_matches_hand_counts():
     assert round(cases["v3_b1_ctx8192"][1] / 1e4) == 4307 and round(cases["v3_b32_append2"][2] / 1e8) == 757
     assert RF.cache_bytes_per_token(512, 64, 2) == 1152
     assert RF.cache_bytes_per_token(512, 64, 2, layers=61) == 70272
+
+
+def test_attention_roofline_counts_cache_rows_only():
+    """The attention kernel's algorithmic bytes are the cache rows (1152 B per
+    key of each sequence); its absorbed queries and weighted latents are
+    workspace intermediates, reported separately."""
+    w = gen.WORKLOADS["v3_b64_ragged"]
+    lens = [1000, 2048, 4096]
+    assert RF.kernel_bytes("sm100_attend", w, lens, 2, 2) == sum(lens) * 1152
+    assert RF.kernel_intermediate_bytes("sm100_attend", w, 2, 2) == w.batch * 128 * (576 + 512) * 2
+    assert RF.kernel_intermediate_bytes("sm100_upproj", w, 2, 2) == 0.0

@@ -197,3 +197,18 @@ def test_one_sequence_in_74_pieces():
     ref = oracle_out(w, host, batches=[0], heads=hs)
     err = rel_err(sampled(gpu_out(prob), [0], hs), sampled(ref, [0], hs))
     assert err <= TOL["bf16"], err
+
+
+def test_plan_for_many_query_tokens():
+    """More query tokens than the staged key-tile plan holds (600 > 512): the
+    plan takes its general path; every sequence is short and ragged, so most
+    clusters hold many whole tokens and the boundaries cut a few."""
+    rng = np.random.default_rng(17)
+    lens = tuple(int(x) for x in rng.integers(1, 300, size=600))
+    w, host = make("bf16_v3", lens=lens, capacity=300, seed=17)
+    prob = DeviceProblem(w, host)
+    prob.step()
+    torch.cuda.synchronize()
+    assert prob.get_status() == 0
+    bs = [0, 1, 255, 256, 511, 512, 513, 599]
+    check(w, host, prob, batches=bs)

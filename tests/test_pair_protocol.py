@@ -23,9 +23,9 @@ import random
 
 import pytest
 
-# key-unit slots, value-unit slots, staged units per tile (key: 3 column
-# groups each; value: 2 latent halves x 2 key halves)
-KS, VS, QB, VC = 3, 3, 3, 4
+# key-tile slots, value-unit slots, staged units per tile (one key tile;
+# value: 2 latent halves)
+KS, VS, QB, VC = 2, 4, 1, 2
 LAG = 1                               # value units of tile g wait for key unit QB (g + 1) + LAG
 
 
