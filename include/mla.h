@@ -83,14 +83,19 @@ typedef struct {
     size_t total;          /* bytes the call needs */
     size_t q_lat;          /* absorbed queries [B][n_q][H][d_c + d_rope], compute dtype */
     size_t q_lat_bytes;
-    size_t o_lat;          /* combined latent outputs [B][n_q][H][d_c], compute dtype */
+    size_t o_lat;          /* latent outputs [B][n_q][H][d_c], compute dtype: combined on the
+                              generic path; on the tensor-core path only for query tokens whose
+                              key tiles one work item covered (a token cut across items keeps its
+                              pieces in part_o / part_lse, merged after the up-projection) */
     size_t o_lat_bytes;
     size_t part_o;         /* split-KV partial latent outputs, each normalised by its own sum:
                               compute dtype on the tensor-core path, float otherwise */
     size_t part_o_bytes;
-    size_t part_lse;       /* split-KV partial log-sum-exp values, float */
+    size_t part_lse;       /* split-KV partial log-sum-exp values, float (tensor-core path: base 2,
+                              [2 splits][2 latent halves][H], the halves normalised separately) */
     size_t part_lse_bytes;
-    size_t sched;          /* device-built work schedule */
+    size_t sched;          /* device-built work schedule (tensor-core path: the key-tile prefix
+                              of the query tokens [B n_q + 1] int32, then each item's first token) */
     size_t sched_bytes;
     int32_t compute_dtype; /* enum mla_dtype of q_lat, o_lat (and part_o on the tensor-core path) */
     int32_t splits;        /* key splits per query (generic path) or work items (tensor-core path) */

@@ -241,6 +241,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         if (elect_one()) {
             tma_prefetch(&map_lat);
             tma_prefetch(&map_rope);
+            const uint64_t stream_policy = l2_policy_evict_first();
             ItemIter iter;
             iter.init(a, pair);
             Item item;
@@ -290,9 +291,12 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                                         rows[4 * g4 + 1], rows[4 * g4 + 2], rows[4 * g4 + 3]);
                         }
                     } else {
-                        // this CTA's four latent column groups in one copy (see launch_attend)
-                        tma_load_4d(st, &map_lat, &full[s], 0, key0, 4 * (int)rank, b);
-                        tma_load_3d(st + 4 * kLatBox, &map_rope, &full[s], 512 + 32 * rank, key0, b);
+                        // this CTA's four latent column groups in one copy (see launch_attend);
+                        // each cache row is read once, so it leaves L2 first, ahead of the
+                        // outputs the up-projection reads next
+                        tma_load_4d_hint(st, &map_lat, &full[s], 0, key0, 4 * (int)rank, b, stream_policy);
+                        tma_load_3d_hint(st + 4 * kLatBox, &map_rope, &full[s], 512 + 32 * rank, key0, b,
+                                         stream_policy);
                     }
                 }
             }

@@ -8,8 +8,8 @@
 // upproj  (aicassindra "Multi-head latent attention", "End-to-end flow": the
 //          value up-projection applied to the weighted latent)
 //     out[n][h][v] = sum_i W_uv[h][i][v] o_lat[n][h][i]
-//   with the split-KV log-sum-exp merge of o_lat folded into its operand
-//   assembly (tokens whose key tiles were cut across attention clusters).
+//   with the split-KV log-sum-exp merge of the tokens whose key tiles were
+//   cut across attention clusters applied after the projection (it is linear).
 //
 // Both are batched over heads: one CTA computes a 128 x N tile D = A_h B_h^T
 // with M = 128 weight rows, N = query tokens, K = 128 (absorb) or 512
@@ -332,23 +332,11 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
-// Split-KV merge of the query tokens' latent rows for head h (log-sum-exp
-// over the pieces): the pieces' normalised partial rows weighted by
-// 2^(lse_piece - lse), lse = log2 sum_piece 2^lse_piece.  A token finished
-// inside one cluster is read from o_lat as it is; a token with an invalid
-// length gives zeros.  Merged rows are also written back to o_lat (the
-// workspace's weighted latents).
-struct MergeArgs {
-    const int32_t* cum;
-    int BJ, pairs;
-    const __nv_bfloat16* part_o;
-    const float* part_lse;
-    __nv_bfloat16* o_lat;
-};
-
-// Pieces of token bj: the clusters pf..pl whose key-tile ranges it spans
-// (clusters with an empty range in between hold nothing).  Cluster p covers
-// tiles [start(p), start(p + 1)), start(p) = p T / pairs; T * pairs fits 32 bits.
+// Split-KV pieces of the query tokens (tokens whose key tiles were cut across
+// attention clusters): cluster p covers tiles [start(p), start(p + 1)),
+// start(p) = p T / pairs (T * pairs fits 32 bits); a cut token has a piece in
+// each cluster pf..pl its tiles reach (clusters with an empty range in between
+// hold nothing): the first in slot 2 pf + 1, the others in slot 2 p.
 struct PieceRange {
     int T, pairs;
     __device__ int start(int p) const { return (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)pairs); }
@@ -361,41 +349,73 @@ struct PieceRange {
         return lo;
     }
     __device__ bool empty(int p) const { return start(p) == (p + 1 < pairs ? start(p + 1) : T); }
-    // slot of the piece in cluster p of a token whose first piece is in cluster pf
-    __device__ static int slot(int p, int pf) { return p == pf ? 2 * p + 1 : 2 * p; }
+};
+
+struct UpArgs {
+    const int32_t* cum;          // [BJ + 1] key-tile prefix of the query tokens
+    int BJ, H, pairs, n_tok;     // n_tok: tokens per CTA (64)
+    int n_cols;                  // MMA N: n_tok + 2 pairs, rounded up to 16 (<= 256)
+    const float* part_lse;       // [2 pairs][2 latent halves][H], log2 domain
+    __nv_bfloat16* out;          // [BJ][H][128]
+    int32_t* status;
 };
 
 constexpr int kUpThreads = 256;
+constexpr int kUpStages = 3;
 
-// One CTA per (head, token tile of <= 64): out[n][h][v] = sum_i W_uv[h][i][v] o_lat[n][h][i].
-// A = W_uv[h] read MN-major (v contiguous), 8 k-blocks of 64 rows, all in flight
-// (an input: fetched before waiting for the attention kernel).  The B operand,
-// the tokens' weighted latents, is assembled by the whole CTA in shared memory
-// (128-byte swizzle, the layout a TMA box would give): each warp merges the
-// split-KV pieces of one token row at a time.
+// One CTA per (head h, tile of 64 query tokens):
+//     out[n][h][v] = sum_i W_uv[h][i][v] o[n][h][i]
+// where o is the token's weighted latent row: o_lat as written by the
+// attention kernel for a token finished inside one cluster, and for a token
+// cut across clusters the log-sum-exp merge of its pieces' normalised
+// partial rows part_o[slot][h] with weights 2^(lse_piece - lse) (per latent
+// half: the two halves of a piece were normalised by the two CTAs of its
+// cluster).  The merge is moved past the projection, which is linear: the
+// B operand holds the tile's o_lat rows and every piece row of head h as
+// they are (two tensor copies per 64-column k-block, no arithmetic), the
+// tensor cores project all of them, D0 over latent columns [0, 256) and D1
+// over [256, 512), and the epilogue combines the 128-wide projected rows of a
+// cut token's pieces with their weights.
+//
+// A = W_uv[h] read MN-major (v contiguous): four 32 KB copies of 128 latent
+// rows, fetched before waiting for the attention kernel (an input).  B: a
+// ring of kUpStages k-blocks of n_cols rows x 128 bytes (128-byte swizzle).
+// Warp 0 loads, warp 1 issues the MMAs; meanwhile warps 2-7 find each
+// token's pieces and weights.  TMEM: D0 at column 0, D1 at column 256.
 __global__ void __launch_bounds__(kUpThreads, 1)
-upproj_kernel(const __grid_constant__ CUtensorMap mapA, ProjArgs a, MergeArgs mg) {
+upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapO,
+              const __grid_constant__ CUtensorMap mapP, UpArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[4], done;
+    __shared__ uint64_t fullA[4], fullB[kUpStages], emptyB[kUpStages], done;
     __shared__ uint32_t tmem_base;
     __shared__ int flag;
-    const int h = blockIdx.x, nt = blockIdx.z;
+    // per piece slot s (column n_tok + s of D): the tile-local token it belongs
+    // to (-1: none in this tile) and its weights for the two latent halves
+    __shared__ int slot_tok[256];
+    __shared__ float slot_w[2][256];
+    __shared__ float slot_lse[2][256];
+    // per token of the tile: 0 invalid length (zeros), 1 finished in one
+    // cluster, 2 cut (merge its pieces); first and last slot of its pieces
+    __shared__ int tok_mode[64], tok_s0[64], tok_s1[64];
+    const int h = blockIdx.x, n0 = blockIdx.z * a.n_tok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int N = a.n_tile;
-    const uint32_t ncols = tmem_cols_for(N);
-    // W_uv[h]: four 32 KB blocks of 128 latent rows, each [2 value-column groups][128 rows][64];
-    // then the token operand: [8 k-blocks of 64 latent columns][N rows][64]
+    const int N = a.n_cols, S = 2 * a.pairs;
     constexpr int kWBlock = 32768;
+    const int kBStage = N * 128;
     uint8_t* sB = smem + 4 * kWBlock;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&fullA[i], 1);
+        for (int i = 0; i < kUpStages; ++i) {
+            mbar_init(&fullB[i], 1);
+            mbar_init(&emptyB[i], 1);
+        }
         mbar_init(&done, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_base, ncols);
+        tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -404,340 +424,188 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, ProjArgs a, MergeArgs mg
     const uint32_t tmem = tmem_base;
 
     if (warp == 0 && elect_one()) {
-        // one copy per 128 latent rows (both 64-column groups of v): a single
-        // thread issues about one tensor copy per 0.3 us, so few large ones
+        // W_uv[h]: one copy per 128 latent rows (both 64-column groups of v)
         for (int j = 0; j < 4; ++j) {
-            mbar_expect_tx(&full[j], kWBlock);
-            tma_load_3d(smem + j * kWBlock, &mapA, &full[j], 0, h * 512 + j * 128, 0);
+            mbar_expect_tx(&fullA[j], kWBlock);
+            tma_load_3d(smem + j * kWBlock, &mapA, &fullA[j], 0, h * 512 + j * 128, 0);
         }
     }
     __syncwarp();
     grid_dep_wait();         // the attention kernel's latents and pieces
     grid_dep_trigger();
 
-    const int nvalid = min(N, a.BJ - nt * N);
-    {
-        // B operand: row n (token nt * N + n), 64-column block kb at sB + kb * N * 128,
-        // 16-byte chunk c of the 128-byte row at ((c ^ (n & 7)) << 4).
-        // Phase 1: the pieces (slots) of each token and their log-sum-exp.  Many
-        // tokens (the usual case: one or two pieces each): one thread per token, up
-        // to kFast pieces' log-sum-exps loaded together.  Few tokens (typically
-        // cut into many pieces): one warp per token, lanes over pieces.
-        // Phase 2 (see below) then assembles the merged rows.
-        constexpr int kFast = 4;
-        const bool few = nvalid <= 8;
-        __shared__ int m_mode[64], m_np[64], m_pf[64], m_pl[64], m_slot[64][kFast];   // mode 0: zeros, 1: o_lat as is, 2: merge
-        __shared__ float m_w[64][kFast], m_M[64], m_inv[64];
-        const PieceRange pr{mg.cum[mg.BJ], mg.pairs};
-        auto token_range = [&](int n, int& mode, int& pf, int& pl) {
-            mode = 0;
-            pf = 0;
-            pl = -1;
-            if (n >= nvalid) return;
-            const int bj = nt * N + n;
-            const int c0 = mg.cum[bj], c1 = mg.cum[bj + 1];
-            if (c1 == c0) return;
-            pf = pr.pair_of(c0);
-            pl = pr.pair_of(c1 - 1);
-            mode = pf == pl ? 1 : 2;
-        };
-        if (few) {
-            if (warp < nvalid) {
-                const int n = warp;
-                int mode, pf, pl;
-                token_range(n, mode, pf, pl);
-                float M = -INFINITY, S = 0.f;
-                if (mode == 2) {
-                    for (int p0 = pf; p0 <= pl; p0 += 32) {
-                        const int p = p0 + lane;
-                        if (p <= pl && (p == pf || !pr.empty(p))) M = fmaxf(M, mg.part_lse[PieceRange::slot(p, pf) * 256 + h]);
-                    }
-    #pragma unroll
-                    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
-                    for (int p0 = pf; p0 <= pl; p0 += 32) {
-                        const int p = p0 + lane;
-                        if (p <= pl && (p == pf || !pr.empty(p))) S += exp2f(mg.part_lse[PieceRange::slot(p, pf) * 256 + h] - M);
-                    }
-    #pragma unroll
-                    for (int d = 16; d > 0; d >>= 1) S += __shfl_xor_sync(0xffffffffu, S, d);
+    if (warp == 0) {
+        if (elect_one()) {
+            // k-block kb: the tile's 64 o_lat rows, then all 2 pairs piece rows
+            // (rows past the tokens or the slots read as zeros)
+            for (int kb = 0; kb < 8; ++kb) {
+                const int st = kb % kUpStages;
+                if (kb >= kUpStages && !mbar_wait(&emptyB[st], ((kb / kUpStages) - 1) & 1, nullptr)) {
+                    set_status(a.status, MLA_ERR_TIMEOUT);
+                    break;
                 }
-                if (lane == 0) {
-                    m_mode[n] = mode;
-                    m_pf[n] = pf;
-                    m_pl[n] = pl;
-                    m_M[n] = M;
-                    m_inv[n] = mode == 2 ? 1.f / S : 0.f;
-                }
-            }
-        } else if (threadIdx.x < N) {
-            const int n = threadIdx.x;
-            int mode, np = 0, pf, pl;
-            token_range(n, mode, pf, pl);
-            float M = -INFINITY, S = 0.f;
-            if (mode == 2) {
-                int sl[kFast];
-                for (int p = pf; p <= pl; ++p) {
-                    if (p != pf && pr.empty(p)) continue;
-                    if (np < kFast) sl[np] = PieceRange::slot(p, pf);
-                    ++np;
-                }
-                float lse[kFast];
-    #pragma unroll
-                for (int i = 0; i < kFast; ++i) lse[i] = i < np ? mg.part_lse[sl[i] * 256 + h] : -INFINITY;
-    #pragma unroll
-                for (int i = 0; i < kFast; ++i) M = fmaxf(M, lse[i]);
-                if (np > kFast) {            // more pieces: the rest one by one
-                    int k = 0;
-                    for (int p = pf; p <= pl; ++p) {
-                        if (p != pf && pr.empty(p)) continue;
-                        if (k++ >= kFast) M = fmaxf(M, mg.part_lse[PieceRange::slot(p, pf) * 256 + h]);
-                    }
-                }
-    #pragma unroll
-                for (int i = 0; i < kFast; ++i) {
-                    const float w = i < np ? exp2f(lse[i] - M) : 0.f;
-                    S += w;
-                    m_w[n][i] = w;
-                    m_slot[n][i] = i < np ? sl[i] : 0;
-                }
-                if (np > kFast) {
-                    int k = 0;
-                    for (int p = pf; p <= pl; ++p) {
-                        if (p != pf && pr.empty(p)) continue;
-                        if (k++ >= kFast) S += exp2f(mg.part_lse[PieceRange::slot(p, pf) * 256 + h] - M);
-                    }
-                }
-            }
-            m_mode[n] = mode;
-            m_np[n] = np;
-            m_pf[n] = pf;
-            m_pl[n] = pl;
-            m_M[n] = M;
-            m_inv[n] = mode == 2 ? 1.f / S : 0.f;
-        }
-        __syncthreads();
-        // row n of the B operand: 64-column block kb at sB + (kb * N + n) * 128, 16-byte chunk c at ((c ^ (n & 7)) << 4);
-        // lane l holds columns [16 l, 16 l + 16): block l / 4, chunks 2 (l % 4) and 2 (l % 4) + 1
-        auto put_row = [&](int n, const uint32_t (&w)[8]) {
-            const int kb = lane >> 2, c = (lane & 3) * 2;
-            const uint32_t row = smem_u32(sB + (kb * N + n) * 128);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((c ^ (n & 7)) << 4)), "r"(w[0]), "r"(w[1]),
-                         "r"(w[2]), "r"(w[3]) : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((c + 1) ^ (n & 7)) << 4)), "r"(w[4]),
-                         "r"(w[5]), "r"(w[6]), "r"(w[7]) : "memory");
-        };
-        auto accumulate = [&](float (&acc)[16], float wt, const uint4& v0, const uint4& v1) {
-            const uint32_t pw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
-                acc[2 * j] = fmaf(wt, f.x, acc[2 * j]);
-                acc[2 * j + 1] = fmaf(wt, f.y, acc[2 * j + 1]);
-            }
-        };
-        if (few) {
-            // Few tokens: warp w assembles 64-column block w of every token row, lanes
-            // over pieces (each lane one piece's 128-byte segment, weighted), then a
-            // butterfly sum across the lanes; rows of tokens past nvalid stay zero.
-            const int kb = warp;
-            for (int n = 0; n < N; ++n) {
-                const int mode = n < nvalid ? m_mode[n] : 0;
-                const int bj = nt * N + n;
-                float acc[64];
-    #pragma unroll
-                for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-                if (mode == 1 && lane == 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512 + 64 * kb);
-    #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = src[c];
-                        const uint32_t pw[4] = {v.x, v.y, v.z, v.w};
-    #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
-                            acc[8 * c + 2 * j] = f.x;
-                            acc[8 * c + 2 * j + 1] = f.y;
-                        }
-                    }
-                } else if (mode == 2) {
-                    const int pf = m_pf[n], pl = m_pl[n];
-                    const float M = m_M[n], inv = m_inv[n];
-                    for (int p0 = pf; p0 <= pl; p0 += 32) {
-                        const int p = p0 + lane;
-                        if (p <= pl && (p == pf || !pr.empty(p))) {
-                            const int sl = PieceRange::slot(p, pf);
-                            const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)sl * 128 + h) * 512 + 64 * kb);
-                            uint4 v[8];
-    #pragma unroll
-                            for (int c = 0; c < 8; ++c) v[c] = src[c];
-                            const float wt = exp2f(mg.part_lse[sl * 256 + h] - M) * inv;
-    #pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                const uint32_t pw[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-    #pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pw[j]));
-                                    acc[8 * c + 2 * j] = fmaf(wt, f.x, acc[8 * c + 2 * j]);
-                                    acc[8 * c + 2 * j + 1] = fmaf(wt, f.y, acc[8 * c + 2 * j + 1]);
-                                }
-                            }
-                        }
-                    }
-                }
-                if (mode == 2) {
-    #pragma unroll
-                    for (int d = 16; d > 0; d >>= 1)
-    #pragma unroll
-                        for (int i = 0; i < 64; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], d);
-                }
-                // lane c (< 8) writes 16-byte chunk c of the 128-byte block: every lane holds
-                // the full sums after the butterfly (mode 1: lane 0 only, broadcast below)
-                if (mode == 1) {
-    #pragma unroll
-                    for (int i = 0; i < 64; ++i) acc[i] = __shfl_sync(0xffffffffu, acc[i], 0);
-                }
-                if (lane < 8) {
-                    uint32_t w[4];
-    #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float lo = 0.f, hi = 0.f;
-    #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            if (c == lane) { lo = acc[8 * c + 2 * j]; hi = acc[8 * c + 2 * j + 1]; }
-                        w[j] = pack_bf16(lo, hi);
-                    }
-                    const uint32_t row = smem_u32(sB + (kb * N + n) * 128);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((lane ^ (n & 7)) << 4)), "r"(w[0]),
-                                 "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
-                    if (n < nvalid && mode != 1)
-                        reinterpret_cast<uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512 + 64 * kb)[lane] =
-                            make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
-        } else {
-        // four tokens per warp and round, the first two pieces of each loaded
-        // together (most tokens have one or two); further pieces follow one by one
-        constexpr int kTok = 4;
-        for (int n0 = kTok * warp; n0 < N; n0 += kTok * (kUpThreads / 32)) {
-            uint4 v[kTok][2][2];
-            int mode[kTok];
-    #pragma unroll
-            for (int u = 0; u < kTok; ++u) {
-                const int n = n0 + u;
-                mode[u] = n < N ? m_mode[n] : 0;
-                const int bj = nt * N + n;
-                if (mode[u] == 1) {
-                    const uint4* src = reinterpret_cast<const uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512) + 2 * lane;
-                    v[u][0][0] = src[0];
-                    v[u][0][1] = src[1];
-                } else if (mode[u] == 2) {
-    #pragma unroll
-                    for (int i = 0; i < 2; ++i) {            // a merged token has at least two pieces
-                        const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)m_slot[n][i] * 128 + h) * 512) + 2 * lane;
-                        v[u][i][0] = src[0];
-                        v[u][i][1] = src[1];
-                    }
-                }
-            }
-    #pragma unroll
-            for (int u = 0; u < kTok; ++u) {
-                const int n = n0 + u;
-                if (n >= N) continue;
-                const int bj = nt * N + n;
-                uint4* orow = reinterpret_cast<uint4*>(mg.o_lat + ((int64_t)bj * 128 + h) * 512) + 2 * lane;
-                uint32_t w[8];
-                if (mode[u] == 0) {
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i) w[i] = 0u;
-                    if (n < nvalid) {
-                        orow[0] = make_uint4(0u, 0u, 0u, 0u);
-                        orow[1] = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                } else if (mode[u] == 1) {
-                    w[0] = v[u][0][0].x; w[1] = v[u][0][0].y; w[2] = v[u][0][0].z; w[3] = v[u][0][0].w;
-                    w[4] = v[u][0][1].x; w[5] = v[u][0][1].y; w[6] = v[u][0][1].z; w[7] = v[u][0][1].w;
-                } else {
-                    float acc[16];
-    #pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-                    accumulate(acc, m_w[n][0], v[u][0][0], v[u][0][1]);
-                    accumulate(acc, m_w[n][1], v[u][1][0], v[u][1][1]);
-                    const int np = m_np[n];
-                    for (int i = 2; i < min(np, kFast); ++i) {
-                        const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)m_slot[n][i] * 128 + h) * 512) + 2 * lane;
-                        accumulate(acc, m_w[n][i], src[0], src[1]);
-                    }
-                    if (np > kFast) {              // the rest one by one
-                        const int pf = m_pf[n];
-                        const float M = m_M[n];
-                        int k = 0;
-                        for (int p = pf; ; ++p) {
-                            if (p != pf && pr.empty(p)) continue;
-                            if (k++ < kFast) continue;
-                            const int sl = PieceRange::slot(p, pf);
-                            const uint4* src = reinterpret_cast<const uint4*>(mg.part_o + ((int64_t)sl * 128 + h) * 512) + 2 * lane;
-                            accumulate(acc, exp2f(mg.part_lse[sl * 256 + h] - M), src[0], src[1]);
-                            if (k == np) break;
-                        }
-                    }
-                    const float inv = m_inv[n];
-    #pragma unroll
-                    for (int i = 0; i < 8; ++i) w[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-                    orow[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    orow[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                }
-                put_row(n, w);
+                uint8_t* dst = sB + st * kBStage;
+                mbar_expect_tx(&fullB[st], (a.n_tok + S) * 128);
+                tma_load_4d(dst, &mapO, &fullB[st], 0, n0, kb, h);
+                tma_load_4d(dst + a.n_tok * 128, &mapP, &fullB[st], 0, 0, kb, h);
             }
         }
-        }
-    }
-    fence_async_smem();      // generic-proxy writes, read by the tensor core
-    __syncthreads();
-
-    if (warp == 1) {
+        __syncwarp();
+    } else if (warp == 1) {
         // whole warp, one elected lane issues (warp-uniform descriptors)
         const uint32_t idesc = idesc_bf16(128, N, true, false);
         const uint64_t da = sdesc(smem_u32(smem), kWBlock / 2, 1024, kSwizzle128);   // v groups 16 KB apart
         const uint64_t db = sdesc(smem_u32(sB), 16, 1024, kSwizzle128);
-        for (int kb = 0; kb < 8; ++kb) {
-            if ((kb & 1) == 0) {
-                int ready = 0;
-                if (lane == 0) ready = mbar_wait(&full[kb >> 1], 0, nullptr) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, ready, 0)) break;
-                tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < 8 && ok; ++kb) {
+            const int st = kb % kUpStages;
+            int ready = 0;
+            if (lane == 0)
+                ready = ((kb & 1) || mbar_wait(&fullA[kb >> 1], 0, nullptr)) &&
+                        mbar_wait(&fullB[st], (kb / kUpStages) & 1, nullptr);
+            ok = __shfl_sync(0xffffffffu, ready, 0) != 0;
+            if (!ok) {
+                if (lane == 0) set_status(a.status, MLA_ERR_TIMEOUT);
+                break;
             }
+            tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_ss_w(tmem, sdesc_add(da, (kb >> 1) * kWBlock + (kb & 1) * 8192 + ks * 2048),
-                         sdesc_add(db, kb * N * 128 + ks * 32), idesc, (kb | ks) ? 1u : 0u);
+                mma_ss_w(tmem + (kb < 4 ? 0u : 256u), sdesc_add(da, (kb >> 1) * kWBlock + (kb & 1) * 8192 + ks * 2048),
+                         sdesc_add(db, st * kBStage + ks * 32), idesc, ((kb & 3) | ks) ? 1u : 0u);
+            mma_commit_w(&emptyB[st]);
         }
         mma_commit_w(&done);
+    } else {
+        // ---- pieces and weights (192 threads)
+        const int t = threadIdx.x - 64;
+        for (int s = t; s < 256; s += 192) slot_tok[s] = -1;
+        named_barrier(1, 192);
+        const PieceRange pr{a.cum[a.BJ], a.pairs};
+        if (t < a.n_tok) {
+            // one thread per token: its mode and the slots of its pieces
+            const int n = n0 + t;
+            int mode = 0, s0 = 0, s1 = -1;
+            if (n < a.BJ) {
+                const int c0 = a.cum[n], c1 = a.cum[n + 1];
+                if (c1 > c0) {
+                    const int pf = pr.pair_of(c0), pl = pr.pair_of(c1 - 1);
+                    mode = pf == pl ? 1 : 2;
+                    if (mode == 2) {
+                        s0 = 2 * pf + 1;
+                        s1 = 2 * pl;
+                        slot_tok[s0] = t;
+                        for (int p = pf + 1; p <= pl; ++p)
+                            if (!pr.empty(p)) slot_tok[2 * p] = t;
+                    }
+                }
+            }
+            tok_mode[t] = mode;
+            tok_s0[t] = s0;
+            tok_s1[t] = s1;
+        }
+        named_barrier(1, 192);
+        // the pieces' log2-sum-exps, all loads at once
+        for (int s = t; s < S; s += 192) {
+            if (slot_tok[s] >= 0) {
+                slot_lse[0][s] = __ldcg(a.part_lse + (2 * s) * a.H + h);
+                slot_lse[1][s] = __ldcg(a.part_lse + (2 * s + 1) * a.H + h);
+            }
+        }
+        named_barrier(1, 192);
+        // each slot's weights for the two latent halves: w = 2^(lse - M) / sum over
+        // the token's pieces of 2^(lse' - M), M their maximum (one thread per
+        // slot, each scanning its token's slot range: no cross-thread steps)
+        for (int s = t; s < S; s += 192) {
+            const int tt = slot_tok[s];
+            if (tt < 0) continue;
+            const int s0 = tok_s0[tt], s1 = tok_s1[tt];
+            float M0 = -INFINITY, M1 = -INFINITY;
+            for (int u = s0; u <= s1; ++u) {
+                if (slot_tok[u] != tt) continue;
+                M0 = fmaxf(M0, slot_lse[0][u]);
+                M1 = fmaxf(M1, slot_lse[1][u]);
+            }
+            float S0 = 0.f, S1 = 0.f;
+            for (int u = s0; u <= s1; ++u) {
+                if (slot_tok[u] != tt) continue;
+                S0 += exp2f(slot_lse[0][u] - M0);
+                S1 += exp2f(slot_lse[1][u] - M1);
+            }
+            slot_w[0][s] = exp2f(slot_lse[0][s] - M0) / S0;
+            slot_w[1][s] = exp2f(slot_lse[1][s] - M1) / S1;
+        }
     }
-    __syncwarp();
+    __syncthreads();         // piece tables complete
 
     if (block_wait(&done, &flag, a.status)) {
-        // stage out[n][h][0:128] as [n][128] bf16 in smem, then 16-byte stores;
-        // warps w and w + 4 share lane quarter w & 3 and split the token columns
+        // Projected rows -> stage[n][128] bf16 (the B ring is free now).  Warps
+        // w and w + 4 share TMEM lane quarter w & 3 (v = 32 (w & 3) + lane):
+        // warps 0-3 take the tokens finished in one cluster (D0 + D1 of their own
+        // column), warps 4-7 the cut tokens (their pieces' columns, weighted).
         tc_fence_after();
-        __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(smem);
-        const int q = warp & 3, m = q * 32 + lane;
-        for (int c0 = (warp >> 2) * 16; c0 < N; c0 += 32) {
-            uint32_t r[16];
-            tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c0, r);
-            tmem_wait_ld();
+        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sB);
+        const int q = warp & 3, v = q * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        // Both loops are branch-free per column: each lane holds one column's
+        // token data and the loop takes it by shuffle, and stores that are not
+        // wanted go to a dummy row, so no iteration waits on a load or a branch.
+        __nv_bfloat16* dummy = stage + 64 * 128;   // past the tile's 64 token rows
+        if (warp < 4) {
+            for (int c0 = 0; c0 < a.n_tok; c0 += 32) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + c0, r0);
+                tmem_ld32(tmem + lane_off + 256 + c0, r1);
+                const int my_mode = tok_mode[c0 + lane];
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 16; ++c) stg[(c0 + c) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[c]));
+                for (int i = 0; i < 32; ++i) {
+                    const int mode = __shfl_sync(0xffffffffu, my_mode, i);
+                    const float val = mode == 1 ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : 0.f;
+                    __nv_bfloat16* dst = mode == 2 ? dummy + v : stage + (c0 + i) * 128 + v;
+                    *dst = __float2bfloat16_rn(val);
+                }
+            }
+        } else {
+            // slot columns in order; a cut token's pieces are consecutive slots
+            // (unused slots between them hold anything and are skipped)
+            int prev = -1;
+            float acc = 0.f;
+            for (int c0 = 0; c0 < S; c0 += 32) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + a.n_tok + c0, r0);
+                tmem_ld32(tmem + lane_off + 256 + a.n_tok + c0, r1);
+                const int my_tok = c0 + lane < S ? slot_tok[c0 + lane] : -1;
+                const float my_w0 = my_tok >= 0 ? slot_w[0][c0 + lane] : 0.f;
+                const float my_w1 = my_tok >= 0 ? slot_w[1][c0 + lane] : 0.f;
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int tok = __shfl_sync(0xffffffffu, my_tok, i);
+                    const float w0 = __shfl_sync(0xffffffffu, my_w0, i);
+                    const float w1 = __shfl_sync(0xffffffffu, my_w1, i);
+                    const float pv = fmaf(w0, __uint_as_float(r0[i]), w1 * __uint_as_float(r1[i]));
+                    const float val = tok >= 0 ? pv : 0.f;
+                    const bool starts = tok >= 0 && tok != prev;    // a new token's first piece
+                    __nv_bfloat16* dst = (starts && prev >= 0) ? stage + prev * 128 + v : dummy + v;
+                    *dst = __float2bfloat16_rn(acc);                // the finished token's row
+                    acc = starts ? val : acc + val;
+                    prev = tok >= 0 ? tok : prev;
+                }
+            }
+            if (prev >= 0) stage[prev * 128 + v] = __float2bfloat16_rn(acc);
         }
         __syncthreads();
+        const int nvalid = min(a.n_tok, a.BJ - n0);
         for (int i = threadIdx.x; i < nvalid * 16; i += kUpThreads) {
             const int n = i >> 4, c = i & 15;
-            reinterpret_cast<uint4*>(a.out + ((int64_t)(nt * N + n) * a.H + h) * 128)[c] =
-                reinterpret_cast<const uint4*>(stg + n * 128)[c];
+            reinterpret_cast<uint4*>(a.out + ((int64_t)(n0 + n) * a.H + h) * 128)[c] =
+                reinterpret_cast<const uint4*>(stage + n * 128)[c];
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, ncols);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 int round_n(int bj, int cap) {
@@ -809,8 +677,11 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
 // W_uv [H][512][128], out [BJ][H][128]
 int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16* part_o, const float* part_lse,
                   const int32_t* cum, int pairs, int* launches) {
-    const int BJ = c.batch * c.n_q, H = c.d.heads, N = round_n(BJ, 64);
-    CUtensorMap A;
+    const int BJ = c.batch * c.n_q, H = c.d.heads;
+    constexpr int kTok = 64;
+    const int n_cols = (kTok + 2 * pairs + 15) / 16 * 16;
+    if (n_cols > 256) return MLA_ERR_UNSUPPORTED;
+    CUtensorMap A, O, P;
     {
         // W_uv rows [H * 512][128] viewed as (column in group, row, group of 64 columns):
         // one box = 128 rows x both groups, landing group-major
@@ -818,20 +689,37 @@ int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16
         const uint32_t box[3] = {64, 128, 2};
         if (!make_map(&A, c.W_uv, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
-    ProjArgs a{};
+    {
+        // o_lat [BJ][H][512] as (column in group, token, group of 64 columns, head):
+        // one box = 64 tokens of one group and head
+        const uint64_t dims[4] = {64, (uint64_t)BJ, 8, (uint64_t)H};
+        const uint64_t str[3] = {(uint64_t)H * 512 * 2, 64 * 2, 512 * 2};
+        const uint32_t box[4] = {64, (uint32_t)kTok, 1, 1};
+        if (!make_map(&O, o_lat, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        // part_o [2 pairs][H][512], the same view over piece slots: one box = every slot
+        const uint64_t dims[4] = {64, (uint64_t)(2 * pairs), 8, (uint64_t)H};
+        const uint64_t str[3] = {(uint64_t)H * 512 * 2, 64 * 2, 512 * 2};
+        const uint32_t box[4] = {64, (uint32_t)(2 * pairs), 1, 1};
+        if (!make_map(&P, part_o, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    UpArgs a{};
+    a.cum = cum;
     a.BJ = BJ;
     a.H = H;
-    a.n_q = c.n_q;
-    a.n_tile = N;
+    a.pairs = pairs;
+    a.n_tok = kTok;
+    a.n_cols = n_cols;
+    a.part_lse = part_lse;
     a.out = (__nv_bfloat16*)c.out;
     a.status = c.status;
-    MergeArgs mg{cum, BJ, pairs, part_o, part_lse, o_lat};
-    const dim3 grid(H, 1, (BJ + N - 1) / N);
-    const size_t smem = 4 * 32768 + 8 * N * 128 + 1024;
+    const dim3 grid(H, 1, (BJ + kTok - 1) / kTok);
+    const size_t smem = 4 * 32768 + (size_t)kUpStages * n_cols * 128 + 1024;
     if (cudaFuncSetAttribute(upproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(c.stream, "sm100_upproj");
-    const cudaError_t e = launch_pdl(upproj_kernel, grid, dim3(kUpThreads), smem, c.stream, A, a, mg);
+    const cudaError_t e = launch_pdl(upproj_kernel, grid, dim3(kUpThreads), smem, c.stream, A, O, P, a);
     prof_end(c.stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;

@@ -22,6 +22,38 @@ SMALL = dict(heads=3, d_c=8, d_rope=4, qk_nope=6, v_dim=5)
 V3 = dict(heads=128, d_c=512, d_rope=64, qk_nope=128, v_dim=128)
 
 
+def merge_pieces(prob, o_lat, BJ, H, d_c):
+    """The tensor-core path leaves a query token whose key tiles were cut across
+    work items as pieces (normalised partial rows, one log2-sum-exp per latent
+    half); merge them here as the up-projection does after projecting.  Item p
+    covers tiles [p T / P, (p + 1) T / P); a cut token's first piece is in slot
+    2 pf + 1, its later ones in slot 2 p."""
+    P = prob.layout["splits"]
+    cum = prob.workspace_view("sched", (-1,), torch.int32)[: BJ + 1].cpu().numpy().astype(np.int64)
+    part_o = prob.workspace_view("part_o", (2 * P, H, d_c), torch.bfloat16).double().cpu().numpy()
+    lse = prob.workspace_view("part_lse", (2 * P, 2, H), torch.float32).double().cpu().numpy()
+    T = int(cum[BJ])
+    start = [p * T // P for p in range(P + 1)]
+    pair_of = lambda t: max(p for p in range(P) if start[p] <= t)  # noqa: E731
+    out = o_lat.copy()
+    for n in range(BJ):
+        c0, c1 = cum[n], cum[n + 1]
+        if c1 == c0:
+            continue
+        pf, pl = pair_of(c0), pair_of(c1 - 1)
+        if pf == pl:
+            continue
+        slots = [2 * pf + 1] + [2 * p for p in range(pf + 1, pl + 1) if start[p] < start[p + 1]]
+        half = d_c // 2
+        for r in range(2):
+            lw = lse[slots, r, :]                                   # [pieces][H]
+            wts = np.exp2(lw - lw.max(axis=0))
+            wts /= wts.sum(axis=0)
+            out[n, :, r * half:(r + 1) * half] = np.einsum("ph,phc->hc", wts,
+                                                           part_o[slots][:, :, r * half:(r + 1) * half])
+    return out
+
+
 def run_and_compare(dtype, g, lens, n_q, splits, heads):
     w = gen.tiny(dtype, lens=lens, n_q=n_q, seed=11, latent_rms_norm=(g is V3), **g)
     host = gen.generate(w)
@@ -34,6 +66,8 @@ def run_and_compare(dtype, g, lens, n_q, splits, heads):
     BJ = w.batch * n_q
     q_lat = prob.workspace_view("q_lat", (BJ, w.heads, w.d), cdt).double().cpu().numpy()
     o_lat = prob.workspace_view("o_lat", (BJ, w.heads, w.d_c), cdt).double().cpu().numpy()
+    if L["compute_dtype"] == 0:
+        o_lat = merge_pieces(prob, o_lat, BJ, w.heads, w.d_c)
     out = gpu_out(prob)
     k_rot = O.rope_cache(host["k_rope"], host["seq_lens"])
     ref_out, inter = O.decode_absorbed(host["q_nope"], host["q_rope"], host["W_uk"], host["W_uv"],
