@@ -89,13 +89,17 @@ typedef struct {
                               pieces in part_o / part_lse, merged after the up-projection) */
     size_t o_lat_bytes;
     size_t part_o;         /* split-KV partial latent outputs, each normalised by its own sum:
-                              compute dtype on the tensor-core path, float otherwise */
+                              compute dtype on the tensor-core path, float otherwise.  On the
+                              tensor-core path head-major and blocked by 64 latent columns:
+                              element (piece slot s, head h, column c) at
+                              ((h * d_c / 64 + c / 64) * 2 splits + s) * 64 + c % 64 */
     size_t part_o_bytes;
     size_t part_lse;       /* split-KV partial log-sum-exp values, float (tensor-core path: base 2,
-                              [2 splits][2 latent halves][H], the halves normalised separately) */
+                              [H][2 splits][2 latent halves], the halves normalised separately) */
     size_t part_lse_bytes;
-    size_t sched;          /* device-built work schedule (tensor-core path: the key-tile prefix
-                              of the query tokens [B n_q + 1] int32, then each item's first token) */
+    size_t sched;          /* device-built work schedule (tensor-core path, int32: the key-tile
+                              prefix of the query tokens [B n_q + 1], each item's first token
+                              [splits], each piece slot's query token [2 splits], -1 if unused) */
     size_t sched_bytes;
     int32_t compute_dtype; /* enum mla_dtype of q_lat, o_lat (and part_o on the tensor-core path) */
     int32_t splits;        /* key splits per query (generic path) or work items (tensor-core path) */

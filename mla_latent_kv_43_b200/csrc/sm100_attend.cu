@@ -77,8 +77,12 @@ struct AttnArgs {
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* o_lat;         // [BJ][128][512]
-    __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
-    float* part_lse;              // [2 * pairs][2 latent halves][128], log2 domain
+    // split-KV pieces, normalised per piece, head-major and blocked by 64
+    // latent columns: element (slot, head h, column c) at
+    // ((h * 8 + c / 64) * 2 pairs + slot) * 64 + c % 64, so that one head's
+    // pieces of a column block are contiguous
+    __nv_bfloat16* part_o;
+    float* part_lse;              // [128 heads][2 * pairs][2 latent halves], log2 domain
     int32_t* status;
     // sparse decode: the selected slots of each query token and their count
     const int32_t* sel;           // [BJ][max_sel]
@@ -691,9 +695,8 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 // bf16, 32 columns (64 bytes) per row and block: the normalised output of a
                 // token finished here, or this piece's normalised partial (plus its
                 // log2-sum-exp) for the combine step
-                __nv_bfloat16* dst = item.slot < 0 ? a.o_lat + (int64_t)item.bj * 128 * 512
-                                                   : a.part_o + (int64_t)item.slot * 128 * 512;
-                char* base = reinterpret_cast<char*>(dst + 256 * rank + 128 * grp);
+                char* base = reinterpret_cast<char*>(a.o_lat + (int64_t)item.bj * 128 * 512 + 256 * rank + 128 * grp);
+                const int S2 = 2 * a.pairs;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
@@ -703,9 +706,17 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         w[i] = pack_bf16(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                    put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 32 * c) * 2; });
+                    if (item.slot < 0) {
+                        put_rows(w, [&](int row) { return base + ((int64_t)row * 512 + 32 * c) * 2; });
+                    } else {
+                        const int kb = 4 * (int)rank + 2 * grp + (c >> 1);
+                        put_rows(w, [&](int row) {
+                            return reinterpret_cast<char*>(a.part_o + (((int64_t)row * 8 + kb) * S2 + item.slot) * 64 +
+                                                           32 * (c & 1));
+                        });
+                    }
                 }
-                if (item.slot >= 0 && grp == 0) a.part_lse[(item.slot * 2 + rank) * 128 + h] = mf + __log2f(lsum);
+                if (item.slot >= 0 && grp == 0) a.part_lse[(h * S2 + item.slot) * 2 + rank] = mf + __log2f(lsum);
             }
             // the next item's first O GEMM (accumulate = 0) may start only after both
             // groups' reads of this item's O

@@ -96,8 +96,10 @@ struct PairArgs {
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
     __nv_bfloat16* o_lat;         // [BJ][128][512]
-    __nv_bfloat16* part_o;        // [2 * pairs][128][512], normalised per piece
-    float* part_lse;              // [2 * pairs][2 latent halves][128], log2 domain
+    // split-KV pieces, normalised per piece: element (slot, head h, column c) at
+    // ((h * 8 + c / 64) * 2 pairs + slot) * 64 + c % 64
+    __nv_bfloat16* part_o;
+    float* part_lse;              // [128 heads][2 * pairs][2 latent halves], log2 domain
     int32_t* status;
 };
 
@@ -625,17 +627,20 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                     const int tt = 32 * q + rr;
                     const int hh = 64 * (int)rank + (tt & 63);
                     const uint4 v = ld_shared_u4(scr + rr * 64 + ((pc ^ (rr & 3)) << 4));
-                    __nv_bfloat16* rowp = (item.slot < 0 ? a.o_lat + ((int64_t)item.bj * 128 + hh) * 512
-                                                         : a.part_o + ((int64_t)item.slot * 128 + hh) * 512);
-                    *reinterpret_cast<uint4*>(rowp + 256 * cv + 128 * (tt >> 6) + 32 * sub + 8 * pc) = v;
+                    const int col = 256 * cv + 128 * (tt >> 6) + 32 * sub + 8 * pc;
+                    __nv_bfloat16* dst =
+                        item.slot < 0 ? a.o_lat + ((int64_t)item.bj * 128 + hh) * 512 + col
+                                      : a.part_o + (((int64_t)hh * 8 + (col >> 6)) * (2 * a.pairs) + item.slot) * 64 +
+                                            (col & 63);
+                    *reinterpret_cast<uint4*>(dst) = v;
                 }
                 __syncwarp();
             }
             if (item.slot >= 0 && part == 0 && cv == 0) {
                 // the same log-sum-exp for both latent halves of the piece
                 const float lse = m_used + __log2f(lsum);
-                a.part_lse[item.slot * 256 + head] = lse;
-                a.part_lse[item.slot * 256 + 128 + head] = lse;
+                a.part_lse[(head * 2 * a.pairs + item.slot) * 2] = lse;
+                a.part_lse[(head * 2 * a.pairs + item.slot) * 2 + 1] = lse;
             }
             // the next item's first value GEMM (accumulate = 0) may start only after
             // both CTAs' reads of this item's O

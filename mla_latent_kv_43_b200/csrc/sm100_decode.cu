@@ -61,7 +61,8 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
     take(BJ * d.heads * d.d_c * 2, &L->o_lat, &L->o_lat_bytes);
     take((size_t)2 * P * d.heads * d.d_c * 2, &L->part_o, &L->part_o_bytes);   // bf16
     take((size_t)4 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);   // [2P pieces][2 latent halves][H]
-    take((BJ + 1 + P) * 4, &L->sched, &L->sched_bytes);   // tile prefix, then each cluster's first token
+    // tile prefix, each cluster's first token, then each piece slot's token
+    take((BJ + 1 + 3 * P) * 4, &L->sched, &L->sched_bytes);
     L->total = off;
     L->compute_dtype = MLA_BF16;
     L->splits = P;

@@ -30,6 +30,12 @@ namespace {
 
 constexpr int kThreads = 128;
 
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 struct ProjArgs {
     int BJ, H, n_q, n_tile;
     // absorb
@@ -40,6 +46,7 @@ struct ProjArgs {
     __nv_bfloat16* q_lat;
     int32_t* cum;            // [BJ + 1] key tiles prefix of each query token
     int32_t* first_bj;       // [pairs] first query token of each attention cluster's tile range
+    int32_t* slot_owner;     // [2 pairs] query token of each split-KV piece slot (-1: unused)
     int pairs;
     const int32_t* n_sel;    // sparse decode: selected keys per query token (nullptr: dense)
     int max_sel;
@@ -68,6 +75,36 @@ __device__ __forceinline__ int32_t tiles_of(const ProjArgs& a, int bj, bool* bad
         return (n + a.tile_keys - 1) / a.tile_keys;
     }
     return (int32_t)((p + a.tile_keys) / a.tile_keys);
+}
+
+// The query token whose piece each split-KV slot holds: slot 2p the piece in
+// cluster p of a token begun in an earlier cluster, slot 2p + 1 the piece of
+// a token begun in p that goes on past it (-1: no such piece).  cum is the
+// tile prefix just built (in shared or global memory).
+__device__ void plan_slots(const ProjArgs& a, const int32_t* cum, int tid) {
+    const int32_t T = cum[a.BJ];
+    // the token holding tile t: the first bj with cum[bj + 1] > t
+    auto holder = [&](int32_t t) {
+        int l = 0, r = a.BJ - 1;
+        while (l < r) {
+            const int mid = (l + r) >> 1;
+            if (cum[mid + 1] > t) r = mid; else l = mid + 1;
+        }
+        return l;
+    };
+    for (int p = tid; p < a.pairs; p += kThreads) {
+        const int32_t s0 = (int32_t)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
+        const int32_t s1 = (int32_t)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
+        int even = -1, odd = -1;
+        if (s1 > s0) {
+            const int bf = holder(s0);
+            if (cum[bf] < s0) even = bf;
+            const int bl = holder(s1 - 1);
+            if (cum[bl] >= s0 && cum[bl + 1] > s1) odd = bl;
+        }
+        a.slot_owner[2 * p] = even;
+        a.slot_owner[2 * p + 1] = odd;
+    }
 }
 
 // Key-tile plan, for any number of query tokens: per-thread token ranges and
@@ -110,6 +147,8 @@ __device__ void plan_tiles_long(const ProjArgs& a, int tid) {
     for (int w = 0; w < kThreads / 32; ++w) T += part_l[w];
     if (T == 0) {
         for (int p = tid; p < a.pairs; p += kThreads) a.first_bj[p] = a.BJ;
+        __syncthreads();
+        plan_slots(a, a.cum, tid);
         return;
     }
     const int p0 = (int)(((int64_t)run_lo * a.pairs + T - 1) / T);
@@ -125,6 +164,8 @@ __device__ void plan_tiles_long(const ProjArgs& a, int tid) {
             }
         }
     }
+    __syncthreads();         // every cum entry of the block is written (and visible to it)
+    plan_slots(a, a.cum, tid);
 }
 
 constexpr int kPlanTokens = 512;           // tokens the staged plan holds in shared memory (2 KB: the absorb CTAs stay four per SM)
@@ -190,6 +231,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
         }
         a.first_bj[p] = T == 0 ? a.BJ : l;
     }
+    plan_slots(a, s_cum, tid);
 }
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
@@ -332,30 +374,12 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     if (warp == 1) tmem_dealloc(tmem, ncols);
 }
 
-// Split-KV pieces of the query tokens (tokens whose key tiles were cut across
-// attention clusters): cluster p covers tiles [start(p), start(p + 1)),
-// start(p) = p T / pairs (T * pairs fits 32 bits); a cut token has a piece in
-// each cluster pf..pl its tiles reach (clusters with an empty range in between
-// hold nothing): the first in slot 2 pf + 1, the others in slot 2 p.
-struct PieceRange {
-    int T, pairs;
-    __device__ int start(int p) const { return (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)pairs); }
-    __device__ int pair_of(int t) const {      // largest p with start(p) <= t
-        int lo = 0, hi = pairs - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (start(mid) <= t) lo = mid; else hi = mid - 1;
-        }
-        return lo;
-    }
-    __device__ bool empty(int p) const { return start(p) == (p + 1 < pairs ? start(p + 1) : T); }
-};
-
 struct UpArgs {
     const int32_t* cum;          // [BJ + 1] key-tile prefix of the query tokens
+    const int32_t* slot_owner;   // [2 pairs] query token of each piece slot (-1: unused)
     int BJ, H, pairs, n_tok;     // n_tok: tokens per CTA (64)
     int n_cols;                  // MMA N: n_tok + 2 pairs, rounded up to 16 (<= 256)
-    const float* part_lse;       // [2 pairs][2 latent halves][H], log2 domain
+    const float* part_lse;       // [H][2 pairs][2 latent halves], log2 domain
     __nv_bfloat16* out;          // [BJ][H][128]
     int32_t* status;
 };
@@ -393,10 +417,9 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     // per piece slot s (column n_tok + s of D): the tile-local token it belongs
     // to (-1: none in this tile) and its weights for the two latent halves
     __shared__ int slot_tok[256];
-    __shared__ float slot_w[2][256];
-    __shared__ float slot_lse[2][256];
+    __shared__ float slot_lse[2][256], slot_w[2][256];
     // per token of the tile: 0 invalid length (zeros), 1 finished in one
-    // cluster, 2 cut (merge its pieces); first and last slot of its pieces
+    // cluster, 2 cut (merge its pieces)
     __shared__ int tok_mode[64], tok_s0[64], tok_s1[64];
     const int h = blockIdx.x, n0 = blockIdx.z * a.n_tok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -477,63 +500,98 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
         }
         mma_commit_w(&done);
     } else {
-        // ---- pieces and weights (192 threads)
+        // ---- piece tables (192 threads): each slot's tile-local token (from the
+        // plan), each token's mode and slot range, and each slot's weights for
+        // the two latent halves, w = 2^(lse - M) / sum over the token's pieces of
+        // 2^(lse' - M) with M their maximum
         const int t = threadIdx.x - 64;
-        for (int s = t; s < 256; s += 192) slot_tok[s] = -1;
-        named_barrier(1, 192);
-        const PieceRange pr{a.cum[a.BJ], a.pairs};
+        int c0 = 0, c1 = 0;
         if (t < a.n_tok) {
-            // one thread per token: its mode and the slots of its pieces
-            const int n = n0 + t;
-            int mode = 0, s0 = 0, s1 = -1;
-            if (n < a.BJ) {
-                const int c0 = a.cum[n], c1 = a.cum[n + 1];
-                if (c1 > c0) {
-                    const int pf = pr.pair_of(c0), pl = pr.pair_of(c1 - 1);
-                    mode = pf == pl ? 1 : 2;
-                    if (mode == 2) {
-                        s0 = 2 * pf + 1;
-                        s1 = 2 * pl;
-                        slot_tok[s0] = t;
-                        for (int p = pf + 1; p <= pl; ++p)
-                            if (!pr.empty(p)) slot_tok[2 * p] = t;
-                    }
+            // the token's pieces lie in slots [2 pf + 1, 2 pl] (pf, pl: the clusters
+            // holding its first and last key tile; cluster p starts at p T / pairs)
+            if (n0 + t < a.BJ) {
+                c0 = a.cum[n0 + t];
+                c1 = a.cum[n0 + t + 1];
+            }
+            const uint32_t T = (uint32_t)a.cum[a.BJ], P = (uint32_t)a.pairs;
+            auto pair_of = [&](uint32_t tile) {          // largest p with p T / P <= tile
+                int lo = 0, hi = a.pairs - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if ((uint32_t)mid * T / P <= tile) lo = mid; else hi = mid - 1;
                 }
+                return lo;
+            };
+            const bool cut = c1 > c0 && pair_of((uint32_t)c0) != pair_of((uint32_t)(c1 - 1));
+            tok_s0[t] = cut ? 2 * pair_of((uint32_t)c0) + 1 : 256;
+            tok_s1[t] = cut ? 2 * pair_of((uint32_t)(c1 - 1)) : -1;
+        }
+        for (int s = t; s < 256; s += 192) {
+            const int owner = s < S ? a.slot_owner[s] - n0 : -1;
+            const int tok = owner >= 0 && owner < a.n_tok ? owner : -1;
+            slot_tok[s] = tok;
+            if (tok >= 0) {
+                slot_lse[0][s] = __ldcg(a.part_lse + (h * S + s) * 2);
+                slot_lse[1][s] = __ldcg(a.part_lse + (h * S + s) * 2 + 1);
             }
-            tok_mode[t] = mode;
-            tok_s0[t] = s0;
-            tok_s1[t] = s1;
         }
         named_barrier(1, 192);
-        // the pieces' log2-sum-exps, all loads at once
-        for (int s = t; s < S; s += 192) {
-            if (slot_tok[s] >= 0) {
-                slot_lse[0][s] = __ldcg(a.part_lse + (2 * s) * a.H + h);
-                slot_lse[1][s] = __ldcg(a.part_lse + (2 * s + 1) * a.H + h);
-            }
-        }
-        named_barrier(1, 192);
-        // each slot's weights for the two latent halves: w = 2^(lse - M) / sum over
-        // the token's pieces of 2^(lse' - M), M their maximum (one thread per
-        // slot, each scanning its token's slot range: no cross-thread steps)
-        for (int s = t; s < S; s += 192) {
-            const int tt = slot_tok[s];
-            if (tt < 0) continue;
+        if (t < a.n_tok) tok_mode[t] = c1 == c0 ? 0 : (tok_s1[t] >= 0 ? 2 : 1);
+        // A token cut into many pieces: one warp, lanes over its slots and
+        // shuffle reductions.  Few pieces (the usual case): one thread per token.
+        const int gw = warp - 2;
+        for (int tt = gw; tt < a.n_tok; tt += 6) {
             const int s0 = tok_s0[tt], s1 = tok_s1[tt];
+            if (s1 - s0 < 8) continue;
             float M0 = -INFINITY, M1 = -INFINITY;
-            for (int u = s0; u <= s1; ++u) {
-                if (slot_tok[u] != tt) continue;
-                M0 = fmaxf(M0, slot_lse[0][u]);
-                M1 = fmaxf(M1, slot_lse[1][u]);
+            for (int s = s0 + lane; s <= s1; s += 32)
+                if (slot_tok[s] == tt) {
+                    M0 = fmaxf(M0, slot_lse[0][s]);
+                    M1 = fmaxf(M1, slot_lse[1][s]);
+                }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) {
+                M0 = fmaxf(M0, __shfl_xor_sync(0xffffffffu, M0, d));
+                M1 = fmaxf(M1, __shfl_xor_sync(0xffffffffu, M1, d));
             }
             float S0 = 0.f, S1 = 0.f;
-            for (int u = s0; u <= s1; ++u) {
-                if (slot_tok[u] != tt) continue;
-                S0 += exp2f(slot_lse[0][u] - M0);
-                S1 += exp2f(slot_lse[1][u] - M1);
+            for (int s = s0 + lane; s <= s1; s += 32)
+                if (slot_tok[s] == tt) {
+                    S0 += ex2_approx(slot_lse[0][s] - M0);
+                    S1 += ex2_approx(slot_lse[1][s] - M1);
+                }
+#pragma unroll
+            for (int d = 16; d > 0; d >>= 1) {
+                S0 += __shfl_xor_sync(0xffffffffu, S0, d);
+                S1 += __shfl_xor_sync(0xffffffffu, S1, d);
             }
-            slot_w[0][s] = exp2f(slot_lse[0][s] - M0) / S0;
-            slot_w[1][s] = exp2f(slot_lse[1][s] - M1) / S1;
+            const float i0 = 1.f / S0, i1 = 1.f / S1;
+            for (int s = s0 + lane; s <= s1; s += 32)
+                if (slot_tok[s] == tt) {
+                    slot_w[0][s] = ex2_approx(slot_lse[0][s] - M0) * i0;
+                    slot_w[1][s] = ex2_approx(slot_lse[1][s] - M1) * i1;
+                }
+        }
+        if (t < a.n_tok && tok_s1[t] - tok_s0[t] < 8) {
+            const int s0 = tok_s0[t], s1 = tok_s1[t];
+            float M0 = -INFINITY, M1 = -INFINITY;
+            for (int s = s0; s <= s1; ++s)
+                if (slot_tok[s] == t) {
+                    M0 = fmaxf(M0, slot_lse[0][s]);
+                    M1 = fmaxf(M1, slot_lse[1][s]);
+                }
+            float S0 = 0.f, S1 = 0.f;
+            for (int s = s0; s <= s1; ++s)
+                if (slot_tok[s] == t) {
+                    S0 += ex2_approx(slot_lse[0][s] - M0);
+                    S1 += ex2_approx(slot_lse[1][s] - M1);
+                }
+            const float i0 = 1.f / S0, i1 = 1.f / S1;
+            for (int s = s0; s <= s1; ++s)
+                if (slot_tok[s] == t) {
+                    slot_w[0][s] = ex2_approx(slot_lse[0][s] - M0) * i0;
+                    slot_w[1][s] = ex2_approx(slot_lse[1][s] - M1) * i1;
+                }
         }
     }
     __syncthreads();         // piece tables complete
@@ -663,6 +721,7 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
     a.q_lat = q_lat;
     a.cum = cum;
     a.first_bj = first_bj;
+    a.slot_owner = first_bj + pairs;
     a.pairs = pairs;
     a.n_sel = c.n_sel;
     a.max_sel = c.max_sel;
@@ -672,8 +731,8 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
     return launch(absorb_kernel, A, B, a, grid, 2 * 16384 + 2 * N * 128 + 1024, c.stream, "sm100_absorb", launches);
 }
 
-// up-projection with the split-KV merge folded into its operand assembly.
-// o_lat [BJ][H][512] bf16, part_o [2P][H][512] bf16, part_lse [2P][H],
+// up-projection with the split-KV merge applied to the projected piece rows.
+// o_lat [BJ][H][512] bf16, part_o [H][8][2P][64] bf16, part_lse [H][2P][2],
 // W_uv [H][512][128], out [BJ][H][128]
 int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16* part_o, const float* part_lse,
                   const int32_t* cum, int pairs, int* launches) {
@@ -698,14 +757,16 @@ int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16
         if (!make_map(&O, o_lat, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
-        // part_o [2 pairs][H][512], the same view over piece slots: one box = every slot
+        // part_o, head-major and blocked by 64 latent columns ([H][8][2 pairs][64]):
+        // one box = every piece slot of one block and head, contiguous
         const uint64_t dims[4] = {64, (uint64_t)(2 * pairs), 8, (uint64_t)H};
-        const uint64_t str[3] = {(uint64_t)H * 512 * 2, 64 * 2, 512 * 2};
+        const uint64_t str[3] = {128, (uint64_t)(2 * pairs) * 128, (uint64_t)(2 * pairs) * 8 * 128};
         const uint32_t box[4] = {64, (uint32_t)(2 * pairs), 1, 1};
         if (!make_map(&P, part_o, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     UpArgs a{};
     a.cum = cum;
+    a.slot_owner = cum + BJ + 1 + pairs;
     a.BJ = BJ;
     a.H = H;
     a.pairs = pairs;
