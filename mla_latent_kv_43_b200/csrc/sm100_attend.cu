@@ -73,6 +73,7 @@ struct AttnArgs {
     const __nv_bfloat16* q_lat;   // [BJ][128][576]
     const int32_t* cum;           // [BJ + 1] tile prefix
     const int32_t* first_bj;      // [pairs] first query token of each cluster's range
+    const int32_t* cut;           // [pairs + 1] first key tile of each cluster's range
     const int32_t* seq_lens;
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
@@ -109,9 +110,8 @@ struct ItemIter {
         lens = a.seq_lens;
         n_sel = a.n_sel;
         pair = p;
-        const int T = cum[BJ];
-        s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        s1 = (int)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
+        s0 = a.cut[p];
+        s1 = a.cut[p + 1];
         bj = a.first_bj[p];           // first bj with cum[bj + 1] > s0 (from the plan)
     }
     __device__ bool next(Item& it) {
@@ -744,7 +744,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 }  // namespace
 
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs,
+                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, const int32_t* cut, int pairs,
                   int* launches) {
     const bool sparse = c.n_sel != nullptr;
     CUtensorMap ml, mr;
@@ -774,6 +774,7 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
     a.q_lat = q_lat;
     a.cum = cum;
     a.first_bj = first_bj;
+    a.cut = cut;
     a.seq_lens = c.seq_lens;
     a.BJ = c.batch * c.n_q;
     a.n_q = c.n_q;

@@ -92,6 +92,7 @@ struct PairArgs {
     const __nv_bfloat16* q_lat;   // [BJ][128][576]
     const int32_t* cum;           // [BJ + 1] 64-key tile prefix
     const int32_t* first_bj;      // [pairs] first query token of each pair's range
+    const int32_t* cut;           // [pairs + 1] first key tile of each pair's range
     const int32_t* seq_lens;
     int BJ, n_q, pairs;
     float scale_log2;             // softmax_scale * log2(e)
@@ -118,9 +119,8 @@ struct ItemIter {
         n_q = a.n_q;
         lens = a.seq_lens;
         pair = p;
-        const int T = cum[BJ];
-        s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        s1 = (int)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
+        s0 = a.cut[p];
+        s1 = a.cut[p + 1];
         bj = a.first_bj[p];
     }
     __device__ bool next(Item& it) {
@@ -669,7 +669,8 @@ attend_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 }  // namespace
 
 int launch_attend_pair(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                       __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches) {
+                       __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, const int32_t* cut, int pairs,
+                       int* launches) {
     // Rows of 576 columns viewed as 9 groups of 64: (column in group, row,
     // group, ...) with the group dimension's stride 128 bytes, so one box of
     // several groups lands group-major (each group a 64-row x 128-byte block).
@@ -693,6 +694,7 @@ int launch_attend_pair(const DecodeCall& c, const __nv_bfloat16* q_lat, const in
     a.q_lat = q_lat;
     a.cum = cum;
     a.first_bj = first_bj;
+    a.cut = cut;
     a.seq_lens = c.seq_lens;
     a.BJ = c.batch * c.n_q;
     a.n_q = c.n_q;

@@ -19,9 +19,11 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
 int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16* part_o, const float* part_lse,
                   const int32_t* cum, int pairs, int* launches);
 int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches);
+                  __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, const int32_t* cut, int pairs,
+                  int* launches);
 int launch_attend_pair(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t* cum, __nv_bfloat16* o_lat,
-                       __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, int pairs, int* launches);
+                       __nv_bfloat16* part_o, float* part_lse, const int32_t* first_bj, const int32_t* cut, int pairs,
+                       int* launches);
 
 namespace {
 
@@ -60,20 +62,21 @@ void sm100_layout(const mla_dims& d, int batch, int n_q, int64_t max_len, int sp
     take(BJ * d.heads * (d.d_c + d.d_rope) * 2, &L->q_lat, &L->q_lat_bytes);
     take(BJ * d.heads * d.d_c * 2, &L->o_lat, &L->o_lat_bytes);
     take((size_t)2 * P * d.heads * d.d_c * 2, &L->part_o, &L->part_o_bytes);   // bf16
-    take((size_t)4 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);   // [2P pieces][2 latent halves][H]
-    // tile prefix, each cluster's first token, then each piece slot's token
-    take((BJ + 1 + 3 * P) * 4, &L->sched, &L->sched_bytes);
+    take((size_t)4 * P * d.heads * 4, &L->part_lse, &L->part_lse_bytes);   // [H][2P pieces][2 latent halves]
+    // tile prefix, each cluster's first token, each piece slot's token, then
+    // each cluster's first tile (and the total)
+    take((BJ + 2 + 4 * P) * 4, &L->sched, &L->sched_bytes);
     L->total = off;
     L->compute_dtype = MLA_BF16;
     L->splits = P;
 }
 
 int sm100_decode(const DecodeCall& c, int* launches) {
-    // The tile ranges of the clusters are p * T / P in 32-bit arithmetic on the
-    // device (T = total key tiles <= B * n_q * ceil(max_len / 64), or
-    // ceil(max_sel / 64) per query for the sparse decode).
+    // Key-tile indices are int32 on the device (T = total key tiles <= B * n_q *
+    // ceil(max_len / 64), or ceil(max_sel / 64) per query for the sparse decode,
+    // plus the plan's per-token charge of 4 tiles).
     const int64_t keys_bound = c.n_sel ? c.max_sel : c.max_len;
-    if ((int64_t)c.batch * c.n_q * ((keys_bound + 63) / 64) * c.L.splits >= ((int64_t)1 << 31))
+    if ((int64_t)c.batch * c.n_q * ((keys_bound + 63) / 64 + 4) >= ((int64_t)1 << 31))
         return MLA_ERR_UNSUPPORTED;
     auto* q_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.q_lat);
     auto* o_lat = reinterpret_cast<__nv_bfloat16*>(c.ws + c.L.o_lat);
@@ -84,13 +87,14 @@ int sm100_decode(const DecodeCall& c, int* launches) {
     const int BJ = c.batch * c.n_q;
     int rc;
     int32_t* first_bj = cum + BJ + 1;
+    const int32_t* cut = first_bj + 3 * P;
     if ((rc = sm100::launch_absorb(c, q_lat, cum, first_bj, P, launches))) return rc;
     // dense decode: the CTA-pair kernel or the latent-split kernel; decode over a
     // selection: the latent-split kernel gathering its rows (64-key tiles throughout).
     // The up-projection merges the split-KV pieces of each token.
     rc = (c.n_sel || !kDecodePairKernel)
-             ? sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, P, launches)
-             : sm100::launch_attend_pair(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, P, launches);
+             ? sm100::launch_attend(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, cut, P, launches)
+             : sm100::launch_attend_pair(c, q_lat, cum, o_lat, part_o, part_lse, first_bj, cut, P, launches);
     if (rc) return rc;
     return sm100::launch_upproj(c, o_lat, part_o, part_lse, cum, P, launches);
 }

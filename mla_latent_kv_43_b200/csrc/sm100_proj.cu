@@ -47,6 +47,7 @@ struct ProjArgs {
     int32_t* cum;            // [BJ + 1] key tiles prefix of each query token
     int32_t* first_bj;       // [pairs] first query token of each attention cluster's tile range
     int32_t* slot_owner;     // [2 pairs] query token of each split-KV piece slot (-1: unused)
+    int32_t* cut;            // [pairs + 1] first key tile of each attention cluster
     int pairs;
     const int32_t* n_sel;    // sparse decode: selected keys per query token (nullptr: dense)
     int max_sel;
@@ -77,12 +78,40 @@ __device__ __forceinline__ int32_t tiles_of(const ProjArgs& a, int bj, bool* bad
     return (int32_t)((p + a.tile_keys) / a.tile_keys);
 }
 
-// The query token whose piece each split-KV slot holds: slot 2p the piece in
+// Cluster ranges, given the key-tile prefix cum of the query tokens.  Cluster
+// p covers tiles [cut[p], cut[p + 1]).  The cuts share out a cost that charges
+// every query token kItemTiles tiles on top of its own (loading its query
+// slice and its epilogue cost about that much time per item), so a cluster
+// that gets more items gets fewer tiles; a cut that falls in a token's fixed
+// share lands on the token's first tile.  Then each cluster's first token and
+// the query token each split-KV piece slot holds: slot 2p the piece in
 // cluster p of a token begun in an earlier cluster, slot 2p + 1 the piece of
-// a token begun in p that goes on past it (-1: no such piece).  cum is the
-// tile prefix just built (in shared or global memory).
-__device__ void plan_slots(const ProjArgs& a, const int32_t* cum, int tid) {
+// a token begun in p that goes on past it (-1: no such piece).
+constexpr int kItemTiles = 4;
+constexpr int kMaxClusters = 256;
+__device__ void plan_clusters(const ProjArgs& a, const int32_t* cum, int tid) {
+    __shared__ int32_t s_cut[kMaxClusters + 1];
     const int32_t T = cum[a.BJ];
+    const int64_t C = (int64_t)T + (int64_t)kItemTiles * a.BJ;
+    for (int p = tid; p <= a.pairs; p += kThreads) {
+        int32_t t = T;
+        if (p < a.pairs) {
+            const int64_t x = (int64_t)p * C / a.pairs;
+            int lo = 0, hi = a.BJ;                     // largest bj with cum[bj] + K bj <= x
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if ((int64_t)cum[mid] + (int64_t)kItemTiles * mid <= x) lo = mid; else hi = mid - 1;
+            }
+            if (lo < a.BJ) {
+                const int64_t o = x - ((int64_t)cum[lo] + (int64_t)kItemTiles * lo) - kItemTiles;
+                const int64_t len = cum[lo + 1] - cum[lo];
+                t = cum[lo] + (int32_t)(o < 0 ? 0 : (o > len ? len : o));
+            }
+        }
+        s_cut[p] = t;
+        a.cut[p] = t;
+    }
+    __syncthreads();
     // the token holding tile t: the first bj with cum[bj + 1] > t
     auto holder = [&](int32_t t) {
         int l = 0, r = a.BJ - 1;
@@ -93,8 +122,8 @@ __device__ void plan_slots(const ProjArgs& a, const int32_t* cum, int tid) {
         return l;
     };
     for (int p = tid; p < a.pairs; p += kThreads) {
-        const int32_t s0 = (int32_t)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        const int32_t s1 = (int32_t)(((uint32_t)(p + 1) * (uint32_t)T) / (uint32_t)a.pairs);
+        const int32_t s0 = s_cut[p], s1 = s_cut[p + 1];
+        a.first_bj[p] = s0 < T ? holder(s0) : a.BJ;
         int even = -1, odd = -1;
         if (s1 > s0) {
             const int bf = holder(s0);
@@ -133,39 +162,13 @@ __device__ void plan_tiles_long(const ProjArgs& a, int tid) {
     int32_t run = incl - sum;
     for (int w = 0; w < warp; ++w) run += part_l[w];
     if (tid == 0) a.cum[0] = 0;
-    const int32_t run_lo = run;                 // cum[lo]
     bool ignored = false;
     for (int bj = lo; bj < hi; ++bj) {
         run += tiles_of(a, bj, &ignored);
         a.cum[bj + 1] = run;
     }
-    // First query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
-    // the first bj with cum[bj + 1] > floor(p T / pairs).  The thread whose prefix
-    // range [cum[lo], cum[hi]) holds that start answers from its own values: those
-    // are the clusters p with ceil(cum[lo] pairs / T) <= p < ceil(cum[hi] pairs / T).
-    int32_t T = 0;
-    for (int w = 0; w < kThreads / 32; ++w) T += part_l[w];
-    if (T == 0) {
-        for (int p = tid; p < a.pairs; p += kThreads) a.first_bj[p] = a.BJ;
-        __syncthreads();
-        plan_slots(a, a.cum, tid);
-        return;
-    }
-    const int p0 = (int)(((int64_t)run_lo * a.pairs + T - 1) / T);
-    const int p1 = min(a.pairs, (int)(((int64_t)run * a.pairs + T - 1) / T));
-    for (int p = p0; p < p1; ++p) {
-        const int s0 = (int)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        int32_t c = run_lo;
-        for (int bj = lo; bj < hi; ++bj) {
-            c += tiles_of(a, bj, &ignored);
-            if (c > s0) {
-                a.first_bj[p] = bj;
-                break;
-            }
-        }
-    }
     __syncthreads();         // every cum entry of the block is written (and visible to it)
-    plan_slots(a, a.cum, tid);
+    plan_clusters(a, a.cum, tid);
 }
 
 constexpr int kPlanTokens = 512;           // tokens the staged plan holds in shared memory (2 KB: the absorb CTAs stay four per SM)
@@ -219,19 +222,7 @@ __device__ void plan_tiles(const ProjArgs& a, int tid) {
         }
     }
     __syncthreads();
-    // First query token of every cluster's tile range [p T / pairs, (p + 1) T / pairs):
-    // the first bj with cum[bj + 1] > floor(p T / pairs) (BJ when there is none).
-    const int32_t T = s_cum[a.BJ];
-    for (int p = tid; p < a.pairs; p += kThreads) {
-        const int32_t s0 = (int32_t)(((uint32_t)p * (uint32_t)T) / (uint32_t)a.pairs);
-        int l = 0, r = a.BJ;
-        while (l < r) {
-            const int mid = (l + r) >> 1;
-            if (s_cum[mid + 1] > s0) r = mid; else l = mid + 1;
-        }
-        a.first_bj[p] = T == 0 ? a.BJ : l;
-    }
-    plan_slots(a, s_cum, tid);
+    plan_clusters(a, s_cum, tid);
 }
 
 __host__ __device__ constexpr uint32_t tmem_cols_for(int n) {
@@ -377,6 +368,7 @@ absorb_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
 struct UpArgs {
     const int32_t* cum;          // [BJ + 1] key-tile prefix of the query tokens
     const int32_t* slot_owner;   // [2 pairs] query token of each piece slot (-1: unused)
+    const int32_t* cut;          // [pairs + 1] first key tile of each attention cluster
     int BJ, H, pairs, n_tok;     // n_tok: tokens per CTA (64)
     int n_cols;                  // MMA N: n_tok + 2 pairs, rounded up to 16 (<= 256)
     const float* part_lse;       // [H][2 pairs][2 latent halves], log2 domain
@@ -421,6 +413,7 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     // per token of the tile: 0 invalid length (zeros), 1 finished in one
     // cluster, 2 cut (merge its pieces)
     __shared__ int tok_mode[64], tok_s0[64], tok_s1[64];
+    __shared__ int32_t s_cut[257];
     const int h = blockIdx.x, n0 = blockIdx.z * a.n_tok;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = a.n_cols, S = 2 * a.pairs;
@@ -506,25 +499,27 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
         // 2^(lse' - M) with M their maximum
         const int t = threadIdx.x - 64;
         int c0 = 0, c1 = 0;
+        if (t < a.n_tok && n0 + t < a.BJ) {
+            c0 = a.cum[n0 + t];
+            c1 = a.cum[n0 + t + 1];
+        }
+        for (int p = t; p <= a.pairs; p += 192) s_cut[p] = a.cut[p];
+        named_barrier(1, 192);
         if (t < a.n_tok) {
             // the token's pieces lie in slots [2 pf + 1, 2 pl] (pf, pl: the clusters
-            // holding its first and last key tile; cluster p starts at p T / pairs)
-            if (n0 + t < a.BJ) {
-                c0 = a.cum[n0 + t];
-                c1 = a.cum[n0 + t + 1];
-            }
-            const uint32_t T = (uint32_t)a.cum[a.BJ], P = (uint32_t)a.pairs;
-            auto pair_of = [&](uint32_t tile) {          // largest p with p T / P <= tile
+            // holding its first and last key tile)
+            auto pair_of = [&](int32_t tile) {           // largest p with cut[p] <= tile
                 int lo = 0, hi = a.pairs - 1;
                 while (lo < hi) {
                     const int mid = (lo + hi + 1) >> 1;
-                    if ((uint32_t)mid * T / P <= tile) lo = mid; else hi = mid - 1;
+                    if (s_cut[mid] <= tile) lo = mid; else hi = mid - 1;
                 }
                 return lo;
             };
-            const bool cut = c1 > c0 && pair_of((uint32_t)c0) != pair_of((uint32_t)(c1 - 1));
-            tok_s0[t] = cut ? 2 * pair_of((uint32_t)c0) + 1 : 256;
-            tok_s1[t] = cut ? 2 * pair_of((uint32_t)(c1 - 1)) : -1;
+            const int pf = pair_of(c0), pl = pair_of(c1 - 1);
+            const bool cut = c1 > c0 && pf != pl;
+            tok_s0[t] = cut ? 2 * pf + 1 : 256;
+            tok_s1[t] = cut ? 2 * pl : -1;
         }
         for (int s = t; s < 256; s += 192) {
             const int owner = s < S ? a.slot_owner[s] - n0 : -1;
@@ -722,6 +717,7 @@ int launch_absorb(const DecodeCall& c, __nv_bfloat16* q_lat, int32_t* cum, int32
     a.cum = cum;
     a.first_bj = first_bj;
     a.slot_owner = first_bj + pairs;
+    a.cut = first_bj + 3 * pairs;
     a.pairs = pairs;
     a.n_sel = c.n_sel;
     a.max_sel = c.max_sel;
@@ -767,6 +763,7 @@ int launch_upproj(const DecodeCall& c, __nv_bfloat16* o_lat, const __nv_bfloat16
     UpArgs a{};
     a.cum = cum;
     a.slot_owner = cum + BJ + 1 + pairs;
+    a.cut = cum + BJ + 1 + 3 * pairs;
     a.BJ = BJ;
     a.H = H;
     a.pairs = pairs;

@@ -26,16 +26,16 @@ def merge_pieces(prob, o_lat, BJ, H, d_c):
     """The tensor-core path leaves a query token whose key tiles were cut across
     work items as pieces (normalised partial rows, one log2-sum-exp per latent
     half); merge them here as the up-projection does after projecting.  Item p
-    covers tiles [p T / P, (p + 1) T / P); a cut token's first piece is in slot
-    2 pf + 1, its later ones in slot 2 p."""
+    covers tiles [start[p], start[p + 1]) (from the schedule); a cut token's
+    first piece is in slot 2 pf + 1, its later ones in slot 2 p."""
     P = prob.layout["splits"]
-    cum = prob.workspace_view("sched", (-1,), torch.int32)[: BJ + 1].cpu().numpy().astype(np.int64)
+    sched = prob.workspace_view("sched", (-1,), torch.int32).cpu().numpy().astype(np.int64)
+    cum = sched[: BJ + 1]
+    start = list(sched[BJ + 1 + 3 * P: BJ + 2 + 4 * P])          # each item's first key tile
     # part_o head-major, blocked by 64 columns: [H][d_c / 64][2P][64]; part_lse [H][2P][2]
     part_o = prob.workspace_view("part_o", (H, d_c // 64, 2 * P, 64), torch.bfloat16).double().cpu().numpy()
     part_o = part_o.transpose(2, 0, 1, 3).reshape(2 * P, H, d_c)
     lse = prob.workspace_view("part_lse", (H, 2 * P, 2), torch.float32).double().cpu().numpy().transpose(1, 2, 0)
-    T = int(cum[BJ])
-    start = [p * T // P for p in range(P + 1)]
     pair_of = lambda t: max(p for p in range(P) if start[p] <= t)  # noqa: E731
     out = o_lat.copy()
     for n in range(BJ):
