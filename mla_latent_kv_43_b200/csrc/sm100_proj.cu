@@ -592,20 +592,19 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
     __syncthreads();         // piece tables complete
 
     if (block_wait(&done, &flag, a.status)) {
-        // Projected rows -> stage[n][128] bf16 (the B ring is free now).  Warps
-        // w and w + 4 share TMEM lane quarter w & 3 (v = 32 (w & 3) + lane):
-        // warps 0-3 take the tokens finished in one cluster (D0 + D1 of their own
-        // column), warps 4-7 the cut tokens (their pieces' columns, weighted).
+        // Projected rows straight to out[n][h][0:128] (lane v of a warp writes
+        // element v: each store covers 64 contiguous bytes).  Warps w and w + 4
+        // share TMEM lane quarter w & 3 (v = 32 (w & 3) + lane): warps 0-3 take
+        // the tokens finished in one cluster (D0 + D1 of their own column), warps
+        // 4-7 the cut tokens (their pieces' columns, weighted).  Each lane holds
+        // one column's token data and the loops take it by shuffle.
         tc_fence_after();
-        __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(sB);
         const int q = warp & 3, v = q * 32 + lane;
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        // Both loops are branch-free per column: each lane holds one column's
-        // token data and the loop takes it by shuffle, and stores that are not
-        // wanted go to a dummy row, so no iteration waits on a load or a branch.
-        __nv_bfloat16* dummy = stage + 64 * 128;   // past the tile's 64 token rows
+        const int nvalid = min(a.n_tok, a.BJ - n0);
+        __nv_bfloat16* out_hv = a.out + ((int64_t)n0 * a.H + h) * 128 + v;   // token n at + n H 128
         if (warp < 4) {
-            for (int c0 = 0; c0 < a.n_tok; c0 += 32) {
+            for (int c0 = 0; c0 < nvalid; c0 += 32) {
                 uint32_t r0[32], r1[32];
                 tmem_ld32(tmem + lane_off + c0, r0);
                 tmem_ld32(tmem + lane_off + 256 + c0, r1);
@@ -615,8 +614,7 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
                 for (int i = 0; i < 32; ++i) {
                     const int mode = __shfl_sync(0xffffffffu, my_mode, i);
                     const float val = mode == 1 ? __uint_as_float(r0[i]) + __uint_as_float(r1[i]) : 0.f;
-                    __nv_bfloat16* dst = mode == 2 ? dummy + v : stage + (c0 + i) * 128 + v;
-                    *dst = __float2bfloat16_rn(val);
+                    if (mode != 2 && c0 + i < nvalid) out_hv[(int64_t)(c0 + i) * a.H * 128] = __float2bfloat16_rn(val);
                 }
             }
         } else {
@@ -640,20 +638,12 @@ upproj_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ 
                     const float pv = fmaf(w0, __uint_as_float(r0[i]), w1 * __uint_as_float(r1[i]));
                     const float val = tok >= 0 ? pv : 0.f;
                     const bool starts = tok >= 0 && tok != prev;    // a new token's first piece
-                    __nv_bfloat16* dst = (starts && prev >= 0) ? stage + prev * 128 + v : dummy + v;
-                    *dst = __float2bfloat16_rn(acc);                // the finished token's row
+                    if (starts && prev >= 0) out_hv[(int64_t)prev * a.H * 128] = __float2bfloat16_rn(acc);
                     acc = starts ? val : acc + val;
                     prev = tok >= 0 ? tok : prev;
                 }
             }
-            if (prev >= 0) stage[prev * 128 + v] = __float2bfloat16_rn(acc);
-        }
-        __syncthreads();
-        const int nvalid = min(a.n_tok, a.BJ - n0);
-        for (int i = threadIdx.x; i < nvalid * 16; i += kUpThreads) {
-            const int n = i >> 4, c = i & 15;
-            reinterpret_cast<uint4*>(a.out + ((int64_t)(n0 + n) * a.H + h) * 128)[c] =
-                reinterpret_cast<const uint4*>(stage + n * 128)[c];
+            if (prev >= 0) out_hv[(int64_t)prev * a.H * 128] = __float2bfloat16_rn(acc);
         }
     }
     tc_fence_before();
