@@ -167,11 +167,14 @@ __device__ __forceinline__ float ex2(float x) {
 template <bool kSparse>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_rope,
-              AttnArgs a) {
+              const __grid_constant__ CUtensorMap map_ql, const __grid_constant__ CUtensorMap map_qr, AttnArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[kStages], empty[kStages];
-    __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, drain;
+    // q0_full: the first item's query slice has landed (tensor copies into
+    // stages 2-3 and the Q-rope area); q0_copied: its latent part is in TMEM
+    // (tcgen05.cp), so stages 2-3 may take cache tiles
+    __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, q0_full, q0_copied, drain;
     __shared__ uint64_t p_ready[kXBufs], xin_full[kXBufs], rx_done[kXBufs];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -211,6 +214,8 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         mbar_init(&o_done[0], 1);           // O GEMMs of even / odd global tiles
         mbar_init(&o_done[1], 1);
         mbar_init(&q_ready, 1);
+        mbar_init(&q0_full, 1);
+        mbar_init(&q0_copied, 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(&m_ready[0][i], 1);   // warp of lane quarter i in the group of an even tile
             mbar_init(&m_ready[1][i], 1);   // ... of an odd tile
@@ -251,6 +256,19 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             Item item;
             uint32_t it = 0;
             bool ok = true;
+            {
+                // The first item's query slice by tensor copies: this CTA's latent half
+                // (four 64-column groups, 64 KB) into stages 2-3, its rope columns into
+                // the Q-rope area.  (Later items' slices are loaded by the exchange
+                // warps, after their predecessor's score GEMMs.)
+                ItemIter peek = iter;
+                Item first;
+                if (peek.next(first)) {
+                    mbar_expect_tx(&q0_full, 4 * 128 * 128 + 128 * 64);
+                    tma_load_4d(smem + 2 * kStageBytes, &map_ql, &q0_full, 0, 0, 4 * (int)rank, first.bj);
+                    tma_load_3d(smem + kOffQr, &map_qr, &q0_full, 512 + 32 * rank, 0, first.bj);
+                }
+            }
             while (ok && iter.next(item)) {
                 const int b = item.bj / a.n_q;
                 for (int t = item.t0; t < item.t1; ++t, ++it) {
@@ -262,6 +280,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     // start-up: the first stage is requested alone, so every SM's first
                     // tile lands before the rest of the start-up burst
                     if (it == 1 && !mbar_wait(&full[0], 0, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    // stages 2-3 hold the first query slice until it is copied to TMEM
+                    if (it == 2 && !mbar_wait(&q0_copied, 0, abort)) {
                         ok = false;
                         break;
                     }
@@ -360,7 +383,21 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             // score GEMM S(gS): 16 K-steps of latent (A = query slice in TMEM), 2 of rope
             if (haveS) {
                 const int s = gS % kStages, sb = gS & 1;
-                if (!qS) qS = mbar_ready_w(&q_ready, nItemsS & 1);
+                if (!qS && nItemsS == 0 && mbar_ready_w(&q0_full, 0)) {
+                    // the first item's latent query slice: stages 2-3 -> TMEM (A operand
+                    // of the score GEMM), 128 rows x 32 bytes per copy, ahead of the
+                    // score GEMMs in this thread's order
+                    tc_fence_after();
+                    const uint64_t dq = sdesc(sbase + 2 * kStageBytes, 16, 1024, kSwizzle128);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tmem_cp_128x256b_w(tmem + kColQ + 32 * g + 8 * j, sdesc_add(dq, g * 16384 + j * 32));
+                    mma_commit_w(&q0_copied);
+                    qS = true;
+                }
+                if (!qS && nItemsS > 0) qS = mbar_ready_w(&q_ready, (nItemsS - 1) & 1);
                 if (qS && mbar_ready_w(&full[s], (gS / kStages) & 1) &&
                     (gS < 2 || mbar_ready_w(&s_free[sb], ((gS >> 1) - 1) & 1))) {
                     tc_fence_after();
@@ -417,10 +454,11 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             if (leader) ex_stop = *abort;
             named_barrier(1, 128);
             if (ex_stop) break;
-            // query slice of this token: latent part -> TMEM, rope part -> smem (SW64 rows).
-            // Every score GEMM of the previous item has completed: its last
-            // score tile was read below before we got here.
-            {
+            // query slice of this token (the first item's comes by tensor copies):
+            // latent part -> TMEM, rope part -> smem (SW64 rows).  Every score GEMM
+            // of the previous item has completed: its last score tile was read
+            // below before we got here.
+            if (it > 0) {
                 // loads in two batches of 16 (plus the rope chunks), each batch issued
                 // before any TMEM store, so the slice costs two memory round trips
                 const uint4* src = reinterpret_cast<const uint4*>(a.q_lat + ((int64_t)item.bj * 128 + h) * 576);
@@ -793,7 +831,25 @@ int launch_attend(const DecodeCall& c, const __nv_bfloat16* q_lat, const int32_t
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MLA_ERR_CUDA;
     prof_begin(c.stream, "sm100_attend");
-    const cudaError_t e = launch_pdl(kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, ml, mr, a);
+    // the first item's query slice: q_lat [BJ][128][576] as (column in group, head,
+    // group of 64 columns, token), one box = all heads x four groups, landing
+    // group-major; its rope columns as (column, head, token), SW64 rows
+    CUtensorMap mql, mqr;
+    const int64_t BJ = (int64_t)c.batch * c.n_q;
+    {
+        const uint64_t dims[4] = {64, 128, 9, (uint64_t)BJ};
+        const uint64_t str[3] = {576 * 2, 64 * 2, 128 * 576 * 2};
+        const uint32_t box[4] = {64, 128, 4, 1};
+        if (!make_map(&mql, q_lat, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+    }
+    {
+        const uint64_t dims[3] = {576, 128, (uint64_t)BJ};
+        const uint64_t str[2] = {576 * 2, 128 * 576 * 2};
+        const uint32_t box[3] = {32, 128, 1};
+        if (!make_map(&mqr, q_lat, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_64B)) return MLA_ERR_CUDA;
+    }
+    const cudaError_t e =
+        launch_pdl(kernel, dim3(2 * pairs), dim3(kThreads), smem, c.stream, ml, mr, mql, mqr, a);
     prof_end(c.stream);
     if (launches) ++*launches;
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? MLA_OK : MLA_ERR_CUDA;

@@ -298,6 +298,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // warp-uniform (instead of running it in one divergent thread) lets the
 // descriptors stay warp-uniform values, which makes issue several times
 // cheaper.
+// Whole warp; one elected lane copies a 128-row x 32-byte shared-memory
+// matrix (described like an MMA operand) into TMEM lanes 0-127, 8 columns
+// from `taddr`.  Ordered with the same thread's tcgen05.mma; tracked by commit.
+__device__ __forceinline__ void tmem_cp_128x256b_w(uint32_t taddr, uint64_t s_desc) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}" ::"r"(taddr),
+        "l"(s_desc)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
     asm volatile(
