@@ -20,7 +20,11 @@ and item_done (committed after each item's last value GEMM; the epilogue
 waits on it rather than on the per-tile o_done[n & 1], whose parity names
 the right completion only if the value GEMM two tiles earlier is done).
 The shipped protocol has both; a control run without them must find the
-hazards, which shows the model can see them."""
+hazards, which shows the model can see them.  The first item's query slice
+arrives by tensor copies into cache stages 2-3 (q0_full) and is copied to
+TMEM by the MMA issuer ahead of its score GEMMs (tcgen05.cp, committed to
+q0_copied); the TMA producer waits for q0_copied before loading tile 2 into
+stage 2, which a further control shows is needed."""
 import random
 
 import pytest
@@ -61,7 +65,7 @@ def wait(bar, parity, nth):
         raise Hazard(f"{bar.name}: {bar.completions} completions, the wait names #{nth}")
 
 
-def run(items, seed, item_barriers=True, rescale_p=0.3):
+def run(items, seed, item_barriers=True, rescale_p=0.3, q0_wait=True):
     rng = random.Random(seed)
     G = sum(items)
     item_of = [n for n, T in enumerate(items) for _ in range(T)]
@@ -82,6 +86,8 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
         c.s_free = [Barrier(f"{r}s_free{i}", 8) for i in range(2)]
         c.o_done = [Barrier(f"{r}o_done{i}") for i in range(2)]
         c.q_ready = Barrier(f"{r}q_ready")
+        c.q0_full = Barrier(f"{r}q0_full")
+        c.q0_copied = Barrier(f"{r}q0_copied")
         c.p_ready = [Barrier(f"{r}p_ready{i}", 4) for i in range(XBUFS)]
         c.xin_full = [Barrier(f"{r}xin_full{i}") for i in range(XBUFS)]
         c.rx_done = [Barrier(f"{r}rx_done{i}") for i in range(XBUFS)]
@@ -99,10 +105,16 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
 
     def tma(r):
         c = ctas[r]
+        # the first item's query slice by tensor copies into stages 2-3
+        c.q0_full.arrive(expect_tx=1)
+        engine.append(("qload", r, None, 0))
+        yield "step"
         for g in range(G):
             s = g % STAGES
             if g >= STAGES:
                 yield from wait(c.empty[s], ((g // STAGES) - 1) & 1, g // STAGES)
+            if g == 2 and q0_wait:                               # stages 2-3 free once copied to TMEM
+                yield from wait(c.q0_copied, 0, 1)
             engine.append(("load", r, s, g))
             yield "step"
 
@@ -125,8 +137,12 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
                 gO += 1
                 progressed = True
             if gS < G:
-                if not q_ok:
-                    q_ok = c.q_ready.passes(items_s & 1)
+                if not q_ok and items_s == 0 and c.q0_full.passes(0):
+                    c.tq.append(("cpQ", 0))                      # stages 2-3 -> TMEM
+                    c.tq.append(("commit", c.q0_copied))
+                    q_ok = True
+                elif not q_ok and items_s > 0:
+                    q_ok = c.q_ready.passes((items_s - 1) & 1)
                 s, sb = gS % STAGES, gS & 1
                 if q_ok and c.full[s].passes((gS // STAGES) & 1) and \
                         (gS < 2 or c.s_free[sb].passes(((gS >> 1) - 1) & 1)):
@@ -143,10 +159,12 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
         c = ctas[r]
         g = 0
         for n, T in enumerate(items):
-            # the previous item's score GEMMs are done (its last score tile was read)
-            c.Q = n
-            c.q_ready.arrive()
-            yield "step"
+            # the previous item's score GEMMs are done (its last score tile was read);
+            # the first item's slice comes by tensor copies
+            if n > 0:
+                c.Q = n
+                c.q_ready.arrive()
+                yield "step"
             for k in range(T):
                 sb, xb = g & 1, g % XBUFS
                 yield from wait(c.s_full[sb], (g >> 1) & 1, (g >> 1) + 1)
@@ -228,7 +246,11 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
             if c.tq:
                 op = c.tq.pop(0)
                 progressed = True
-                if op[0] == "S":
+                if op[0] == "cpQ":
+                    if c.stage[2] != "Q" or c.stage[3] != "Q":
+                        raise Hazard(f"cta {r}: the query copy reads stages holding {c.stage[2:4]}")
+                    c.Q = 0
+                elif op[0] == "S":
                     g = op[1]
                     if c.stage[g % STAGES] != g:
                         raise Hazard(f"cta {r}: S({g}) reads stage holding {c.stage[g % STAGES]}")
@@ -251,7 +273,10 @@ def run(items, seed, item_barriers=True, rescale_p=0.3):
                 kind, r, i, g = engine.pop(rng.randrange(len(engine)))
                 c = ctas[r]
                 progressed = True
-                if kind == "load":
+                if kind == "qload":
+                    c.stage[2] = c.stage[3] = "Q"
+                    c.q0_full.complete_tx(1)
+                elif kind == "load":
                     c.stage[i] = g
                     c.full[i].arrive()
                 else:
@@ -278,6 +303,21 @@ SHAPES = [(1, 1, 1, 1), (2, 1, 3), (3, 3), (1, 5, 2, 1), (4,), (1,) * 7, (2, 2, 
 def test_decode_protocol_shipped(items):
     for seed in range(25):
         run(list(items), seed * 31 + len(items))
+
+
+def test_model_finds_the_overwritten_query_without_the_copy_wait():
+    """Control: without the loader's wait for q0_copied, a cache tile can land
+    in stage 2 or 3 before tcgen05.cp has read the first query slice."""
+    found = False
+    for items in SHAPES:
+        if sum(items) < 3:
+            continue
+        for seed in range(25):
+            try:
+                run(list(items), seed * 31 + len(items), q0_wait=False)
+            except Hazard as e:
+                found = found or "query copy" in str(e)
+    assert found
 
 
 def test_model_finds_the_hazards_without_the_item_barriers():
