@@ -47,6 +47,8 @@ DEFAULT_WORKLOAD = "v3_b64_ragged"
 FLUSH_BYTES = 512 << 20
 KERNEL_SOURCES = {  # kernel name prefix -> source file whose hash keys committed ncu traffic
     "sm100_attend": "mla_latent_kv_43_b200/csrc/sm100_attend.cu",
+    "sm100_upproj": "mla_latent_kv_43_b200/csrc/sm100_proj.cu",
+    "sm100_absorb": "mla_latent_kv_43_b200/csrc/sm100_proj.cu",
     "generic_attend": "mla_latent_kv_43_b200/csrc/generic.cu",
     "sm100_oproj": "mla_latent_kv_43_b200/csrc/sm100_append.cu",
     "sm100_prefill_attend": "mla_latent_kv_43_b200/csrc/sm100_prefill.cu",
