@@ -117,33 +117,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-// try_wait with a suspend-time hint: the thread sleeps until the phase
-// completes (or about `ns` nanoseconds pass) instead of re-polling, so a
-// waiting thread does not keep the shared-memory pipe busy.
-template <bool kCluster>
-__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    if (kCluster)
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
-            : "memory");
-    else
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
-            : "memory");
-    return ok != 0;
-}
-
-constexpr uint32_t kWaitSleepNs = 20000;   // per try_wait; the time limit is checked every 256
-
 // Wait for the phase with parity `parity` to complete.  Returns false when
 // the time limit passed or *abort became non-zero.
 template <bool kCluster = false>
@@ -152,7 +125,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_test_sleep<kCluster>(bar, parity, kWaitSleepNs)) return true;
+        if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (abort && *abort) return false;
             if (globaltimer() - t0 > limit_ns) return false;
