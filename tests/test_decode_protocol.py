@@ -296,7 +296,8 @@ def run(items, seed, item_barriers=True, rescale_p=0.3, q0_wait=True):
             raise Hazard("deadlock")
 
 
-SHAPES = [(1, 1, 1, 1), (2, 1, 3), (3, 3), (1, 5, 2, 1), (4,), (1,) * 7, (2, 2, 2, 2), (5, 1, 1, 6)]
+SHAPES = [(1, 1, 1, 1), (2, 1, 3), (3, 3), (1, 5, 2, 1), (4,), (1,) * 7, (2, 2, 2, 2), (5, 1, 1, 6),
+          (12, 12), (3, 25, 2)]
 
 
 @pytest.mark.parametrize("items", SHAPES)
