@@ -26,7 +26,9 @@
 // share every key and value tile.  Per 64-key tile and group:
 // S = [q_nope || q_rot] [Kn || k_rope]^T (M 128, N 64, K 192) into one of the
 // group's two TMEM score buffers; the softmax warps (one thread per query
-// row) mask keys past the row's position, keep a base-2 running maximum that
+// row, the row read from TMEM once and the buffer released at once) mask keys
+// past the row's position (only in warps whose rows reach the diagonal; the
+// others take a select-free path with paired FMAs), keep a base-2 running maximum that
 // moves only when it grows by more than 2^8 (O and the row sum are rescaled
 // then) and write P as bf16 into the group's shared-memory tile;
 // O += P V (M 128, N 128, K 64) with V read MN-major.  Keys and values have
@@ -37,8 +39,12 @@
 // warp issues both groups' score GEMMs of tile i, then their value GEMMs of
 // tile i - 1, so one group's softmax runs while the tensor core works for the
 // other.
-// Roles (320 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 softmax of
-// group 0, warps 6-9 of group 1.
+// Roles (352 threads): warp 0 TMA for the queries and keys, warp 10 TMA for
+// the values (so a key load never waits behind a value buffer's release),
+// warp 1 MMA issue, warps 2-5 softmax of group 0, warps 6-9 of group 1.
+// Each key or value tile arrives in one tensor copy (both 64-column halves
+// of its 128-wide rows, viewed as two groups of stride 128 bytes), the rope
+// key in a second one.
 // TMEM: O of group g at [128 g, 128 g + 128), S double buffers at
 // [256 + 128 g, 256 + 128 g + 128).
 #include <cuda_bf16.h>
@@ -67,7 +73,7 @@ constexpr int kVBytes = 2 * kBox;                  // value tile: V[0:64], V[64:
 constexpr int kOffV = kOffK + kKStages * kKBytes;
 constexpr int kOffP = kOffV + kVStages * kVBytes;
 constexpr int kSmemBytes = kOffP + kGroups * kQBox;  // one P tile per group (128 queries x 64 keys, bf16)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr uint32_t kColO = 0, kColS = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -92,6 +98,17 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// a * b + c on two fp32 lanes at once (one paired FMA), denormals flushed
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.ftz.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
 }
 
 // q_rot[t][h][0:64] = RoPE(q_rope[t][h], p(t)): one thread per (token, head).
@@ -316,50 +333,58 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
         // ------------------------------------------------------------ TMA producer
         if (n_all > 0 && elect_one()) {
             tma_prefetch(&map_kn);
-            tma_prefetch(&map_v);
+            tma_prefetch(&map_qn);
             const int qrow = b * a.n_q + q0;
             // both query tiles (rows past n_q belong to the next sequence or are zero filled)
             mbar_expect_tx(&q_full, kGroups * 3 * kQBox);
 #pragma unroll
             for (int g = 0; g < kGroups; ++g) {
                 uint8_t* qs = smem + g * 3 * kQBox;
-                tma_load_3d(qs, &map_qn, &q_full, 0, h, qrow + g * kQ);
-                tma_load_3d(qs + kQBox, &map_qn, &q_full, 64, h, qrow + g * kQ);
+                tma_load_4d(qs, &map_qn, &q_full, 0, h, qrow + g * kQ, 0);
                 tma_load_3d(qs + 2 * kQBox, &map_qr, &q_full, 0, h, qrow + g * kQ);
             }
             const int krow = (h * a.B + b) * (int)a.max_len, crow = b * (int)a.capacity;
-            // rows past the sequence are zero (Kn, V) or masked (k_rope); past the
+            // rows past the sequence are zero (Kn) or masked (k_rope); past the
             // tensor they are zero filled
-            int nk = 0, nv = 0;
+            int nk = 0;
             bool ok = true;
             for (int i = 0; ok && i < n_all; ++i) {
-                const int t0 = i * kKeys;
-                const int sk = i % kKStages, sv = i % kVStages;
+                const int sk = i % kKStages;
                 if (i >= kKStages && !mbar_wait(&k_empty[sk], ((i / kKStages) - 1) & 1, abort)) {
                     ok = false;
                     break;
                 }
                 uint8_t* kt = smem + kOffK + sk * kKBytes;
                 mbar_expect_tx(&k_full[sk], kKBytes);
-                tma_load_2d(kt, &map_kn, &k_full[sk], 0, krow + t0);
-                tma_load_2d(kt + kBox, &map_kn, &k_full[sk], 64, krow + t0);
-                tma_load_2d(kt + 2 * kBox, &map_kr, &k_full[sk], 512, crow + t0);
+                tma_load_3d(kt, &map_kn, &k_full[sk], 0, krow + i * kKeys, 0);
+                tma_load_2d(kt + 2 * kBox, &map_kr, &k_full[sk], 512, crow + i * kKeys);
                 ++nk;
-                if (i >= kVStages && !mbar_wait(&v_empty[sv], ((i / kVStages) - 1) & 1, abort)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* vt = smem + kOffV + sv * kVBytes;
-                mbar_expect_tx(&v_full[sv], kVBytes);
-                tma_load_2d(vt, &map_v, &v_full[sv], 0, krow + t0);
-                tma_load_2d(vt + kBox, &map_v, &v_full[sv], 64, krow + t0);
-                ++nv;
             }
             if (!ok) fail();
             // no copy of this CTA may still be in flight when it exits
             mbar_wait(&q_full, 0, nullptr);
             for (int k = nk > kKStages ? nk - kKStages : 0; k < nk; ++k)
                 mbar_wait(&k_full[k % kKStages], (k / kKStages) & 1, nullptr);
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ TMA producer, values
+        if (n_all > 0 && elect_one()) {
+            tma_prefetch(&map_v);
+            const int krow = (h * a.B + b) * (int)a.max_len;
+            int nv = 0;
+            bool ok = true;
+            for (int i = 0; ok && i < n_all; ++i) {
+                const int sv = i % kVStages;
+                if (i >= kVStages && !mbar_wait(&v_empty[sv], ((i / kVStages) - 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* vt = smem + kOffV + sv * kVBytes;
+                mbar_expect_tx(&v_full[sv], kVBytes);
+                tma_load_3d(vt, &map_v, &v_full[sv], 0, krow + i * kKeys, 0);
+                ++nv;
+            }
+            if (!ok) fail();
             for (int k = nv > kVStages ? nv - kVStages : 0; k < nv; ++k)
                 mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1, nullptr);
         }
@@ -443,27 +468,41 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 const int sb = i & 1;
                 if (!(ok = wait_w(&s_full[g][sb], (i >> 1) & 1))) break;
                 tc_fence_after();
-                // The score row is read twice from TMEM (maximum, then exponentials), so
-                // only 32 scores are live at a time; the causal mask is a select, so
-                // whatever lies past the sequence never leaks in.
-                const int64_t key0 = (int64_t)i * kKeys;
-                const bool masked = key0 + kKeys - 1 > p;
-                float mx = -INFINITY;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem + lane_off + colS + 64 * sb + 32 * half, rr);
+                // The score row is read once; the score buffer is free for the GEMM two
+                // tiles later as soon as it is in registers.
+                float x[kKeys];
+                {
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tmem + lane_off + colS + 64 * sb, r0);
+                    tmem_ld32(tmem + lane_off + colS + 64 * sb + 32, r1);
                     tmem_wait_ld();
-                    float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                     for (int k = 0; k < 32; ++k) {
-                        float v = __uint_as_float(rr[k]);
-                        if (masked && key0 + 32 * half + k > p) v = -INFINITY;
-                        m4[k & 3] = fmaxf(m4[k & 3], v);
+                        x[k] = __uint_as_float(r0[k]);
+                        x[32 + k] = __uint_as_float(r1[k]);
                     }
-                    mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
                 }
-                mx *= a.scale_log2;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_free[g][sb]);
+                // Causal mask: keys past the row's position become -inf (a select, so
+                // whatever lies past the sequence never leaks in).  Warp-uniform: a warp
+                // takes the masked path if any of its rows needs it.
+                const int64_t key0 = (int64_t)i * kKeys;
+                const bool masked = __any_sync(0xffffffffu, key0 + kKeys - 1 > p);
+                if (masked) {
+                    const int lim = (int)max((int64_t)-1, min((int64_t)kKeys, p - key0));   // last visible column
+#pragma unroll
+                    for (int n = 0; n < kKeys; ++n) x[n] = n > lim ? -INFINITY : x[n];
+                }
+                float m8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    m8[k] = fmaxf(fmaxf(fmaxf(x[k], x[k + 8]), fmaxf(x[k + 16], x[k + 24])),
+                                  fmaxf(fmaxf(x[k + 32], x[k + 40]), fmaxf(x[k + 48], x[k + 56])));
+                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) *
+                                 a.scale_log2;
                 // the maximum moves only when it grew by more than 2^8 (-inf + 8 is -inf)
                 const float m = mx > m_used + kRescaleThreshold ? mx : m_used;
                 // the P tile and O are free once the group's O GEMM i - 1 is done
@@ -489,35 +528,41 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 }
                 if (need) l *= ex2(m_used - m);
                 m_used = m;
-                const bool live = m_used != -INFINITY;      // a row with no visible key yet (or none at all)
                 const uint32_t prow = sbase + kOffP + g * kQBox + r * 128;
                 float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (!masked) {
+                    // every key of the tile is visible to every row of this warp (so the
+                    // maximum is finite): p = 2^(s * scale - m), two at a time
+                    const float2 sc = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_used, -m_used);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t rr[32];
-                    tmem_ld32(tmem + lane_off + colS + 64 * sb + 32 * half, rr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 8; ++c) {
                         uint32_t pw[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const int n = 8 * c + 2 * k;            // column within the half
-                            const bool v0 = live && !(masked && key0 + 32 * half + n > p);
-                            const bool v1 = live && !(masked && key0 + 32 * half + n + 1 > p);
-                            const float p0 = v0 ? ex2(fmaf(__uint_as_float(rr[n]), a.scale_log2, -m_used)) : 0.f;
-                            const float p1 = v1 ? ex2(fmaf(__uint_as_float(rr[n + 1]), a.scale_log2, -m_used)) : 0.f;
+                            const float2 y = ffma2(make_float2(x[8 * c + 2 * k], x[8 * c + 2 * k + 1]), sc, nm);
+                            const float p0 = ex2(y.x), p1 = ex2(y.y);
                             ps4[k] += p0 + p1;
                             pw[k] = pack_bf16(p0, p1);
                         }
-                        const int chunk = 4 * half + c;
-                        st_shared_u4(prow + ((chunk ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                        st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
+                    }
+                } else {
+                    // masked keys are -inf (p = 0); a row with no visible key yet keeps P = 0
+                    const bool live = m_used != -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t pw[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int n = 8 * c + 2 * k;
+                            const float p0 = live ? ex2(fmaf(x[n], a.scale_log2, -m_used)) : 0.f;
+                            const float p1 = live ? ex2(fmaf(x[n + 1], a.scale_log2, -m_used)) : 0.f;
+                            ps4[k] += p0 + p1;
+                            pw[k] = pack_bf16(p0, p1);
+                        }
+                        st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                     }
                 }
-                // both reads of score buffer sb are done
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[g][sb]);
                 l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
                 fence_async_smem();
                 __syncwarp();
@@ -623,9 +668,11 @@ int prefill_launch(const PrefillCall& c, int* launches) {
     // 3. causal attention
     CUtensorMap mqn, mqr, mkn, mkr, mv;
     {
-        const uint64_t dims[3] = {128, (uint64_t)H, (uint64_t)BJ}, str[2] = {256, (uint64_t)H * 256};
-        const uint32_t box[3] = {64, 1, (uint32_t)kQ};
-        if (!make_map(&mqn, c.q_nope, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        // q_nope [BJ][H][128] as (column in half, head, token, half): one box = 128
+        // tokens of one head, both 64-column halves, landing half-major
+        const uint64_t dims[4] = {64, (uint64_t)H, (uint64_t)BJ, 2}, str[3] = {256, (uint64_t)H * 256, 128};
+        const uint32_t box[4] = {64, 1, (uint32_t)kQ, 2};
+        if (!make_map(&mqn, c.q_nope, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
         const uint64_t dims[3] = {64, (uint64_t)H, (uint64_t)BJ}, str[2] = {128, (uint64_t)H * 128};
@@ -633,11 +680,12 @@ int prefill_launch(const PrefillCall& c, int* launches) {
         if (!make_map(&mqr, q_rot, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
-        // head-major rows: (h * B + b) * max_len + t
-        const uint64_t dims[2] = {128, (uint64_t)H * B * c.max_len}, str[1] = {256};
-        const uint32_t box[2] = {64, (uint32_t)kKeys};
-        if (!make_map(&mkn, kn, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
-        if (!make_map(&mv, v, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        // head-major rows (h * B + b) * max_len + t, as (column in half, row, half):
+        // one box = 64 rows, both halves, landing half-major
+        const uint64_t dims[3] = {64, (uint64_t)H * B * c.max_len, 2}, str[2] = {256, 128};
+        const uint32_t box[3] = {64, (uint32_t)kKeys, 2};
+        if (!make_map(&mkn, kn, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
+        if (!make_map(&mv, v, 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B)) return MLA_ERR_CUDA;
     }
     {
         const uint64_t dims[2] = {576, (uint64_t)B * c.capacity}, str[1] = {576 * 2};
