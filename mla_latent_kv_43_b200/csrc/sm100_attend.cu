@@ -162,6 +162,26 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// a * b + c and a + b on two fp32 lanes at once (paired instructions), denormals flushed
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.ftz.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // kSparse: the key tiles are gathered rows (tile::gather4 from 2-D maps over
 // [batch * capacity][576]); otherwise 64 consecutive keys (3-D maps).
 template <bool kSparse>
@@ -509,22 +529,20 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 // my raw partial scores rounded to fp16, stored straight into the peer's
                 // buffer (the peer adds exactly these values; so do I)
                 const uint32_t row = xin_peer + xb * kTileBytes + h * 128;
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_off + kColS + 64 * sb, r0);
+                tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32 * half, r);
-                    tmem_wait_ld();
+                for (int chunk = 0; chunk < 8; ++chunk) {
+                    const uint32_t* r = chunk < 4 ? r0 + 8 * chunk : r1 + 8 * (chunk - 4);
+                    uint32_t hw[4];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t hw[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            __half2 v = __floats2half2_rn(__uint_as_float(r[8 * c + 2 * i]), __uint_as_float(r[8 * c + 2 * i + 1]));
-                            hw[i] = *reinterpret_cast<uint32_t*>(&v);
-                        }
-                        const int chunk = 4 * half + c;
-                        st_async_u4(row + ((chunk ^ (h & 7)) << 4), hw[0], hw[1], hw[2], hw[3], xbar_peer[xb]);
+                    for (int i = 0; i < 4; ++i) {
+                        __half2 v = __floats2half2_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                        hw[i] = *reinterpret_cast<uint32_t*>(&v);
                     }
+                    st_async_u4(row + ((chunk ^ (h & 7)) << 4), hw[0], hw[1], hw[2], hw[3], xbar_peer[xb]);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -586,15 +604,15 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                 tc_fence_after();
                 float x[64];
                 {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, r);
+                    uint32_t r0[32], r1[32];
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb, r0);
+                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r1);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
-                    tmem_ld32(tmem + lane_off + kColS + 64 * sb + 32, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < 32; ++i) {
+                        x[i] = __uint_as_float(r0[i]);
+                        x[32 + i] = __uint_as_float(r1[i]);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -607,8 +625,9 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const float2 b2 = __half22float2(*reinterpret_cast<const __half2*>(&pw[i]));
-                        x[8 * c + 2 * i] += b2.x;
-                        x[8 * c + 2 * i + 1] += b2.y;
+                        const float2 s2 = fadd2(make_float2(x[8 * c + 2 * i], x[8 * c + 2 * i + 1]), b2);
+                        x[8 * c + 2 * i] = s2.x;
+                        x[8 * c + 2 * i + 1] = s2.y;
                     }
                 }
                 if (valid < kKeys) {
@@ -673,13 +692,15 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
                     }
                 }
                 float ps4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m, -m);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t pw[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const float p0 = ex2(fmaf(x[8 * c + 2 * i], a.scale_log2, -m));
-                        const float p1 = ex2(fmaf(x[8 * c + 2 * i + 1], a.scale_log2, -m));
+                        const float2 y = ffma2(make_float2(x[8 * c + 2 * i], x[8 * c + 2 * i + 1]), sc2, nm2);
+                        const float p0 = ex2(y.x);
+                        const float p1 = ex2(y.y);
                         ps4[i] += p0 + p1;
                         pw[i] = pack_bf16(p0, p1);
                     }
