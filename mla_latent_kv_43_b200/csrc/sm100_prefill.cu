@@ -30,23 +30,33 @@
 // past the row's position (only in warps whose rows reach the diagonal; the
 // others take a select-free path with paired FMAs), keep a base-2 running maximum that
 // moves only when it grows by more than 2^8 (O and the row sum are rescaled
-// then) and write P as bf16 into the group's shared-memory tile;
-// O += P V (M 128, N 128, K 64) with V read MN-major.  Keys and values have
-// rings of their own: a key tile is released when its last score GEMM
-// completes, a value tile when its last value GEMM does.  The grid runs head
+// then) and write P as bf16 over the first 32 columns of the very score
+// buffer they read; O += P V (M 128, N 128, K 64) takes P from TMEM (A
+// operand) and V MN-major from shared memory, and its completion frees the
+// score buffer.  P is thus double-buffered with the scores: a group's softmax
+// of tile i waits for the value GEMM of tile i - 1 only when O must be
+// rescaled.  Keys and values have rings of their own (three tiles each): a key
+// tile is released when its last score GEMM completes, a value tile when its
+// last value GEMM does.  The grid runs head
 // by head (the query tiles of one head, longest first, then the next head),
 // so the CTAs in flight share a few heads' keys and values in L2.  The MMA
 // warp issues both groups' score GEMMs of tile i, then their value GEMMs of
 // tile i - 1, so one group's softmax runs while the tensor core works for the
 // other.
-// Roles (352 threads): warp 0 TMA for the queries and keys, warp 10 TMA for
+// Roles (384 threads): warp 0 TMA for the queries and keys, warp 10 TMA for
 // the values (so a key load never waits behind a value buffer's release),
-// warp 1 MMA issue, warps 2-5 softmax of group 0, warps 6-9 of group 1.
+// warp 1 issues the score GEMMs, warp 11 the value GEMMs, warps 2-5 softmax
+// of group 0, warps 6-9 of group 1.  With one issuer, the value GEMM of a
+// tile whose P was ready waited about a microsecond behind the issue of the
+// next score GEMMs (an issuing thread stalls while the tensor pipe is full),
+// and the score GEMM two tiles later waits for that value GEMM; two issuers
+// keep that chain short.  The tensor pipe runs both warps' GEMMs in arrival
+// order, and each warp's commits track its own GEMMs.
 // Each key or value tile arrives in one tensor copy (both 64-column halves
 // of its 128-wide rows, viewed as two groups of stride 128 bytes), the rope
 // key in a second one.
 // TMEM: O of group g at [128 g, 128 g + 128), S double buffers at
-// [256 + 128 g, 256 + 128 g + 128).
+// [256 + 128 g, 256 + 128 g + 128) (P over the first half of each).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -64,16 +74,15 @@ namespace {
 constexpr int kQ = 128;                            // queries per group
 constexpr int kGroups = 2;                         // query groups per CTA
 constexpr int kKeys = 64;                          // keys per tile
-constexpr int kKStages = 2, kVStages = 2;
+constexpr int kKStages = 3, kVStages = 3;
 constexpr int kBox = 8192;                         // 64 rows x 128 B
 constexpr int kQBox = 16384;                       // 128 rows x 128 B
 constexpr int kOffK = kGroups * 3 * kQBox;         // Q per group: q_nope[0:64], q_nope[64:128], q_rot
 constexpr int kKBytes = 3 * kBox;                  // key tile: Kn[0:64], Kn[64:128], k_rope
 constexpr int kVBytes = 2 * kBox;                  // value tile: V[0:64], V[64:128]
 constexpr int kOffV = kOffK + kKStages * kKBytes;
-constexpr int kOffP = kOffV + kVStages * kVBytes;
-constexpr int kSmemBytes = kOffP + kGroups * kQBox;  // one P tile per group (128 queries x 64 keys, bf16)
-constexpr int kThreads = 352;
+constexpr int kSmemBytes = kOffV + kVStages * kVBytes;
+constexpr int kThreads = 384;
 constexpr uint32_t kColO = 0, kColS = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -96,9 +105,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
 
 // a * b + c on two fp32 lanes at once (one paired FMA), denormals flushed
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
@@ -260,12 +266,15 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                       const __grid_constant__ CUtensorMap map_v, PrefillArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // Per group g: s_full/s_free[g][b] guard score buffer b, p_full[g] the P
-    // tile, o_done[g][t & 1] completes when O GEMM t of the group is done.
-    // Every waiter sees each completion of a barrier in order, so a parity
-    // names exactly one completion.
+    // Per group g and buffer b: s_full[g][b] the score GEMM into buffer b is
+    // done, p_full[g][b] its P is written over it, s_free[g][b] the value GEMM
+    // that read that P is done (the buffer may take the next score GEMM);
+    // o_done[g][t & 1] completes when O GEMM t of the group is done.  A tile's
+    // barrier of buffer b is two completions after the previous one of the same
+    // buffer and cannot run ahead of it, so a parity names exactly one completion.
     __shared__ uint64_t q_full, k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-    __shared__ uint64_t s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups], o_done[kGroups][2], drain;
+    __shared__ uint64_t s_full[kGroups][2], s_free[kGroups][2], p_full[kGroups][2], o_done[kGroups][2], drain,
+        drain_o;
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
 
@@ -299,12 +308,13 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
         for (int g = 0; g < kGroups; ++g) {
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&s_full[g][i], 1);
-                mbar_init(&s_free[g][i], 4);   // the group's four softmax warps have read the score tile
+                mbar_init(&s_free[g][i], 1);   // committed after the value GEMM that read buffer i
                 mbar_init(&o_done[g][i], 1);
+                mbar_init(&p_full[g][i], 4);   // the group's four softmax warps have written P
             }
-            mbar_init(&p_full[g], 4);          // ... have written their P rows
         }
         mbar_init(&drain, 1);
+        mbar_init(&drain_o, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -389,33 +399,13 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 mbar_wait(&v_full[k % kVStages], (k / kVStages) & 1, nullptr);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // Per key tile i: the score GEMMs of both groups, then the value GEMMs
-        // of tile i - 1, so each group's softmax overlaps the other's GEMMs.
+        // ------------------------------------------------------------ score GEMM issuer
+        // Per key tile i: the score GEMMs of both groups, each into its buffer
+        // i & 1 once the value GEMM that read that buffer (tile i - 2) is done.
         if (n_all > 0) {
             constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
-            constexpr uint32_t idO = idesc_bf16(128, 128, false, true);
             const uint64_t dQ = sdesc(sbase, 16, 1024, kSwizzle128);                   // K-major
             const uint64_t dK = sdesc(sbase + kOffK, 16, 1024, kSwizzle128);           // K-major
-            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);         // MN-major
-            const uint64_t dP = sdesc(sbase + kOffP, 16, 1024, kSwizzle128);           // K-major
-            auto issue_o = [&](int t) -> bool {
-                const int sv = t % kVStages;
-                if (!wait_w(&v_full[sv], (t / kVStages) & 1)) return false;
-#pragma unroll
-                for (int g = 0; g < kGroups; ++g) {
-                    if (t >= (g == 0 ? n_g0 : n_g1)) continue;
-                    if (!wait_w(&p_full[g], t & 1)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss_w(tmem + kColO + 128 * g, sdesc_add(dP, g * kQBox + ks * 32),
-                                 sdesc_add(dV, sv * kVBytes + ks * 2048), idO, (t | ks) ? 1u : 0u);
-                    mma_commit_w(&o_done[g][t & 1]);
-                }
-                mma_commit_w(&v_empty[sv]);
-                return true;
-            };
             bool ok = wait_w(&q_full, 0);
             for (int i = 0; ok && i < n_all; ++i) {
                 const int sk = i % kKStages, sb = i & 1;
@@ -436,12 +426,43 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 }
                 if (!ok) break;
                 mma_commit_w(&k_empty[sk]);
-                if (i >= 1) ok = issue_o(i - 1);
             }
-            if (ok) ok = issue_o(n_all - 1);
             if (!ok && lane == 0) fail();
             mma_commit_w(&drain);
             if (lane == 0) mbar_wait(&drain, 0, nullptr);
+            __syncwarp();
+        }
+    } else if (warp == 11) {
+        // ------------------------------------------------------------ value GEMM issuer
+        // Per key tile t and group: O += P V as soon as the group's P and the
+        // value tile are in; the commit frees the score buffer that held P.
+        if (n_all > 0) {
+            constexpr uint32_t idO = idesc_bf16(128, 128, false, true);
+            const uint64_t dV = sdesc(sbase + kOffV, kBox, 1024, kSwizzle128);         // MN-major
+            bool ok = true;
+            for (int t = 0; ok && t < n_all; ++t) {
+                const int sv = t % kVStages;
+                if (!(ok = wait_w(&v_full[sv], (t / kVStages) & 1))) break;
+#pragma unroll
+                for (int g = 0; g < kGroups; ++g) {
+                    if (!ok || t >= (g == 0 ? n_g0 : n_g1)) continue;
+                    if (!(ok = wait_w(&p_full[g][t & 1], (t >> 1) & 1))) break;
+                    tc_fence_after();
+                    // A = P in TMEM (bf16 pairs, 8 columns per 16 keys)
+                    const uint32_t aP = tmem + kColS + 128 * g + 64 * (t & 1);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ts_w(tmem + kColO + 128 * g, aP + 8 * ks, sdesc_add(dV, sv * kVBytes + ks * 2048), idO,
+                                 (t | ks) ? 1u : 0u);
+                    mma_commit_w(&o_done[g][t & 1]);
+                    mma_commit_w(&s_free[g][t & 1]);
+                }
+                if (!ok) break;
+                mma_commit_w(&v_empty[sv]);
+            }
+            if (!ok && lane == 0) fail();
+            mma_commit_w(&drain_o);
+            if (lane == 0) mbar_wait(&drain_o, 0, nullptr);
             __syncwarp();
         }
     } else {
@@ -482,9 +503,6 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                         x[32 + k] = __uint_as_float(r1[k]);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_free[g][sb]);
                 // Causal mask: keys past the row's position become -inf (a select, so
                 // whatever lies past the sequence never leaks in).  Warp-uniform: a warp
                 // takes the masked path if any of its rows needs it.
@@ -505,12 +523,12 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                                  a.scale_log2;
                 // the maximum moves only when it grew by more than 2^8 (-inf + 8 is -inf)
                 const float m = mx > m_used + kRescaleThreshold ? mx : m_used;
-                // the P tile and O are free once the group's O GEMM i - 1 is done
-                if (i >= 1 && !(ok = wait_w(&o_done[g][(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
-                // O holds tiles 0 .. i - 1 relative to m_used: rescale it when m moved.
-                // TMEM accesses are warp-collective, so lanes that need none multiply by 1.
+                // O holds tiles 0 .. i - 1 relative to m_used: rescale it when m moved,
+                // once the group's O GEMM i - 1 is done.  TMEM accesses are
+                // warp-collective, so lanes that need none multiply by 1.
                 const bool need = m_used != -INFINITY && m > m_used;
                 if (__any_sync(0xffffffffu, need)) {
+                    if (i >= 1 && !(ok = wait_w(&o_done[g][(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
                     tc_fence_after();
                     const float alpha = need ? ex2(m_used - m) : 1.f;
 #pragma unroll 1
@@ -528,7 +546,8 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                 }
                 if (need) l *= ex2(m_used - m);
                 m_used = m;
-                const uint32_t prow = sbase + kOffP + g * kQBox + r * 128;
+                // P (bf16 pairs of consecutive keys) for the first 32 columns of the buffer
+                uint32_t pa[16], pb[16];
                 float ps4[4] = {0.f, 0.f, 0.f, 0.f};
                 if (!masked) {
                     // every key of the tile is visible to every row of this warp (so the
@@ -536,37 +555,37 @@ prefill_attend_kernel(const __grid_constant__ CUtensorMap map_qn, const __grid_c
                     const float2 sc = make_float2(a.scale_log2, a.scale_log2), nm = make_float2(-m_used, -m_used);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        uint32_t pw[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const float2 y = ffma2(make_float2(x[8 * c + 2 * k], x[8 * c + 2 * k + 1]), sc, nm);
                             const float p0 = ex2(y.x), p1 = ex2(y.y);
                             ps4[k] += p0 + p1;
-                            pw[k] = pack_bf16(p0, p1);
+                            (c < 4 ? pa : pb)[4 * (c & 3) + k] = pack_bf16(p0, p1);
                         }
-                        st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                     }
                 } else {
                     // masked keys are -inf (p = 0); a row with no visible key yet keeps P = 0
                     const bool live = m_used != -INFINITY;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        uint32_t pw[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int n = 8 * c + 2 * k;
                             const float p0 = live ? ex2(fmaf(x[n], a.scale_log2, -m_used)) : 0.f;
                             const float p1 = live ? ex2(fmaf(x[n + 1], a.scale_log2, -m_used)) : 0.f;
                             ps4[k] += p0 + p1;
-                            pw[k] = pack_bf16(p0, p1);
+                            (c < 4 ? pa : pb)[4 * (c & 3) + k] = pack_bf16(p0, p1);
                         }
-                        st_shared_u4(prow + ((c ^ (r & 7)) << 4), pw[0], pw[1], pw[2], pw[3]);
                     }
                 }
                 l += (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]);
-                fence_async_smem();
+                // the whole score row is in registers, so P may overwrite it
+                tmem_st16(tmem + lane_off + colS + 64 * sb, pa);
+                tmem_st16(tmem + lane_off + colS + 64 * sb + 16, pb);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[g]);
+                if (lane == 0) mbar_arrive(&p_full[g][sb]);
             }
             // every O GEMM of the group is done once its last one is
             if (ok) ok = wait_w(&o_done[g][(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
