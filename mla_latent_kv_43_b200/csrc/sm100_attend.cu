@@ -30,10 +30,11 @@
 // [384,512) (A operand of the score GEMM); the 32 rope columns of Q are an
 // smem operand.
 //
-// Roles (448 threads): warp 0 TMA, warp 1 MMA issue, warps 2-5 "exchange"
-// (score tile -> fp16 -> peer smem, query loads; thread <-> head <-> TMEM lane),
-// warps 6-13 "softmax" (P, O rescale, epilogue): two groups of four warps that
-// take alternate tiles, one thread per head row.
+// Roles (480 threads): warp 0 TMA, warp 1 score-GEMM issue, warp 14
+// latent-GEMM issue, warps 2-5 "exchange" (score tile -> fp16 -> peer smem,
+// query loads; thread <-> head <-> TMEM lane), warps 6-13 "softmax" (P, O
+// rescale, epilogue): two groups of four warps that take alternate tiles, one
+// thread per head row.
 //
 // Work items.  The key tiles of all query tokens are concatenated and cut
 // into one contiguous range per cluster.  A token whose tiles all fall in one
@@ -65,7 +66,7 @@ constexpr int kXBufs = 3;                          // exchange buffers
 constexpr int kOffXin = kStages * kStageBytes;     // the peer's partial scores, then P
 constexpr int kOffQr = kOffXin + kXBufs * kTileBytes;  // 128 heads x 32 rope columns, SW64
 constexpr int kSmemBytes = kOffQr + 128 * 64;
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -194,7 +195,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
     // q0_full: the first item's query slice has landed (tensor copies into
     // stages 2-3 and the Q-rope area); q0_copied: its latent part is in TMEM
     // (tcgen05.cp), so stages 2-3 may take cache tiles
-    __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, q0_full, q0_copied, drain;
+    __shared__ uint64_t s_full[2], s_free[2], o_done[2], q_ready, q0_full, q0_copied, drain, drain_o;
     __shared__ uint64_t p_ready[kXBufs], xin_full[kXBufs], rx_done[kXBufs];
     __shared__ uint32_t tmem_base;
     __shared__ int abort_flag;
@@ -244,6 +245,7 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         }
         mbar_init(&item_done, 1);           // committed after each item's last O GEMM
         mbar_init(&drain, 1);
+        mbar_init(&drain_o, 1);
         abort_flag = 0;
         fence_mbar_init();
     }
@@ -352,56 +354,34 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
             for (uint32_t i = first; i < it; ++i) mbar_wait(&full[i % kStages], (i / kStages) & 1, nullptr);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // Two streams in tile order: score GEMMs S(g) and latent GEMMs O(g).
-        // Each is issued as soon as its inputs are ready, so S runs ahead of O
-        // as far as the two S buffers allow.  The whole warp runs this loop
-        // (every decision is lane 0's observation, broadcast) and one elected
-        // lane issues each instruction.
+        // ------------------------------------------------------------ score GEMM issuer
+        // Score GEMMs S(g) in tile order, each as soon as its stage has landed
+        // and its score buffer is free (and, at an item's start, the item's
+        // query slice is in TMEM).  The latent GEMMs O(g) come from warp 14: an
+        // issuing thread stalls while the tensor pipe is full, so one issuer for
+        // both streams held a ready O(g) behind the next score batch.  The tensor
+        // pipe runs both warps' GEMMs in arrival order; each warp's commits track
+        // its own.  The whole warp runs this loop (every decision is lane 0's
+        // observation, broadcast) and one elected lane issues each instruction.
         constexpr uint32_t idS = idesc_bf16(128, 64, false, false);
-        constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
         // descriptors of stage 0 / P buffer 0; other stages and steps are byte offsets
         const uint64_t dLatK = sdesc(sbase, 16, 1024, kSwizzle128);          // cache tile, K-major (score)
-        const uint64_t dLatN = sdesc(sbase, kLatBox, 1024, kSwizzle128);     // cache tile, MN-major (latent)
         const uint64_t dRope = sdesc(sbase + 4 * kLatBox, 16, 512, kSwizzle64);
         const uint64_t dQr = sdesc(sbase + kOffQr, 16, 512, kSwizzle64);
-        const uint64_t dP = sdesc(sbase + kOffXin, 16, 1024, kSwizzle128);
-        ItemIter iterS, iterO;
+        ItemIter iterS;
         iterS.init(a, pair);
-        iterO.init(a, pair);
-        Item itS, itO;
-        bool haveS = iterS.next(itS), haveO = iterO.next(itO);
-        int kS = 0, kO = 0;
-        uint32_t gS = 0, gO = 0, nItemsS = 0;
+        Item itS;
+        bool haveS = iterS.next(itS);
+        int kS = 0;
+        uint32_t gS = 0, nItemsS = 0;
         bool qS = false;                           // q_ready observed for the current S item
         uint32_t idle = 0;                         // consecutive passes without progress
         uint64_t t_idle = 0;                       // timer at the 256th of them
         bool ok = true;
-        while (ok && haveO) {
+        while (ok && haveS) {
             bool progressed = false;
-            // O GEMMs first: they release the stage and unblock the softmax two tiles later
-            if (gO < gS && mbar_ready_w(&p_ready[gO % kXBufs], (gO / kXBufs) & 1)) {
-                tc_fence_after();
-                const int s = gO % kStages;
-                const uint32_t so = s * kStageBytes, po = (gO % kXBufs) * kTileBytes;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_ss_w(tmem + kColO, sdesc_add(dP, po + ks * 32), sdesc_add(dLatN, so + ks * 2048), idO,
-                             (kO == 0 && ks == 0) ? 0u : 1u);
-                mma_commit_w(&empty[s]);
-                mma_commit_w(&o_done[gO & 1]);
-                // P buffer gO % 3 is free again: the peer may send its tile gO + 3 into it
-                mma_commit_mc_w(&rx_done[gO % kXBufs], (uint16_t)(1u << peer));
-                ++gO;
-                if (++kO == itO.t1 - itO.t0) {
-                    mma_commit_w(&item_done);
-                    kO = 0;
-                    haveO = iterO.next(itO);
-                }
-                progressed = true;
-            }
             // score GEMM S(gS): 16 K-steps of latent (A = query slice in TMEM), 2 of rope
-            if (haveS) {
+            {
                 const int s = gS % kStages, sb = gS & 1;
                 if (!qS && nItemsS == 0 && mbar_ready_w(&q0_full, 0)) {
                     // the first item's latent query slice: stages 2-3 -> TMEM (A operand
@@ -454,6 +434,59 @@ attend_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant
         if (!ok && lane == 0) fail();
         mma_commit_w(&drain);
         mbar_wait(&drain, 0, nullptr);
+    } else if (warp == 14) {
+        // ------------------------------------------------------------ latent GEMM issuer
+        // O(g) += P(g) V(g) in tile order, each as soon as its P tile is written
+        // (P(g) implies S(g) was issued).  The commits release the cache stage,
+        // tell the softmax O(g) is done, hand the exchange buffer back to the
+        // peer and, after an item's last tile, signal item_done.
+        constexpr uint32_t idO = idesc_bf16(128, 256, false, true);
+        const uint64_t dLatN = sdesc(sbase, kLatBox, 1024, kSwizzle128);     // cache tile, MN-major (latent)
+        const uint64_t dP = sdesc(sbase + kOffXin, 16, 1024, kSwizzle128);
+        ItemIter iterO;
+        iterO.init(a, pair);
+        Item itO;
+        bool haveO = iterO.next(itO);
+        int kO = 0;
+        uint32_t gO = 0;
+        uint32_t idle = 0;                         // consecutive passes without progress
+        uint64_t t_idle = 0;                       // timer at the 256th of them
+        bool ok = true;
+        while (ok && haveO) {
+            bool progressed = false;
+            if (mbar_ready_w(&p_ready[gO % kXBufs], (gO / kXBufs) & 1)) {
+                tc_fence_after();
+                const int s = gO % kStages;
+                const uint32_t so = s * kStageBytes, po = (gO % kXBufs) * kTileBytes;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_ss_w(tmem + kColO, sdesc_add(dP, po + ks * 32), sdesc_add(dLatN, so + ks * 2048), idO,
+                             (kO == 0 && ks == 0) ? 0u : 1u);
+                mma_commit_w(&empty[s]);
+                mma_commit_w(&o_done[gO & 1]);
+                // P buffer gO % 3 is free again: the peer may send its tile gO + 3 into it
+                mma_commit_mc_w(&rx_done[gO % kXBufs], (uint16_t)(1u << peer));
+                ++gO;
+                if (++kO == itO.t1 - itO.t0) {
+                    mma_commit_w(&item_done);
+                    kO = 0;
+                    haveO = iterO.next(itO);
+                }
+                progressed = true;
+            }
+            // bounded idle time: the timer is read once per 256 idle passes
+            if (progressed) {
+                idle = 0;
+            } else if ((++idle & 255u) == 0) {
+                const uint64_t now = globaltimer();
+                if (idle == 256) t_idle = now;
+                const int quit = (*abort || now - t_idle > kWaitLimitNs) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, quit, 0)) ok = false;
+            }
+        }
+        if (!ok && lane == 0) fail();
+        mma_commit_w(&drain_o);
+        mbar_wait(&drain_o, 0, nullptr);
     } else if (warp < 6) {
         // ------------------------------------------------------------ exchange warpgroup
         // One leader does every mbarrier wait (bounded) and a named barrier

@@ -1,9 +1,10 @@
 """The barrier protocol of the decode attention kernel (csrc/sm100_attend.cu,
 attend_kernel), modelled on the CPU.
 
-Two CTAs of a cluster, each with its TMA producer, MMA issuer (a polling
-loop, value GEMMs first), exchange warpgroup and two softmax groups of four
-warps taking alternate key tiles, run as coroutines interleaved at random;
+Two CTAs of a cluster, each with its TMA producer, score-GEMM issuer,
+latent-GEMM issuer (two warps feeding one in-order tensor pipe), exchange
+warpgroup and two softmax groups of four warps taking alternate key tiles,
+run as coroutines interleaved at random;
 each CTA's tensor core completes its work in issue order, the copy engine
 (cache loads and the st.async partial-score stores into the peer) in any
 order.  Each mbarrier is a completion counter with expect-tx bytes whose
@@ -118,14 +119,12 @@ def run(items, seed, item_barriers=True, rescale_p=0.3, q0_wait=True):
             engine.append(("load", r, s, g))
             yield "step"
 
-    def mma(r):
+    def mma_o(r):
+        # latent GEMMs in tile order, each once its P tile is written
         c = ctas[r]
-        gS = gO = 0
-        items_s = 0
-        q_ok = False
+        gO = 0
         while gO < G:
-            progressed = False
-            if gO < gS and c.p_ready[gO % XBUFS].passes((gO // XBUFS) & 1):
+            if c.p_ready[gO % XBUFS].passes((gO // XBUFS) & 1):
                 if c.p_ready[gO % XBUFS].completions != gO // XBUFS + 1:
                     raise Hazard("p_ready aliasing")
                 c.tq.append(("O", gO))
@@ -135,24 +134,34 @@ def run(items, seed, item_barriers=True, rescale_p=0.3, q0_wait=True):
                 if item_barriers and (gO + 1 == G or item_of[gO + 1] != item_of[gO]):
                     c.tq.append(("commit", c.item_done))          # the item's last value GEMM
                 gO += 1
+                yield "step"
+            else:
+                yield "blocked"
+
+    def mma_s(r):
+        # score GEMMs in tile order (and the first query slice's copy to TMEM)
+        c = ctas[r]
+        gS = 0
+        items_s = 0
+        q_ok = False
+        while gS < G:
+            progressed = False
+            if not q_ok and items_s == 0 and c.q0_full.passes(0):
+                c.tq.append(("cpQ", 0))                          # stages 2-3 -> TMEM
+                c.tq.append(("commit", c.q0_copied))
+                q_ok = True
+            elif not q_ok and items_s > 0:
+                q_ok = c.q_ready.passes((items_s - 1) & 1)
+            s, sb = gS % STAGES, gS & 1
+            if q_ok and c.full[s].passes((gS // STAGES) & 1) and \
+                    (gS < 2 or c.s_free[sb].passes(((gS >> 1) - 1) & 1)):
+                c.tq.append(("S", gS))
+                c.tq.append(("commit", c.s_full[sb]))
+                gS += 1
+                if gS == G or item_of[gS] != item_of[gS - 1]:
+                    q_ok = False
+                    items_s += 1
                 progressed = True
-            if gS < G:
-                if not q_ok and items_s == 0 and c.q0_full.passes(0):
-                    c.tq.append(("cpQ", 0))                      # stages 2-3 -> TMEM
-                    c.tq.append(("commit", c.q0_copied))
-                    q_ok = True
-                elif not q_ok and items_s > 0:
-                    q_ok = c.q_ready.passes((items_s - 1) & 1)
-                s, sb = gS % STAGES, gS & 1
-                if q_ok and c.full[s].passes((gS // STAGES) & 1) and \
-                        (gS < 2 or c.s_free[sb].passes(((gS >> 1) - 1) & 1)):
-                    c.tq.append(("S", gS))
-                    c.tq.append(("commit", c.s_full[sb]))
-                    gS += 1
-                    if gS == G or item_of[gS] != item_of[gS - 1]:
-                        q_ok = False
-                        items_s += 1
-                    progressed = True
             yield "step" if progressed else "blocked"
 
     def exchange(r):
@@ -231,7 +240,8 @@ def run(items, seed, item_barriers=True, rescale_p=0.3, q0_wait=True):
     roles = {}
     for r in range(2):
         roles[f"tma{r}"] = tma(r)
-        roles[f"mma{r}"] = mma(r)
+        roles[f"mma_s{r}"] = mma_s(r)
+        roles[f"mma_o{r}"] = mma_o(r)
         roles[f"ex{r}"] = exchange(r)
         for grp in range(2):
             for q in range(4):
