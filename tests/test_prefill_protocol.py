@@ -1,22 +1,28 @@
 """The barrier protocol of the prefill attention kernel (csrc/sm100_prefill.cu,
 prefill_attend_kernel), modelled on the CPU.
 
-The roles -- the TMA producer, the MMA issuer, and the four softmax warps of
-each of the two query groups -- run as coroutines interleaved at random; the
-tensor core completes its work in issue order (MMAs, then the commits behind
-them) and the copy engine in any order.  Each mbarrier is a completion
-counter whose parity waits behave as on the device.  Checked for every
+The roles -- the key producer (queries and keys), the value producer, the
+score-GEMM issuer, the value-GEMM issuer, and the four softmax warps of each
+of the two query groups -- run as coroutines interleaved at random; the
+tensor core completes the two issuers' work in arrival order (MMAs, then the
+commits behind them) and the copy engine in any order.  Each mbarrier is a
+completion counter whose parity waits behave as on the device.
+
+Each group's softmax writes P over the first half of the score buffer it
+read; the value GEMM takes P from there and its commit frees the buffer for
+the score GEMM two tiles later, so a softmax waits for the previous value
+GEMM only when it rescales O (drawn at random here).  Checked for every
 interleaving drawn: no wait passes on a completion other than the one it
-names (no phase aliasing), no key, value, score or P buffer is reused before
-its consumer is done, each group's value GEMMs accumulate in order, and the
-whole tile schedule finishes (no deadlock) -- for group lengths that differ,
-that are equal, and with an empty second group.  A change to the kernel's
-waits or commits must be mirrored here."""
+names (no phase aliasing), no key, value or score buffer is reused before its
+consumer is done, P is what a value GEMM reads, each group's value GEMMs
+accumulate in order, and the whole tile schedule finishes (no deadlock) --
+for group lengths that differ, that are equal, and with an empty second
+group.  A change to the kernel's waits or commits must be mirrored here."""
 import random
 
 import pytest
 
-K_STAGES = V_STAGES = 2          # key and value rings
+K_STAGES = V_STAGES = 3          # key and value rings
 GROUPS, WARPS = 2, 4             # query groups per CTA, softmax warps per group
 
 
@@ -41,7 +47,7 @@ def wait(bar, parity, nth):
     assert bar.completions == nth, f"{bar.name}: {bar.completions} completions, the wait names #{nth}"
 
 
-def run_schedule(n_g, seed):
+def run_schedule(n_g, seed, rescale_p=0.3, free_wait=True):
     rng = random.Random(seed)
     n_all = max(n_g)
     q_full = Barrier("q_full")
@@ -50,79 +56,80 @@ def run_schedule(n_g, seed):
     v_full = [Barrier(f"v_full{i}") for i in range(V_STAGES)]
     v_empty = [Barrier(f"v_empty{i}") for i in range(V_STAGES)]
     s_full = [[Barrier(f"s_full{g}{b}") for b in range(2)] for g in range(GROUPS)]
-    s_free = [[Barrier(f"s_free{g}{b}", WARPS) for b in range(2)] for g in range(GROUPS)]
-    p_full = [Barrier(f"p_full{g}", WARPS) for g in range(GROUPS)]
+    s_free = [[Barrier(f"s_free{g}{b}") for b in range(2)] for g in range(GROUPS)]
+    p_full = [[Barrier(f"p_full{g}{b}", WARPS) for b in range(2)] for g in range(GROUPS)]
     o_done = [[Barrier(f"o_done{g}{b}") for b in range(2)] for g in range(GROUPS)]
-    tensor_queue, copies = [], []                    # tensor core in order; copies in any order
+    tensor_queue, copies = [], []                    # tensor core in arrival order; copies in any order
     k_tile, v_tile = [None] * K_STAGES, [None] * V_STAGES
-    s_tile = [[None, None] for _ in range(GROUPS)]   # tile held by each score buffer
-    p_tile = [None] * GROUPS                          # tile held by each group's P buffer
+    # per score buffer and lane quarter (each softmax warp owns 32 rows):
+    # ("S", i), ("P", i) or ("used", i)
+    s_buf = [[[None] * WARPS for _ in range(2)] for _ in range(GROUPS)]
     o_last = [-1] * GROUPS                            # last value GEMM accumulated per group
 
-    def producer():
+    def key_producer():
         copies.append((q_full, None, None))
         for i in range(n_all):
             if i >= K_STAGES:
                 yield from wait(k_empty[i % K_STAGES], ((i // K_STAGES) - 1) & 1, i // K_STAGES)
             copies.append((k_full[i % K_STAGES], ("k", i % K_STAGES), i))
             yield "step"
+
+    def value_producer():
+        for i in range(n_all):
             if i >= V_STAGES:
                 yield from wait(v_empty[i % V_STAGES], ((i // V_STAGES) - 1) & 1, i // V_STAGES)
             copies.append((v_full[i % V_STAGES], ("v", i % V_STAGES), i))
             yield "step"
 
-    def issuer():
+    def score_issuer():
         yield from wait(q_full, 0, 1)
-
-        def value_gemms(t):
-            sv = t % V_STAGES
-            yield from wait(v_full[sv], (t // V_STAGES) & 1, t // V_STAGES + 1)
-            for g in range(GROUPS):
-                if t >= n_g[g]:
-                    continue
-                yield from wait(p_full[g], t & 1, t + 1)
-                tensor_queue.append(("O", g, t, sv))
-                tensor_queue.append(("commit", o_done[g][t & 1]))
-                yield "step"
-            tensor_queue.append(("commit", v_empty[sv]))
-
         for i in range(n_all):
             sk, sb = i % K_STAGES, i & 1
             yield from wait(k_full[sk], (i // K_STAGES) & 1, i // K_STAGES + 1)
             for g in range(GROUPS):
                 if i >= n_g[g]:
                     continue
-                if i >= 2:
+                if i >= 2 and free_wait:              # the value GEMM of tile i - 2 read this buffer
                     yield from wait(s_free[g][sb], ((i >> 1) - 1) & 1, i >> 1)
                 tensor_queue.append(("S", g, i, sk))
                 tensor_queue.append(("commit", s_full[g][sb]))
                 yield "step"
             tensor_queue.append(("commit", k_empty[sk]))
-            if i >= 1:
-                yield from value_gemms(i - 1)
-        yield from value_gemms(n_all - 1)
+
+    def value_issuer():
+        for t in range(n_all):
+            sv = t % V_STAGES
+            yield from wait(v_full[sv], (t // V_STAGES) & 1, t // V_STAGES + 1)
+            for g in range(GROUPS):
+                if t >= n_g[g]:
+                    continue
+                yield from wait(p_full[g][t & 1], (t >> 1) & 1, (t >> 1) + 1)
+                tensor_queue.append(("O", g, t, sv))
+                tensor_queue.append(("commit", o_done[g][t & 1]))
+                tensor_queue.append(("commit", s_free[g][t & 1]))
+                yield "step"
+            tensor_queue.append(("commit", v_empty[sv]))
 
     def softmax(g, warp):
         for i in range(n_g[g]):
             sb = i & 1
             yield from wait(s_full[g][sb], (i >> 1) & 1, (i >> 1) + 1)
-            assert s_tile[g][sb] == i
-            if i >= 1:                                # O and the P tile are free
+            assert s_buf[g][sb][warp] == ("S", i), f"score rows hold {s_buf[g][sb][warp]} at the read of {i}"
+            yield "step"
+            if i >= 1 and rng.random() < rescale_p:     # O rescaled: the previous value GEMM is done
                 yield from wait(o_done[g][(i - 1) & 1], ((i - 1) >> 1) & 1, ((i - 1) >> 1) + 1)
                 assert o_last[g] == i - 1
-            yield "step"
-            assert s_tile[g][sb] == i, "score buffer overwritten before the second read"
-            if warp == 0:
-                p_tile[g] = i
-            s_free[g][sb].arrive()
-            p_full[g].arrive()
+                yield "step"
+            assert s_buf[g][sb][warp] == ("S", i), "score rows overwritten before P replaced them"
+            s_buf[g][sb][warp] = ("P", i)
+            p_full[g][sb].arrive()
             yield "step"
         if n_g[g]:
             last = n_g[g] - 1
             yield from wait(o_done[g][last & 1], (last >> 1) & 1, (last >> 1) + 1)
             assert o_last[g] == last
 
-    roles = {"producer": producer(), "issuer": issuer()}
+    roles = {"kprod": key_producer(), "vprod": value_producer(), "sis": score_issuer(), "ois": value_issuer()}
     roles.update({f"softmax{g}{w}": softmax(g, w) for g in range(GROUPS) for w in range(WARPS)})
     finished, idle = set(), 0
     while len(finished) < len(roles):
@@ -135,12 +142,17 @@ def run_schedule(n_g, seed):
                 if op[0] == "S":
                     _, g, i, sk = op
                     assert k_tile[sk] == i, "key tile replaced before its score GEMM"
-                    s_tile[g][i & 1] = i
+                    for w in range(WARPS):
+                        prev = s_buf[g][i & 1][w]
+                        assert prev is None or prev == ("used", i - 2), f"score GEMM {i} over {prev}"
+                        s_buf[g][i & 1][w] = ("S", i)
                 elif op[0] == "O":
                     _, g, t, sv = op
-                    assert v_tile[sv] == t and p_tile[g] == t, "value or P tile replaced too early"
+                    assert v_tile[sv] == t, "value tile replaced too early"
+                    assert all(x == ("P", t) for x in s_buf[g][t & 1]), f"value GEMM {t} reads {s_buf[g][t & 1]}"
                     assert o_last[g] == t - 1
                     o_last[g] = t
+                    s_buf[g][t & 1] = [("used", t)] * WARPS
                 else:
                     op[1].arrive()
         elif who == "copy":
@@ -164,3 +176,16 @@ def run_schedule(n_g, seed):
 def test_prefill_barrier_protocol(n_g):
     for seed in range(12):
         run_schedule(n_g, seed * 13 + sum(n_g))
+
+
+def test_model_finds_p_overwritten_without_the_buffer_release():
+    """Control: if the score GEMM did not wait for the value GEMM that read P
+    out of its buffer, some interleaving overwrites P before it is read."""
+    found = False
+    for n_g in [(8, 8), (30, 32), (3, 5)]:
+        for seed in range(12):
+            try:
+                run_schedule(n_g, seed * 13 + sum(n_g), free_wait=False)
+            except AssertionError as e:
+                found = found or "over" in str(e) or "reads" in str(e)
+    assert found
