@@ -56,12 +56,17 @@ __device__ __forceinline__ void rope_pair_turn(float x0, float x1, int64_t pos, 
 // (__sincosf, absolute error about 2^-21 on [-pi, pi), far below bf16's 2^-9
 // relative rounding) instead of the correctly reduced sincosf, which costs
 // microseconds per token in the absorb and prefill kernels.
-__device__ __forceinline__ void rope_pair_turn_bf16(float x0, float x1, int64_t pos, uint64_t turn, float* y0,
-                                                    float* y1) {
+// cos and sin of the angle pos * turn (turn: fractions of a full turn, 2^-64 units)
+__device__ __forceinline__ void rope_cos_sin_turn(int64_t pos, uint64_t turn, float* c, float* s) {
     const uint64_t t = (uint64_t)pos * turn;
     const float ang = (float)(int32_t)(uint32_t)(t >> 32) * 1.46291807926715968e-9f;   // 2 pi / 2^32
+    __sincosf(ang, s, c);
+}
+
+__device__ __forceinline__ void rope_pair_turn_bf16(float x0, float x1, int64_t pos, uint64_t turn, float* y0,
+                                                    float* y1) {
     float s, c;
-    __sincosf(ang, &s, &c);
+    rope_cos_sin_turn(pos, turn, &c, &s);
     *y0 = x0 * c - x1 * s;
     *y1 = x0 * s + x1 * c;
 }

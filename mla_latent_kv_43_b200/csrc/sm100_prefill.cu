@@ -117,31 +117,39 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return d;
 }
 
-// q_rot[t][h][0:64] = RoPE(q_rope[t][h], p(t)): one thread per (token, head).
+// q_rot[t][h][0:64] = RoPE(q_rope[t][h], p(t)): one CTA per query token.  The
+// rotation of pair i depends only on the token's position, so the token's 32
+// (cos, sin) pairs are computed once (the same fixed-point angle reduction as
+// the decode path's, so the results are identical) and every head reuses
+// them; the token's H x 64 values then stream through in 16-byte chunks that
+// consecutive threads take in order (coalesced loads and stores).
 __global__ void __launch_bounds__(128) prefill_qrope_kernel(const __nv_bfloat16* __restrict__ q_rope,
                                                             const int32_t* __restrict__ seq_lens, int BJ, int n_q,
                                                             int H, RopeTurns rt, __nv_bfloat16* __restrict__ q_rot) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)BJ * H) return;
-    const int t = (int)(i / H);
+    __shared__ float2 cs[32];
+    const int t = blockIdx.x;
+    if (t >= BJ) return;
     const int b = t / n_q, j = t % n_q;
     const int64_t p = query_pos(seq_lens[b], n_q, j);
-    const uint4* src = reinterpret_cast<const uint4*>(q_rope + i * 64);
-    uint4* dst = reinterpret_cast<uint4*>(q_rot + i * 64);
-    uint4 v[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) v[c] = src[c];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+    if (threadIdx.x < 32) {
+        float c, s;
+        rope_cos_sin_turn(p, rt.turn[threadIdx.x], &c, &s);
+        cs[threadIdx.x] = make_float2(c, s);
+    }
+    __syncthreads();
+    const uint4* src = reinterpret_cast<const uint4*>(q_rope + (int64_t)t * H * 64);
+    uint4* dst = reinterpret_cast<uint4*>(q_rot + (int64_t)t * H * 64);
+    for (int i = threadIdx.x; i < H * 8; i += blockDim.x) {
+        const uint4 v = src[i];
+        const int pair0 = 4 * (i & 7);               // chunk i % 8 of a head row: pairs 4 (i % 8) ..
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[k]));
-            float y0, y1;
-            rope_pair_turn_bf16(x.x, x.y, p, rt.turn[4 * c + k], &y0, &y1);
-            w[k] = pack_bf16(y0, y1);
+            const float2 r = cs[pair0 + k];
+            w[k] = pack_bf16(x.x * r.x - x.y * r.y, x.x * r.y + x.y * r.x);
         }
-        dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -639,10 +647,9 @@ int prefill_launch(const PrefillCall& c, int* launches) {
     RopeTurns rt;
     rope_turn_table(c.d.rope_base, 64, rt.turn);
     {
-        const int64_t n = (int64_t)BJ * H;
         prof_begin(c.stream, "sm100_prefill_qrope");
-        prefill_qrope_kernel<<<(unsigned)((n + 127) / 128), 128, 0, c.stream>>>(
-            (const __nv_bfloat16*)c.q_rope, c.seq_lens, BJ, n_q, H, rt, q_rot);
+        prefill_qrope_kernel<<<(unsigned)BJ, 128, 0, c.stream>>>((const __nv_bfloat16*)c.q_rope, c.seq_lens, BJ, n_q,
+                                                                 H, rt, q_rot);
         prof_end(c.stream);
         ++*launches;
         if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
