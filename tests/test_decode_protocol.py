@@ -344,3 +344,20 @@ def test_model_finds_the_hazards_without_the_item_barriers():
                 msg = str(e)
                 found.add("epilogue" if "epilogue" in msg else "parity" if "completions" in msg else msg)
     assert {"epilogue", "parity"} <= found, found
+
+
+try:
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+except ImportError:          # the fixed shapes above still run
+    given = None
+
+if given is not None:
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(items=st.lists(st.integers(min_value=1, max_value=12), min_size=1, max_size=5),
+           seed=st.integers(min_value=0, max_value=2**31 - 1),
+           rescale_p=st.sampled_from([0.0, 0.3, 1.0]))
+    def test_decode_protocol_random_items(items, seed, rescale_p):
+        """Drawn item lists (1-5 items of 1-12 tiles), interleavings and
+        rescale frequencies: the shipped protocol never hazards or deadlocks."""
+        run(items, seed, rescale_p=rescale_p)

@@ -189,3 +189,23 @@ def test_model_finds_p_overwritten_without_the_buffer_release():
             except AssertionError as e:
                 found = found or "over" in str(e) or "reads" in str(e)
     assert found
+
+
+try:
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+except ImportError:          # the fixed group lengths above still run
+    given = None
+
+if given is not None:
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(g0=st.integers(min_value=1, max_value=20), extra=st.integers(min_value=0, max_value=4),
+           second_empty=st.booleans(), seed=st.integers(min_value=0, max_value=2**31 - 1),
+           rescale_p=st.sampled_from([0.0, 0.3, 1.0]))
+    def test_prefill_protocol_random_lengths(g0, extra, second_empty, seed, rescale_p):
+        """Drawn group lengths (the second group, rows further along the causal
+        diagonal, has at least as many key tiles as the first, or none when its
+        rows lie past the last query), seeds and rescale frequencies: the
+        shipped protocol never hazards or deadlocks."""
+        n_g = (g0, 0) if second_empty else (g0, g0 + extra)
+        run_schedule(n_g, seed, rescale_p=rescale_p)
